@@ -1,0 +1,320 @@
+"""CPU oracle for the SALAD hybrid-attention forward pass (float64, numpy).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The CUDA library
+never calls it and shares no code with it.
+
+Every function restates one step of the method as the SALAD pages give it, in
+float64, with no blocking, fusion or reordering beyond what the step states.
+Sources (page title, then section):
+  * "SALAD ... (paper.rainbus.top)": 前置知识 -- Sparse Attention (mask
+    M in {-inf, 0}^{N x N}), Linear Attention (H = phi(K)^T V, Z = phi(K)^T 1,
+    O = phi(Q) H / (phi(Q) Z), phi = ReLU); 方法步骤详情 steps 2-6 (sparse branch
+    O_s, linear branch O_l, zero-init projection O_l' = ZeroInitProj(O_l),
+    sigmoid gate s, residual O~ = O_s + s * O_l').
+  * "视频扩散模型中的稀疏注意力机制解析 (ijyty.com)": 1.1 (ST-SWA: frame-major
+    flattening, per-head regrouping by spatial position, 1-D sliding window),
+    1.2 (Top-K: block partition, block mean vectors, similarity to key-block
+    means, keep Top-K blocks, attend only to them), 2.3 (gate: token mean ->
+    linear -> sigmoid).
+Readings where the pages are silent (each is listed in the design notes):
+  softmax scale 1/sqrt(d); query side of the selection pooled per query block;
+  block means over valid rows only; no forced blocks; ties broken towards the
+  lower block index; eps = 1e-6 added to the linear-attention denominator;
+  gate s = sigmoid(w . mean_tokens(X) + b) with X already time-modulated;
+  W_lin per head, d x d, right-multiplying row vectors; no 3-D RoPE in the
+  linear branch; space-major order r = (y * Wh + x) * F + f; window
+  |r - c| <= W clipped at the sequence ends.
+
+Parity pins: every function here is checked by ``tests/test_oracle_pins.py``
+against brute force, closed forms, library routines or hand-derived fixtures.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Iterable, List, Optional, Sequence
+
+import numpy as np
+
+__all__ = [
+    "as64", "gate", "block_means", "block_scores", "select_topk",
+    "topk_attention_rows", "topk_attention", "space_major_order",
+    "swa_attention_rows", "swa_attention", "dense_attention",
+    "linear_state", "linear_apply", "combine", "forward",
+    "near_tie_equivalent",
+]
+
+
+def as64(t) -> np.ndarray:
+    """bf16/fp32 torch tensor or array -> float64 numpy array (exact)."""
+    try:
+        import torch
+        if isinstance(t, torch.Tensor):
+            return t.detach().to("cpu").double().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(t, dtype=np.float64)
+
+
+# ----------------------------------------------------------------- gate ----
+def gate(x: np.ndarray, w: np.ndarray, bias: float) -> np.ndarray:
+    """Input-aware scalar gate, one value per batch sample.
+
+    "SALAD ... (paper.rainbus.top)" 方法步骤详情 step 5 and
+    "视频扩散模型中的稀疏注意力机制解析" 2.3: average the hidden state over tokens,
+    apply a linear map, then a sigmoid.  x: [B, N, D]; w: [D]; returns s [B].
+    """
+    x = as64(x)
+    w = as64(w)
+    xbar = x.mean(axis=1)                      # token mean   [B, D]
+    z = xbar @ w + float(bias)                 # linear       [B]
+    return 1.0 / (1.0 + np.exp(-z))            # sigmoid      [B]
+
+
+# ------------------------------------------------------ Top-K selection ----
+def block_means(t: np.ndarray, block: int) -> np.ndarray:
+    """Mean vector of each block of ``block`` consecutive rows (valid rows only).
+
+    "视频扩散模型中的稀疏注意力机制解析" 1.2, step "块划分与均值计算".
+    t: [N, d] -> [nb, d], nb = ceil(N / block); the last block averages the
+    rows it actually holds.
+    """
+    t = as64(t)
+    N = t.shape[0]
+    nb = (N + block - 1) // block
+    out = np.empty((nb, t.shape[1]), np.float64)
+    for i in range(nb):
+        rows = t[i * block:min(N, (i + 1) * block)]
+        out[i] = rows.sum(axis=0) / rows.shape[0]
+    return out
+
+
+def block_scores(q: np.ndarray, k: np.ndarray, block: int) -> np.ndarray:
+    """Similarity of every query-block mean with every key-block mean.
+
+    "视频扩散模型中的稀疏注意力机制解析" 1.2, step "相似度筛选": dot products of
+    block means (unscaled; the ranking does not depend on a scale).
+    q, k: [N, d] -> [nb, nb] with S[i, j] = qbar_i . kbar_j.
+    """
+    return block_means(q, block) @ block_means(k, block).T
+
+
+def select_topk(scores: np.ndarray, topk: int) -> np.ndarray:
+    """For each query block, the ``topk`` key blocks of largest score.
+
+    Order: score descending, then block index ascending (tie rule).  The kept
+    indices are returned in ascending order.  scores: [nb, nb] -> [nb, topk].
+    """
+    nb = scores.shape[1]
+    if not 1 <= topk <= nb:
+        raise ValueError("topk must be in [1, nb]")
+    out = np.empty((scores.shape[0], topk), np.int64)
+    cols = np.arange(nb)
+    for i in range(scores.shape[0]):
+        # np.lexsort sorts by the last key first: (-score) then column index.
+        order = np.lexsort((cols, -scores[i]))
+        out[i] = np.sort(order[:topk])
+    return out
+
+
+def _softmax_attend(q_rows, k_cols, v_cols, extra_mask=None) -> np.ndarray:
+    """softmax(q k^T / sqrt(d) + M) v for a set of rows, max-subtracted."""
+    d = q_rows.shape[1]
+    s = (q_rows @ k_cols.T) / math.sqrt(d)
+    if extra_mask is not None:
+        s = s + extra_mask
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    return (p @ v_cols) / p.sum(axis=1, keepdims=True)
+
+
+def topk_attention_rows(q, k, v, idx, block: int, qblocks: Iterable[int]) -> Dict[int, np.ndarray]:
+    """Top-K block-sparse attention for the listed query blocks of one head.
+
+    "视频扩散模型中的稀疏注意力机制解析" 1.2, step "局部注意力计算": each query
+    token attends only to the tokens of the key blocks selected for its block.
+    q, k, v: [N, d]; idx: [nb, topk].  Returns {i: [rows_i, d]}.
+    """
+    q, k, v = as64(q), as64(k), as64(v)
+    N = q.shape[0]
+    out = {}
+    for i in qblocks:
+        rows = slice(i * block, min(N, (i + 1) * block))
+        cols = np.concatenate([np.arange(j * block, min(N, (j + 1) * block)) for j in idx[i]])
+        out[i] = _softmax_attend(q[rows], k[cols], v[cols])
+    return out
+
+
+def topk_attention(q, k, v, idx, block: int) -> np.ndarray:
+    """Top-K block-sparse attention over all query blocks of one head: [N, d]."""
+    q = as64(q)
+    nb = idx.shape[0]
+    res = topk_attention_rows(q, k, v, idx, block, range(nb))
+    return np.concatenate([res[i] for i in range(nb)], axis=0)
+
+
+# -------------------------------------------------------------- ST-SWA ----
+def space_major_order(F: int, Hh: int, Wh: int) -> np.ndarray:
+    """Token permutation of the spatio-temporal sliding window.
+
+    "视频扩散模型中的稀疏注意力机制解析" 1.1: the latent is flattened with time
+    slowest, t = (f * Hh + y) * Wh + x; heads with temporal locality regroup the
+    tokens by spatial position so that one position's frames are adjacent:
+    r = (y * Wh + x) * F + f.  Returns perm with perm[r] = t.
+    """
+    perm = np.empty(F * Hh * Wh, np.int64)
+    for f in range(F):
+        for y in range(Hh):
+            for x in range(Wh):
+                t = (f * Hh + y) * Wh + x
+                r = (y * Wh + x) * F + f
+                perm[r] = t
+    return perm
+
+
+def swa_attention_rows(q, k, v, window: int, rows: Sequence[int]) -> np.ndarray:
+    """Sliding-window attention for the listed rows of one (already ordered) head.
+
+    Row r attends to every key c with |r - c| <= window, clipped to [0, N).
+    The band is written as the page's additive mask M in {-inf, 0}.
+    """
+    q, k, v = as64(q), as64(k), as64(v)
+    N = q.shape[0]
+    rows = np.asarray(list(rows), np.int64)
+    lo = max(0, int(rows.min()) - window)
+    hi = min(N, int(rows.max()) + window + 1)
+    cols = np.arange(lo, hi)
+    mask = np.where(np.abs(rows[:, None] - cols[None, :]) <= window, 0.0, -np.inf)
+    return _softmax_attend(q[rows], k[cols], v[cols], mask)
+
+
+def swa_attention(q, k, v, window: int, space_major: bool, F: int, Hh: int, Wh: int,
+                  chunk: int = 64) -> np.ndarray:
+    """ST-SWA for one head in frame-major token order: [N, d].
+
+    A space-major head is reordered, attended with the 1-D window, and its
+    output rows are put back at their frame-major positions.
+    """
+    q, k, v = as64(q), as64(k), as64(v)
+    N = q.shape[0]
+    if space_major:
+        perm = space_major_order(F, Hh, Wh)
+        qo, ko, vo = q[perm], k[perm], v[perm]
+    else:
+        qo, ko, vo = q, k, v
+    out_o = np.empty_like(qo)
+    for r0 in range(0, N, chunk):
+        rows = np.arange(r0, min(N, r0 + chunk))
+        out_o[rows] = swa_attention_rows(qo, ko, vo, window, rows)
+    if not space_major:
+        return out_o
+    out = np.empty_like(out_o)
+    out[perm] = out_o
+    return out
+
+
+def dense_attention(q, k, v) -> np.ndarray:
+    """Full softmax attention softmax(Q K^T / sqrt(d)) V for one head."""
+    q, k, v = as64(q), as64(k), as64(v)
+    out = np.empty_like(q)
+    for r0 in range(0, q.shape[0], 256):
+        out[r0:r0 + 256] = _softmax_attend(q[r0:r0 + 256], k, v)
+    return out
+
+
+# ------------------------------------------------------ linear branch -----
+def linear_state(k, v):
+    """H = phi(K)^T V and Z = phi(K)^T 1 with phi = ReLU, for one head.
+
+    "SALAD ... (paper.rainbus.top)" 前置知识 Linear Attention.  k, v: [N, d]
+    -> H [d, d], Z [d].
+    """
+    k, v = as64(k), as64(v)
+    pk = np.maximum(k, 0.0)
+    return pk.T @ v, pk.sum(axis=0)
+
+
+def linear_apply(q, Hst, Z, eps: float) -> np.ndarray:
+    """O_l = phi(Q) H / (phi(Q) Z + eps) for one head: [N, d]."""
+    q = as64(q)
+    pq = np.maximum(q, 0.0)
+    return (pq @ Hst) / ((pq @ Z) + eps)[:, None]
+
+
+# ------------------------------------------------------------ combine -----
+def combine(o_sparse, o_lin, w_lin_h, s: float) -> np.ndarray:
+    """O = O_s + s * (O_l W_lin) for one head (steps 4 and 6 of the method)."""
+    return as64(o_sparse) + float(s) * (as64(o_lin) @ as64(w_lin_h))
+
+
+# ------------------------------------------------------------ forward -----
+def forward(inp: Dict, *, mode: str, block: int = 64, topk: int = 0, window: int = 0,
+            space_major_heads: Sequence[int] = (), F: int = 0, Hh: int = 0, Wh: int = 0,
+            eps: float = 1e-6, gate_override: Optional[float] = None,
+            idx_override: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+    """The whole hybrid layer, in the step order of the method.
+
+    inp: q, k, v [B, H, N, d]; x [B, N, D]; w_gate [D]; bias; w_lin [H, d, d].
+    mode: "topk" | "swa" | "dense".  ``idx_override`` replaces the selection
+    (used when another correct selection is compared at a near tie).
+    Returns s [B], idx [B, H, nb, topk] (topk mode), scores, o_sparse, o_lin, o.
+    """
+    q, k, v = as64(inp["q"]), as64(inp["k"]), as64(inp["v"])
+    B, H, N, d = q.shape
+    s = gate(inp["x"], inp["w_gate"], inp["bias"]) if gate_override is None \
+        else np.full(B, float(gate_override))
+    w_lin = as64(inp["w_lin"])
+    nb = (N + block - 1) // block
+    o_sparse = np.empty_like(q)
+    o_lin = np.empty_like(q)
+    o = np.empty_like(q)
+    idx = np.zeros((B, H, nb, max(topk, 1)), np.int64) if mode == "topk" else None
+    scores = np.zeros((B, H, nb, nb)) if mode == "topk" else None
+    for b in range(B):
+        for h in range(H):
+            if mode == "topk":
+                scores[b, h] = block_scores(q[b, h], k[b, h], block)
+                idx[b, h] = select_topk(scores[b, h], topk) if idx_override is None \
+                    else idx_override[b, h]
+                o_sparse[b, h] = topk_attention(q[b, h], k[b, h], v[b, h], idx[b, h], block)
+            elif mode == "swa":
+                o_sparse[b, h] = swa_attention(q[b, h], k[b, h], v[b, h], window,
+                                               h in space_major_heads, F, Hh, Wh)
+            elif mode == "dense":
+                o_sparse[b, h] = dense_attention(q[b, h], k[b, h], v[b, h])
+            else:
+                raise ValueError(mode)
+            Hst, Z = linear_state(k[b, h], v[b, h])
+            o_lin[b, h] = linear_apply(q[b, h], Hst, Z, eps)
+            o[b, h] = combine(o_sparse[b, h], o_lin[b, h], w_lin[h], s[b])
+    return {"s": s, "idx": idx, "scores": scores, "o_sparse": o_sparse,
+            "o_lin": o_lin, "o": o}
+
+
+# ------------------------------------------------- selection comparison ---
+def near_tie_equivalent(scores_row: np.ndarray, idx_ref: Sequence[int], idx_other: Sequence[int],
+                        rel: float = 1e-5) -> bool:
+    """Whether another kept set is an acceptable answer at a near tie.
+
+    Equal sets always pass.  Otherwise the reference's k-th and (k+1)-th
+    largest scores must lie within ``rel`` (relative) of each other, and every
+    block that differs between the two sets must score within that band.
+    """
+    a, b = set(int(x) for x in idx_ref), set(int(x) for x in idx_other)
+    if a == b:
+        return True
+    if len(b) != len(a) or len(b) != len(list(idx_other)):
+        return False
+    srt = np.sort(scores_row)[::-1]
+    kk = len(a)
+    if kk >= len(srt):
+        return False
+    sk, sk1 = srt[kk - 1], srt[kk]
+    scale = max(abs(sk), abs(sk1), np.finfo(np.float64).tiny)
+    if abs(sk - sk1) >= rel * scale:
+        return False
+    band_lo, band_hi = sk1 - rel * scale, sk + rel * scale
+    for j in a.symmetric_difference(b):
+        if not band_lo <= scores_row[j] <= band_hi:
+            return False
+    return True

@@ -1,0 +1,204 @@
+/*
+ * salad.h -- C ABI of the SALAD hybrid-attention forward library (sm_100a).
+ *
+ * SALAD runs two attention branches on shared Q, K, V and mixes them with a
+ * gated, projected residual:
+ *     O = O_sparse + s_b * ((phi(Q) H / (phi(Q) Z + eps)) W_lin[h])
+ * with phi = ReLU, H = phi(K)^T V, Z = phi(K)^T 1 and
+ * s_b = sigmoid(w . mean_tokens(X[b]) + bias).
+ * Sources, by page title and section:
+ *   "SALAD ... (paper.rainbus.top)": 前置知识 (sparse mask, linear attention),
+ *       方法步骤详情 steps 2-6 (parallel branches, zero-init projection, gate,
+ *       residual sum).
+ *   "视频扩散模型中的稀疏注意力机制解析 (ijyty.com)": 1.1 (ST-SWA token
+ *       regrouping + sliding window), 1.2 (Top-K block selection from block
+ *       means), 2.3 (gate: token mean, linear, sigmoid).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors Q, K, V, O are bf16, contiguous, [B, H, N, d] with the exact
+ *     token count N (no caller padding).  d must be 64 or 128; the block
+ *     size must be 64.  N must be in [1, 262144].
+ *   - All tensor pointers are DEVICE pointers, 16-byte aligned, owned by the
+ *     caller.  Pointers documented as HOST are read during the call only.
+ *   - The library never allocates, frees or synchronises.  Scratch memory is
+ *     a caller-provided device workspace whose size is returned by the
+ *     matching *_workspace_bytes query; 256-byte alignment is required.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) in call order.  All argument checks run on the host before any
+ *     launch: an invalid call returns an error and enqueues nothing.
+ *   - Waits inside the kernels are bounded.  A wait that runs out sets a
+ *     device-side error word instead of trapping; salad_check_error() reads
+ *     it (and is the only call that synchronises).
+ */
+#ifndef SALAD_H_
+#define SALAD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int salad_status;
+#define SALAD_OK                0
+#define SALAD_ERR_INVALID_ARG  (-1)   /* null pointer, bad size, misaligned */
+#define SALAD_ERR_UNSUPPORTED  (-2)   /* d not in {64,128}, block != 64, no sm_100 device */
+#define SALAD_ERR_CUDA         (-3)   /* a CUDA runtime call or launch failed */
+#define SALAD_ERR_TIMEOUT      (-4)   /* a bounded device-side wait ran out */
+#define SALAD_ERR_WORKSPACE    (-5)   /* workspace missing, too small or misaligned */
+
+/* Sparse-branch patterns. */
+#define SALAD_MODE_TOPK   0   /* Top-K block-sparse (ijyty.com 1.2) */
+#define SALAD_MODE_SWA    1   /* spatio-temporal sliding window (ijyty.com 1.1) */
+#define SALAD_MODE_DENSE  2   /* every key (the full-attention special case) */
+
+typedef void* salad_stream;   /* cudaStream_t */
+
+/* Human-readable text of a status code; never NULL. */
+const char* salad_status_string(salad_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int salad_version(void);
+
+/*
+ * Gate (paper.rainbus.top 方法步骤详情 step 5; ijyty.com 2.3):
+ *   s[b] = sigmoid( sum_c w[c] * (1/N) sum_n x[b,n,c] + bias ).
+ * x: bf16 [B, N, D] device; w: bf16 [D] device; s: float32 [B] device (out).
+ * D must be a multiple of 8.  Workspace: salad_gate_workspace_bytes(B, N, D).
+ */
+size_t salad_gate_workspace_bytes(int B, int N, int D);
+salad_status salad_gate(const void* x, const void* w, float bias, int B, int N, int D,
+                        float* s, void* workspace, size_t workspace_bytes,
+                        salad_stream stream);
+
+/*
+ * Top-K block selection (ijyty.com 1.2): split tokens into blocks of `block`
+ * rows, average each block over its valid rows (float64), score every
+ * query-block mean against every key-block mean (float64 dot product), keep
+ * the `topk` largest per query block (ties: lower block index first).
+ * q, k: bf16 [B, H, N, d] device.  idx: int32 [B, H, nb, topk] device (out),
+ * nb = ceil(N/block), each row in ascending block order.  1 <= topk <= nb.
+ * Workspace: salad_select_workspace_bytes(B, H, N, d, block).
+ */
+size_t salad_select_workspace_bytes(int B, int H, int N, int d, int block);
+salad_status salad_select_blocks(const void* q, const void* k, int B, int H, int N, int d,
+                                 int block, int topk, int32_t* idx,
+                                 void* workspace, size_t workspace_bytes,
+                                 salad_stream stream);
+
+/*
+ * Linear-attention state (paper.rainbus.top 前置知识 Linear Attention):
+ *   Hst[b,h] = relu(K[b,h])^T V[b,h]   float32 [B, H, d, d] device (out)
+ *   Z[b,h]   = relu(K[b,h])^T 1        float32 [B, H, d]    device (out)
+ * Hst is row-major: Hst[b,h][c][j] = sum_n relu(k[n][c]) v[n][j].
+ * Workspace: salad_linear_state_workspace_bytes(B, H, N, d).
+ */
+size_t salad_linear_state_workspace_bytes(int B, int H, int N, int d);
+salad_status salad_linear_state(const void* k, const void* v, int B, int H, int N, int d,
+                                float* Hst, float* Z, void* workspace, size_t workspace_bytes,
+                                salad_stream stream);
+
+/*
+ * Linear-attention output: o_lin[b,h,n,:] = relu(q) Hst / (relu(q) . Z + eps).
+ * q: bf16 [B,H,N,d]; Hst, Z: float32 as produced above; o_lin: bf16 [B,H,N,d]
+ * (out).  Needs no workspace.
+ */
+salad_status salad_linear_apply(const void* q, const float* Hst, const float* Z, float eps,
+                                int B, int H, int N, int d, void* o_lin, salad_stream stream);
+
+/*
+ * Token permutation of the ST-SWA heads (ijyty.com 1.1).  The latent grid
+ * F x Hh x Wh (N = F*Hh*Wh) is flattened frame-major, t = (f*Hh + y)*Wh + x;
+ * the space-major order is r = (y*Wh + x)*F + f.
+ * src, dst: bf16 [S, N, d] device, S = number of (batch, head) slabs.
+ * inverse = 0: dst[s][r] = src[s][t(r)] (frame-major -> space-major);
+ * inverse = 1: dst[s][t(r)] = src[s][r] (space-major -> frame-major).
+ * src and dst must not overlap.
+ */
+salad_status salad_permute_tokens(const void* src, void* dst, int S, int N, int d,
+                                  int F, int Hh, int Wh, int inverse, salad_stream stream);
+
+/*
+ * Sparse branch alone: normalised softmax attention over the pattern,
+ * o_sparse = softmax(Q K^T / sqrt(d) + M) V, bf16 [B,H,N,d] (out).
+ *   mode SALAD_MODE_TOPK : M keeps, for query block i, the key blocks
+ *                          idx[b,h,i,0..topk) (device int32, ascending).
+ *   mode SALAD_MODE_SWA  : M keeps |r - c| <= window in each head's order;
+ *                          heads with space_major_heads[h] != 0 (HOST uint8
+ *                          [H], may be NULL = none) are regrouped
+ *                          space-major with the (F, Hh, Wh) grid and their
+ *                          output rows are returned in frame-major order.
+ *   mode SALAD_MODE_DENSE: every key.
+ * Workspace: salad_sparse_attn_workspace_bytes(...).
+ */
+size_t salad_sparse_attn_workspace_bytes(int B, int H, int N, int d, int mode, int topk,
+                                         const uint8_t* space_major_heads);
+salad_status salad_sparse_attn(const void* q, const void* k, const void* v,
+                               int B, int H, int N, int d, int mode, int block, int topk,
+                               const int32_t* idx, int window,
+                               const uint8_t* space_major_heads, int F, int Hh, int Wh,
+                               void* o_sparse, void* workspace, size_t workspace_bytes,
+                               salad_stream stream);
+
+/*
+ * Dense flash attention on the same shapes (the comparator the method is
+ * measured against): o = softmax(Q K^T / sqrt(d)) V, bf16 [B,H,N,d] (out).
+ * Needs no workspace.
+ */
+salad_status salad_dense_attn(const void* q, const void* k, const void* v,
+                              int B, int H, int N, int d, void* o, salad_stream stream);
+
+/*
+ * The whole hybrid layer (paper.rainbus.top 方法步骤详情 steps 2-6):
+ * gate, sparse branch, linear branch, per-head projection W_lin (d x d,
+ * right-multiplying row vectors: O_l' = O_l W_lin[h]), gated residual sum.
+ */
+typedef struct salad_forward_args {
+    const void* q;              /* bf16 [B,H,N,d] device */
+    const void* k;              /* bf16 [B,H,N,d] device */
+    const void* v;              /* bf16 [B,H,N,d] device */
+    const void* x;              /* bf16 [B,N,D] device: gate input (time-modulated hidden state) */
+    const void* w_gate;         /* bf16 [D] device */
+    float gate_bias;
+    const void* w_lin;          /* bf16 [H,d,d] device */
+    void* o;                    /* bf16 [B,H,N,d] device (out) */
+    int B, H, N, d, D;
+    int mode;                   /* SALAD_MODE_* */
+    int block;                  /* must be 64 */
+    int topk;                   /* TOPK mode: key blocks per query block, 1..nb */
+    int window;                 /* SWA mode: half-width, >= 0 */
+    const uint8_t* space_major_heads;  /* SWA mode: HOST uint8 [H] or NULL */
+    int F, Hh, Wh;              /* SWA mode: latent grid, F*Hh*Wh == N */
+    float eps;                  /* linear-attention denominator eps (1e-6) */
+    float gate_override;        /* NaN: use the gate; otherwise s_b = this value */
+    float* s_out;               /* optional device float32 [B] (out), may be NULL */
+    int32_t* idx_out;           /* optional device int32 [B,H,nb,topk] (out), may be NULL */
+    void* workspace;            /* device scratch, >= salad_forward_workspace_bytes() */
+    size_t workspace_bytes;
+} salad_forward_args;
+
+size_t salad_forward_workspace_bytes(const salad_forward_args* args);
+salad_status salad_forward(const salad_forward_args* args, salad_stream stream);
+
+/*
+ * Reads and clears the device-side error word after synchronising `stream`.
+ * Returns SALAD_ERR_TIMEOUT if any kernel gave up a bounded wait since the
+ * last check, SALAD_ERR_CUDA if the stream reports an error, else SALAD_OK.
+ */
+salad_status salad_check_error(salad_stream stream);
+
+/*
+ * Test hook for the bounded-wait machinery: launches one CTA that waits on
+ * an mbarrier nothing will ever arrive on, with a limit of `timeout_ns`
+ * nanoseconds, then records SALAD_ERR_TIMEOUT in the device error word and
+ * exits.  Used to check that a wait which runs out surfaces as an error
+ * status rather than a hang or a trap.
+ */
+salad_status salad_debug_wait_timeout(unsigned long long timeout_ns, salad_stream stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* SALAD_H_ */

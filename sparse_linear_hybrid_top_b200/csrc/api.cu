@@ -1,0 +1,507 @@
+// api.cu -- the C ABI declared in include/salad.h: host-side argument checks,
+// workspace carve-up, tensor-map creation and the launch sequence of the
+// hybrid layer.  Every check runs before the first launch of a call.
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "salad.h"
+
+namespace salad {
+
+// The library's device error word (one per device, read by salad_check_error).
+__device__ unsigned g_err_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxN = 262144;
+constexpr int kMaxHeads = 256;
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
+
+struct DevInfo {
+  bool ready = false;
+  bool supported = false;
+  int num_sms = 0;
+  unsigned* err = nullptr;
+};
+DevInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+unsigned long long wait_limit_ns() {
+  const char* s = std::getenv("SALAD_WAIT_NS");
+  if (s != nullptr) {
+    const unsigned long long v = std::strtoull(s, nullptr, 10);
+    if (v > 0) return v;
+  }
+  return kDefaultWaitNs;
+}
+
+// Fills the launch context for the current device.  Returns SALAD_OK, or an
+// error when no usable sm_100 device is current.
+salad_status get_ctx(salad_stream stream, Ctx* c) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SALAD_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.ready) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return SALAD_ERR_CUDA;
+    d.supported = (prop.major == 10 && prop.minor == 0);
+    d.num_sms = prop.multiProcessorCount;
+    if (d.supported) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return SALAD_ERR_CUDA;
+      d.err = static_cast<unsigned*>(p);
+    }
+    d.ready = true;
+  }
+  if (!d.supported) return SALAD_ERR_UNSUPPORTED;
+  c->stream = static_cast<cudaStream_t>(stream);
+  c->err = d.err;
+  c->num_sms = d.num_sms;
+  c->wait_ns = wait_limit_ns();
+  return SALAD_OK;
+}
+
+inline bool aligned(const void* p, size_t a) {
+  return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+inline salad_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SALAD_OK : SALAD_ERR_CUDA; }
+
+// Common shape checks for [B, H, N, d] attention tensors.
+salad_status check_bhnd(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1) return SALAD_ERR_INVALID_ARG;
+  if (H > kMaxHeads || N > kMaxN) return SALAD_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 65535) return SALAD_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SALAD_ERR_UNSUPPORTED;
+  return SALAD_OK;
+}
+
+salad_status check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return SALAD_OK;
+  if (ws == nullptr || have < need || !aligned(ws, 256)) return SALAD_ERR_WORKSPACE;
+  return SALAD_OK;
+}
+
+inline int nblocks(int N) { return (N + 63) / 64; }
+
+// Regrouped (space-major) heads of an SWA call: slots and count.
+int space_major_slots(int H, const uint8_t* flags, int* slot) {
+  int n = 0;
+  for (int h = 0; h < H; ++h) slot[h] = (flags != nullptr && flags[h] != 0) ? n++ : -1;
+  return n;
+}
+
+}  // namespace
+
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, int S, int N, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(S)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * d * 2};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------- forward layout --
+struct FwdLayout {
+  size_t gate, s, sel, idx, lists, counts, lin, hst, z, g, qp, kp, vp, total;
+  int Hs;
+  int slot[kMaxHeads];
+};
+
+static FwdLayout forward_layout(const salad_forward_args* a) {
+  FwdLayout L;
+  std::memset(&L, 0, sizeof(L));
+  const size_t B = a->B, H = a->H, N = a->N, d = a->d;
+  const size_t nb = static_cast<size_t>(nblocks(a->N));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  L.gate = take(gate_ws_bytes(a->B, a->N, a->D));
+  L.s = take(B * sizeof(float));
+  if (a->mode == SALAD_MODE_TOPK) {
+    L.sel = take(select_ws_bytes(a->B, a->H, a->N, a->d, 64));
+    L.idx = take(B * H * nb * a->topk * sizeof(int32_t));
+    const size_t items = B * H * ((nb + 1) / 2);
+    L.lists = take(items * 2 * a->topk * sizeof(int32_t));
+    L.counts = take(items * sizeof(int32_t));
+  }
+  L.lin = take(linear_state_ws_bytes(a->B, a->H, a->N, a->d));
+  L.hst = take(B * H * d * d * sizeof(float));
+  L.z = take(B * H * d * sizeof(float));
+  L.g = take(B * H * d * d * sizeof(float));
+  L.Hs = 0;
+  for (int h = 0; h < kMaxHeads; ++h) L.slot[h] = -1;
+  if (a->mode == SALAD_MODE_SWA && a->H <= kMaxHeads)
+    L.Hs = space_major_slots(a->H, a->space_major_heads, L.slot);
+  if (L.Hs > 0) {
+    const size_t bytes = B * static_cast<size_t>(L.Hs) * N * d * 2;
+    L.qp = take(bytes);
+    L.kp = take(bytes);
+    L.vp = take(bytes);
+  }
+  L.total = off;
+  return L;
+}
+
+}  // namespace salad
+
+using namespace salad;
+
+extern "C" {
+
+const char* salad_status_string(salad_status s) {
+  switch (s) {
+    case SALAD_OK: return "ok";
+    case SALAD_ERR_INVALID_ARG: return "invalid argument";
+    case SALAD_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case SALAD_ERR_CUDA: return "CUDA error";
+    case SALAD_ERR_TIMEOUT: return "bounded device wait timed out";
+    case SALAD_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    default: return "unknown status";
+  }
+}
+
+int salad_version(void) { return 100; }
+
+// ------------------------------------------------------------------ gate --
+size_t salad_gate_workspace_bytes(int B, int N, int D) {
+  if (B < 1 || N < 1 || D < 8) return 0;
+  return gate_ws_bytes(B, N, D);
+}
+
+salad_status salad_gate(const void* x, const void* w, float bias, int B, int N, int D, float* s,
+                        void* workspace, size_t workspace_bytes, salad_stream stream) {
+  if (B < 1 || N < 1 || D < 8 || D % 8 != 0 || B > 65535) return SALAD_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w, 16) || !aligned(s, 4)) return SALAD_ERR_INVALID_ARG;
+  salad_status st = check_ws(workspace, workspace_bytes, gate_ws_bytes(B, N, D));
+  if (st != SALAD_OK) return st;
+  Ctx c;
+  if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
+  return from_cuda(launch_gate(c, x, w, bias, B, N, D, s, workspace));
+}
+
+// ---------------------------------------------------------------- select --
+size_t salad_select_workspace_bytes(int B, int H, int N, int d, int block) {
+  if (check_bhnd(B, H, N, d) != SALAD_OK || block != 64) return 0;
+  return select_ws_bytes(B, H, N, d, block);
+}
+
+salad_status salad_select_blocks(const void* q, const void* k, int B, int H, int N, int d,
+                                 int block, int topk, int32_t* idx, void* workspace,
+                                 size_t workspace_bytes, salad_stream stream) {
+  salad_status st = check_bhnd(B, H, N, d);
+  if (st != SALAD_OK) return st;
+  if (block != 64) return SALAD_ERR_UNSUPPORTED;
+  if (topk < 1 || topk > nblocks(N)) return SALAD_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(idx, 4)) return SALAD_ERR_INVALID_ARG;
+  if ((st = check_ws(workspace, workspace_bytes, select_ws_bytes(B, H, N, d, block))) != SALAD_OK)
+    return st;
+  Ctx c;
+  if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
+  return from_cuda(launch_select(c, q, k, B, H, N, d, topk, idx, workspace));
+}
+
+// ---------------------------------------------------------------- linear --
+size_t salad_linear_state_workspace_bytes(int B, int H, int N, int d) {
+  if (check_bhnd(B, H, N, d) != SALAD_OK) return 0;
+  return linear_state_ws_bytes(B, H, N, d);
+}
+
+salad_status salad_linear_state(const void* k, const void* v, int B, int H, int N, int d,
+                                float* Hst, float* Z, void* workspace, size_t workspace_bytes,
+                                salad_stream stream) {
+  salad_status st = check_bhnd(B, H, N, d);
+  if (st != SALAD_OK) return st;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(Hst, 16) || !aligned(Z, 4))
+    return SALAD_ERR_INVALID_ARG;
+  if ((st = check_ws(workspace, workspace_bytes, linear_state_ws_bytes(B, H, N, d))) != SALAD_OK)
+    return st;
+  Ctx c;
+  if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
+  return from_cuda(launch_linear_state(c, k, v, B, H, N, d, Hst, Z, workspace));
+}
+
+salad_status salad_linear_apply(const void* q, const float* Hst, const float* Z, float eps, int B,
+                                int H, int N, int d, void* o_lin, salad_stream stream) {
+  salad_status st = check_bhnd(B, H, N, d);
+  if (st != SALAD_OK) return st;
+  if (!aligned(q, 16) || !aligned(Hst, 4) || !aligned(Z, 4) || !aligned(o_lin, 16))
+    return SALAD_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return SALAD_ERR_INVALID_ARG;
+  Ctx c;
+  if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
+  return from_cuda(launch_linear_apply(c, q, Hst, Z, eps, B, H, N, d, o_lin));
+}
+
+// --------------------------------------------------------------- permute --
+salad_status salad_permute_tokens(const void* src, void* dst, int S, int N, int d, int F, int Hh,
+                                  int Wh, int inverse, salad_stream stream) {
+  if (S < 1 || N < 1 || F < 1 || Hh < 1 || Wh < 1) return SALAD_ERR_INVALID_ARG;
+  if (static_cast<long long>(F) * Hh * Wh != N) return SALAD_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SALAD_ERR_UNSUPPORTED;
+  if (!aligned(src, 16) || !aligned(dst, 16) || (inverse != 0 && inverse != 1))
+    return SALAD_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(S) * N * d * 2;
+  const char* a = static_cast<const char*>(src);
+  const char* b = static_cast<const char*>(dst);
+  if (a < b + bytes && b < a + bytes) return SALAD_ERR_INVALID_ARG;  // overlap
+  salad_status st;
+  Ctx c;
+  if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
+  return from_cuda(launch_permute(c, src, dst, S, N, d, F, Hh, Wh, inverse));
+}
+
+// ----------------------------------------------------------- sparse attn --
+size_t salad_sparse_attn_workspace_bytes(int B, int H, int N, int d, int mode, int topk,
+                                         const uint8_t* space_major_heads) {
+  if (check_bhnd(B, H, N, d) != SALAD_OK) return 0;
+  if (mode == SALAD_MODE_TOPK) {
+    if (topk < 1 || topk > nblocks(N)) return 0;
+    return pairs_ws_bytes(B, H, N, topk);
+  }
+  if (mode == SALAD_MODE_SWA) {
+    int slot[kMaxHeads];
+    const int hs = space_major_slots(H, space_major_heads, slot);
+    return 3 * align256(static_cast<size_t>(B) * hs * N * d * 2);
+  }
+  return 0;
+}
+
+salad_status salad_sparse_attn(const void* q, const void* k, const void* v, int B, int H, int N,
+                               int d, int mode, int block, int topk, const int32_t* idx,
+                               int window, const uint8_t* space_major_heads, int F, int Hh,
+                               int Wh, void* o_sparse, void* workspace, size_t workspace_bytes,
+                               salad_stream stream) {
+  salad_status st = check_bhnd(B, H, N, d);
+  if (st != SALAD_OK) return st;
+  if (block != 64) return SALAD_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o_sparse, 16))
+    return SALAD_ERR_INVALID_ARG;
+  if (mode != SALAD_MODE_TOPK && mode != SALAD_MODE_SWA && mode != SALAD_MODE_DENSE)
+    return SALAD_ERR_INVALID_ARG;
+  int slot[kMaxHeads];
+  int Hs = 0;
+  if (mode == SALAD_MODE_TOPK) {
+    if (topk < 1 || topk > nblocks(N) || !aligned(idx, 4)) return SALAD_ERR_INVALID_ARG;
+  } else if (mode == SALAD_MODE_SWA) {
+    if (window < 0) return SALAD_ERR_INVALID_ARG;
+    Hs = space_major_slots(H, space_major_heads, slot);
+    if (Hs > 0 && (F < 1 || Hh < 1 || Wh < 1 || static_cast<long long>(F) * Hh * Wh != N))
+      return SALAD_ERR_INVALID_ARG;
+  }
+  const size_t need =
+      salad_sparse_attn_workspace_bytes(B, H, N, d, mode, topk, space_major_heads);
+  if ((st = check_ws(workspace, workspace_bytes, need)) != SALAD_OK) return st;
+  Ctx c;
+  if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
+
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v;
+  a.B = B; a.H = H; a.N = N; a.d = d;
+  a.window = window; a.F = F; a.Hh = Hh; a.Wh = Wh;
+  a.o = o_sparse;
+  a.gate_override = 0.f;
+  char* ws = static_cast<char*>(workspace);
+  if (mode == SALAD_MODE_TOPK) {
+    const int nb = nblocks(N);
+    const size_t items = static_cast<size_t>(B) * H * ((nb + 1) / 2);
+    int32_t* lists = reinterpret_cast<int32_t*>(ws);
+    int32_t* counts = reinterpret_cast<int32_t*>(ws + align256(items * 2 * topk * sizeof(int32_t)));
+    cudaError_t e = launch_pair_union(c, idx, B * H, nb, topk, lists, counts);
+    if (e != cudaSuccess) return SALAD_ERR_CUDA;
+    a.mode = kModeTopk;
+    a.lists = lists;
+    a.counts = counts;
+    a.list_stride = 2 * topk;
+  } else if (mode == SALAD_MODE_SWA) {
+    a.mode = kModeBand;
+    if (Hs > 0) {
+      const size_t bytes = align256(static_cast<size_t>(B) * Hs * N * d * 2);
+      a.qp = ws;
+      a.kp = ws + bytes;
+      a.vp = ws + 2 * bytes;
+      a.Hs = Hs;
+      a.head_slot = slot;
+      int sel[kMaxHeads];
+      for (int h = 0; h < H; ++h)
+        if (slot[h] >= 0) sel[slot[h]] = h;
+      cudaError_t e = launch_gather_heads_space_major(c, q, k, v, ws, ws + bytes, ws + 2 * bytes,
+                                                      B, H, N, d, F, Hh, Wh, sel, Hs);
+      if (e != cudaSuccess) return SALAD_ERR_CUDA;
+    }
+  } else {
+    a.mode = kModeDense;
+  }
+  return from_cuda(launch_attention(c, a));
+}
+
+salad_status salad_dense_attn(const void* q, const void* k, const void* v, int B, int H, int N,
+                              int d, void* o, salad_stream stream) {
+  return salad_sparse_attn(q, k, v, B, H, N, d, SALAD_MODE_DENSE, 64, 0, nullptr, 0, nullptr, 0,
+                           0, 0, o, nullptr, 0, stream);
+}
+
+// --------------------------------------------------------------- forward --
+size_t salad_forward_workspace_bytes(const salad_forward_args* a) {
+  if (a == nullptr || check_bhnd(a->B, a->H, a->N, a->d) != SALAD_OK) return 0;
+  if (a->D < 8) return 0;
+  if (a->mode == SALAD_MODE_TOPK && (a->topk < 1 || a->topk > nblocks(a->N))) return 0;
+  return forward_layout(a).total;
+}
+
+salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
+  if (a == nullptr) return SALAD_ERR_INVALID_ARG;
+  salad_status st = check_bhnd(a->B, a->H, a->N, a->d);
+  if (st != SALAD_OK) return st;
+  if (a->block != 64) return SALAD_ERR_UNSUPPORTED;
+  if (a->mode != SALAD_MODE_TOPK && a->mode != SALAD_MODE_SWA && a->mode != SALAD_MODE_DENSE)
+    return SALAD_ERR_INVALID_ARG;
+  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->o, 16) ||
+      !aligned(a->x, 16) || !aligned(a->w_gate, 16) || !aligned(a->w_lin, 16))
+    return SALAD_ERR_INVALID_ARG;
+  if (a->D < 8 || a->D % 8 != 0) return SALAD_ERR_INVALID_ARG;
+  if (!(a->eps >= 0.0f) || !std::isfinite(a->eps)) return SALAD_ERR_INVALID_ARG;
+  if (a->s_out != nullptr && !aligned(a->s_out, 4)) return SALAD_ERR_INVALID_ARG;
+  if (a->idx_out != nullptr && !aligned(a->idx_out, 4)) return SALAD_ERR_INVALID_ARG;
+  const bool override_gate = !std::isnan(a->gate_override);
+  if (override_gate && !std::isfinite(a->gate_override)) return SALAD_ERR_INVALID_ARG;
+  if (a->mode == SALAD_MODE_TOPK && (a->topk < 1 || a->topk > nblocks(a->N)))
+    return SALAD_ERR_INVALID_ARG;
+  if (a->mode == SALAD_MODE_SWA && a->window < 0) return SALAD_ERR_INVALID_ARG;
+  const FwdLayout L = forward_layout(a);
+  if (L.Hs > 0 && (a->F < 1 || a->Hh < 1 || a->Wh < 1 ||
+                   static_cast<long long>(a->F) * a->Hh * a->Wh != a->N))
+    return SALAD_ERR_INVALID_ARG;
+  if ((st = check_ws(a->workspace, a->workspace_bytes, L.total)) != SALAD_OK) return st;
+  Ctx c;
+  if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
+
+  char* ws = static_cast<char*>(a->workspace);
+  const int B = a->B, H = a->H, N = a->N, d = a->d;
+  const int nb = nblocks(N);
+  cudaError_t e;
+  // 1. gate (paper.rainbus.top 方法步骤详情 step 5)
+  float* s = a->s_out != nullptr ? a->s_out : reinterpret_cast<float*>(ws + L.s);
+  if (override_gate) {
+    e = launch_fill_f32(c, s, a->gate_override, B);
+  } else {
+    e = launch_gate(c, a->x, a->w_gate, a->gate_bias, B, N, a->D, s, ws + L.gate);
+  }
+  if (e != cudaSuccess) return SALAD_ERR_CUDA;
+
+  AttnArgs at;
+  std::memset(&at, 0, sizeof(at));
+  at.q = a->q; at.k = a->k; at.v = a->v;
+  at.B = B; at.H = H; at.N = N; at.d = d;
+  at.window = a->window; at.F = a->F; at.Hh = a->Hh; at.Wh = a->Wh;
+  at.o = a->o;
+  at.eps = a->eps;
+  at.s = s;
+  // 2. sparse-branch pattern (ijyty.com 1.1 / 1.2)
+  if (a->mode == SALAD_MODE_TOPK) {
+    int32_t* idx = a->idx_out != nullptr ? a->idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+    e = launch_select(c, a->q, a->k, B, H, N, d, a->topk, idx, ws + L.sel);
+    if (e != cudaSuccess) return SALAD_ERR_CUDA;
+    int32_t* lists = reinterpret_cast<int32_t*>(ws + L.lists);
+    int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+    e = launch_pair_union(c, idx, B * H, nb, a->topk, lists, counts);
+    if (e != cudaSuccess) return SALAD_ERR_CUDA;
+    at.mode = kModeTopk;
+    at.lists = lists;
+    at.counts = counts;
+    at.list_stride = 2 * a->topk;
+  } else if (a->mode == SALAD_MODE_SWA) {
+    at.mode = kModeBand;
+    if (L.Hs > 0) {
+      int sel[kMaxHeads];
+      for (int h = 0; h < H; ++h)
+        if (L.slot[h] >= 0) sel[L.slot[h]] = h;
+      e = launch_gather_heads_space_major(c, a->q, a->k, a->v, ws + L.qp, ws + L.kp, ws + L.vp, B,
+                                          H, N, d, a->F, a->Hh, a->Wh, sel, L.Hs);
+      if (e != cudaSuccess) return SALAD_ERR_CUDA;
+      at.qp = ws + L.qp;
+      at.kp = ws + L.kp;
+      at.vp = ws + L.vp;
+      at.Hs = L.Hs;
+      at.head_slot = L.slot;
+    }
+  } else {
+    at.mode = kModeDense;
+  }
+  // 3. linear branch state and the folded projection G = H W_lin (steps 3-4)
+  float* Hst = reinterpret_cast<float*>(ws + L.hst);
+  float* Z = reinterpret_cast<float*>(ws + L.z);
+  float* G = reinterpret_cast<float*>(ws + L.g);
+  e = launch_linear_state(c, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin);
+  if (e != cudaSuccess) return SALAD_ERR_CUDA;
+  e = launch_linear_fold(c, Hst, a->w_lin, B, H, d, G);
+  if (e != cudaSuccess) return SALAD_ERR_CUDA;
+  at.G = G;
+  at.Z = Z;
+  // 4. sparse attention with the gated residual epilogue (steps 2, 6)
+  return from_cuda(launch_attention(c, at));
+}
+
+// ------------------------------------------------------------- errors --
+salad_status salad_check_error(salad_stream stream) {
+  Ctx c;
+  salad_status st = get_ctx(stream, &c);
+  if (st != SALAD_OK) return st;
+  if (cudaStreamSynchronize(c.stream) != cudaSuccess) return SALAD_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpy(&word, c.err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SALAD_ERR_CUDA;
+  if (word != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(c.err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return SALAD_ERR_CUDA;
+    return SALAD_ERR_TIMEOUT;
+  }
+  return SALAD_OK;
+}
+
+salad_status salad_debug_wait_timeout(unsigned long long timeout_ns, salad_stream stream) {
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return SALAD_ERR_INVALID_ARG;
+  Ctx c;
+  salad_status st = get_ctx(stream, &c);
+  if (st != SALAD_OK) return st;
+  c.wait_ns = timeout_ns;
+  return from_cuda(launch_debug_wait(c));
+}
+
+}  // extern "C"

@@ -1,0 +1,133 @@
+// gate.cu -- the input-aware scalar gate of the hybrid layer.
+//
+// "SALAD ... (paper.rainbus.top)" 方法步骤详情 step 5 and "视频扩散模型中的稀疏
+// 注意力机制解析" 2.3: average the hidden state over tokens, apply a linear map
+// and a sigmoid:  s_b = sigmoid(w . mean_n X[b, n, :] + bias).
+// Because the map is linear, w . mean_n X = (1/N) sum_{n,c} w_c X[b,n,c]: one
+// streaming pass over X (the only HBM traffic), a per-CTA partial in float32,
+// then a fixed-order float64 sum of the partials (deterministic).
+#include "common.cuh"
+#include "internal.h"
+
+namespace salad {
+namespace {
+
+constexpr int kGateThreads = 256;
+constexpr int kGateUnroll = 4;
+
+__device__ __forceinline__ float dot8(const uint4& xv, const uint4& wv) {
+  const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+  const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 a = unpack_bf16x2(xs[i]);
+    float2 b = unpack_bf16x2(ws[i]);
+    acc = fmaf(a.x, b.x, acc);
+    acc = fmaf(a.y, b.y, acc);
+  }
+  return acc;
+}
+
+// grid (ctas_per_b, B).  X[b] is read as a flat run of 16-byte chunks; chunk
+// q covers columns 8*(q % CD) .. +7 with CD = D / 8.
+__global__ void __launch_bounds__(kGateThreads) gate_partial_kernel(
+    const uint4* __restrict__ x, const uint4* __restrict__ w, long long chunks_per_b, int CD,
+    float* __restrict__ partial) {
+  const int b = blockIdx.y;
+  const uint4* xb = x + static_cast<long long>(b) * chunks_per_b;
+  const long long stride = static_cast<long long>(gridDim.x) * kGateThreads;
+  long long q = static_cast<long long>(blockIdx.x) * kGateThreads + threadIdx.x;
+  int col = static_cast<int>(q % CD);
+  const int col_step = static_cast<int>(stride % CD);
+  float acc = 0.f;
+  // Main loop: kGateUnroll independent loads in flight per thread.
+  for (; q + (kGateUnroll - 1) * stride < chunks_per_b; q += kGateUnroll * stride) {
+    uint4 xv[kGateUnroll];
+    int cs[kGateUnroll];
+#pragma unroll
+    for (int u = 0; u < kGateUnroll; ++u) {
+      xv[u] = __ldcs(xb + q + u * stride);
+      cs[u] = col;
+      col += col_step;
+      if (col >= CD) col -= CD;
+    }
+#pragma unroll
+    for (int u = 0; u < kGateUnroll; ++u) acc += dot8(xv[u], __ldg(w + cs[u]));
+  }
+  for (; q < chunks_per_b; q += stride) {
+    acc += dot8(__ldcs(xb + q), __ldg(w + col));
+    col += col_step;
+    if (col >= CD) col -= CD;
+  }
+  // Block reduction (fixed order).
+  __shared__ float red[kGateThreads / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int i = 0; i < kGateThreads / 32; ++i) t += red[i];
+    partial[static_cast<long long>(b) * gridDim.x + blockIdx.x] = t;
+  }
+}
+
+__global__ void gate_final_kernel(const float* __restrict__ partial, int nparts, int N,
+                                  float bias, float* __restrict__ s) {
+  const int b = blockIdx.x;
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x)
+    acc += static_cast<double>(partial[static_cast<long long>(b) * nparts + i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < static_cast<int>(blockDim.x) / 32; ++i) t += red[i];
+    const double z = t / static_cast<double>(N) + static_cast<double>(bias);
+    s[b] = static_cast<float>(1.0 / (1.0 + exp(-z)));
+  }
+}
+
+__global__ void fill_f32_kernel(float* dst, float value, int n) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = value;
+}
+
+int gate_ctas_per_b(int B, int N, int D, int num_sms) {
+  const long long chunks = static_cast<long long>(N) * (D / 8);
+  long long want = (chunks + kGateThreads * kGateUnroll - 1) / (kGateThreads * kGateUnroll);
+  long long cap = (static_cast<long long>(num_sms) * 8 + B - 1) / B;  // ~8 CTAs per SM overall
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  return static_cast<int>(want);
+}
+
+}  // namespace
+
+size_t gate_ws_bytes(int B, int N, int D) {
+  // Sized for the largest grid the launch can pick (up to 8 CTAs per SM on a
+  // 256-SM part), independent of the device.
+  return align256(static_cast<size_t>(B) * gate_ctas_per_b(B, N, D, 256) * sizeof(float));
+}
+
+cudaError_t launch_gate(const Ctx& c, const void* x, const void* w, float bias, int B, int N,
+                        int D, float* s, void* ws) {
+  const int nparts = gate_ctas_per_b(B, N, D, c.num_sms < 256 ? c.num_sms : 256);
+  const long long chunks_per_b = static_cast<long long>(N) * (D / 8);
+  float* partial = static_cast<float*>(ws);
+  gate_partial_kernel<<<dim3(nparts, B), kGateThreads, 0, c.stream>>>(
+      static_cast<const uint4*>(x), static_cast<const uint4*>(w), chunks_per_b, D / 8, partial);
+  gate_final_kernel<<<B, 256, 0, c.stream>>>(partial, nparts, N, bias, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_f32(const Ctx& c, float* dst, float value, int n) {
+  fill_f32_kernel<<<(n + 255) / 256, 256, 0, c.stream>>>(dst, value, n);
+  return cudaGetLastError();
+}
+
+}  // namespace salad

@@ -1,0 +1,95 @@
+// internal.h -- launch wrappers shared between the kernel files and the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace salad {
+
+// Per-call launch context.
+struct Ctx {
+  cudaStream_t stream;
+  unsigned* err;              // device error word
+  int num_sms;
+  unsigned long long wait_ns; // limit of every bounded device wait
+};
+
+// Round up to a multiple of 256 bytes (workspace carve-up alignment).
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// ---- gate (gate.cu)
+size_t gate_ws_bytes(int B, int N, int D);
+cudaError_t launch_gate(const Ctx& c, const void* x, const void* w, float bias, int B, int N,
+                        int D, float* s, void* ws);
+cudaError_t launch_fill_f32(const Ctx& c, float* dst, float value, int n);
+
+// ---- block selection (select.cu)
+size_t select_ws_bytes(int B, int H, int N, int d, int block);
+cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
+                          int topk, int32_t* idx, void* ws);
+// Merge the kept lists of query blocks (2p, 2p+1) into one ascending list of
+// entries (j | mask << 16), mask bit 0 = block 2p keeps j, bit 1 = block 2p+1.
+size_t pairs_ws_bytes(int B, int H, int N, int topk);
+cudaError_t launch_pair_union(const Ctx& c, const int32_t* idx, int BH, int nb, int topk,
+                              int32_t* lists, int32_t* counts);
+
+// ---- linear branch (linear.cu)
+size_t linear_state_ws_bytes(int B, int H, int N, int d);
+cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int B, int H, int N,
+                                int d, float* Hst, float* Z, void* ws);
+// G[b,h] = Hst[b,h] W_lin[h]  (float32 [B,H,d,d])
+cudaError_t launch_linear_fold(const Ctx& c, const float* Hst, const void* w_lin, int B, int H,
+                               int d, float* G);
+cudaError_t launch_linear_apply(const Ctx& c, const void* q, const float* Hst, const float* Z,
+                                float eps, int B, int H, int N, int d, void* o);
+
+// ---- permutation (permute.cu)
+cudaError_t launch_permute(const Ctx& c, const void* src, void* dst, int S, int N, int d, int F,
+                           int Hh, int Wh, int inverse);
+// Gather the listed heads (host list, nsel <= 256) of Q, K, V [B,H,N,d] into
+// space-major slabs [B,nsel,N,d].
+cudaError_t launch_gather_heads_space_major(const Ctx& c, const void* q, const void* k,
+                                            const void* v, void* qp, void* kp, void* vp, int B,
+                                            int H, int N, int d, int F, int Hh, int Wh,
+                                            const int* sel, int nsel);
+
+// ---- attention (attn.cu)
+enum AttnMode : int { kModeTopk = 0, kModeBand = 1, kModeDense = 2 };
+
+struct AttnArgs {
+  // Frame-major inputs [B,H,N,d] and, for space-major heads, the regrouped
+  // copies [B,Hs,N,d] (may be null when no head is regrouped).
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* qp;
+  const void* kp;
+  const void* vp;
+  const int* head_slot;       // HOST [H] (or null): slot in the regrouped copies or -1
+  int B, H, N, d, Hs;
+  int mode;                   // AttnMode
+  int window;                 // band half-width
+  int F, Hh, Wh;              // grid of the regrouped heads
+  const int32_t* lists;       // topk: [B*H*npairs][2*topk] entries j | mask<<16
+  const int32_t* counts;      // topk: [B*H*npairs]
+  int list_stride;            // 2*topk
+  // Hybrid epilogue (null G = plain normalised attention output).
+  const float* G;             // [B,H,d,d] float32: Hst W_lin
+  const float* Z;             // [B,H,d]
+  const float* s;             // [B] gate values (device)
+  float gate_override;        // used when s is null
+  float eps;
+  void* o;                    // bf16 [B,H,N,d]
+};
+cudaError_t launch_attention(const Ctx& c, const AttnArgs& a);
+
+// Debug: one CTA waits on an mbarrier nothing arrives on, bounded.
+cudaError_t launch_debug_wait(const Ctx& c);
+
+// Tensor map for a bf16 [S, N, d] tensor viewed as 3-D (d, N, S), box
+// (64, 64, 1), 128-byte swizzle.  Returns false on failure.
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, int S, int N, int d);
+
+}  // namespace salad

@@ -11,3 +11,6 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: large CPU work (oracle at full size)")
+    # The binding loads libsalad.so at import; build it first if it is stale.
+    from sparse_linear_hybrid_top_b200 import build as _build
+    _build.build()

@@ -1,0 +1,175 @@
+"""GPU parity of the whole hybrid layer (salad_forward) against the oracle.
+
+Small cases are compared element by element on every output.  The full-size
+workloads are run in the launch configuration the benchmark times and
+compared on every output (480p Top-K) or on seeded samples of query blocks
+the oracle computes one by one (the rest).  Selections may differ from the
+oracle's only at near ties (k-th and (k+1)-th scores within 1e-5 relative);
+the output is then compared under the GPU's selection.
+Bar: max |err| <= 2e-2, relative L2 <= 5e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import WORKLOADS, generate
+from tests._parity import assert_close, device_inputs, to64
+from tests.test_gpu_attention import SWA_SMALL, SWA_SMALL64
+from tests.test_gpu_kernels import CASES, RAGGED128
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def salad():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import sparse_linear_hybrid_top_b200 as m
+    return m
+
+
+def _plan(salad, w, dev, **kw):
+    extra = {}
+    if w.mode == "swa":
+        extra = dict(window=w.window, space_major_heads=w.space_major_heads, F=w.F, Hh=w.Hh,
+                     Wh=w.Wh)
+    nb = w.nb
+    idx_out = torch.empty(w.B, w.H, nb, max(w.topk, 1), dtype=torch.int32, device="cuda") \
+        if w.mode == "topk" else None
+    s_out = torch.empty(w.B, dtype=torch.float32, device="cuda")
+    return salad.ForwardPlan(dev["q"], dev["k"], dev["v"], dev["x"], dev["w_gate"], dev["w_lin"],
+                             mode=w.mode, topk=w.topk, bias=w.bias, eps=w.eps, idx_out=idx_out,
+                             s_out=s_out, **extra, **kw)
+
+
+def _selection_used(w, inp, idx_gpu):
+    """GPU kept sets, after checking each against the oracle (near-tie rule)."""
+    q, k = to64(inp["q"]), to64(inp["k"])
+    idx = idx_gpu.cpu().numpy().astype(np.int64)
+    for b in range(w.B):
+        for h in range(w.H):
+            S = oracle.block_scores(q[b, h], k[b, h], w.block)
+            ref = oracle.select_topk(S, w.topk)
+            for i in range(w.nb):
+                assert oracle.near_tie_equivalent(S[i], ref[i], idx[b, h, i]), (b, h, i)
+    return idx
+
+
+@pytest.mark.parametrize("w", CASES + [SWA_SMALL, SWA_SMALL64], ids=lambda w: w.name)
+def test_forward_small_full_compare(salad, w):
+    inp = generate(w)
+    dev = device_inputs(inp)
+    plan = _plan(salad, w, dev)
+    o = plan.run()
+    torch.cuda.synchronize()
+    salad.check_error()
+    kw = dict(mode=w.mode, block=w.block, topk=w.topk, window=w.window,
+              space_major_heads=w.space_major_heads, F=w.F, Hh=w.Hh, Wh=w.Wh, eps=w.eps)
+    if w.mode == "topk":
+        kw["idx_override"] = _selection_used(w, inp, plan.idx_out)
+    ref = oracle.forward(inp, **kw)
+    np.testing.assert_allclose(to64(plan.s_out), ref["s"], rtol=0, atol=1e-5)
+    assert_close(o, ref["o"], f"forward {w.name}")
+
+
+def test_forward_gate_zero_and_zero_projection_give_sparse_branch(salad):
+    w = RAGGED128
+    inp = generate(w)
+    dev = device_inputs(inp)
+    plan = _plan(salad, w, dev, gate_override=0.0)
+    o = plan.run().clone()
+    o_sparse = salad.sparse_attn(dev["q"], dev["k"], dev["v"], "topk", topk=w.topk,
+                                 idx=plan.idx_out)
+    assert torch.equal(o, o_sparse)
+    dev0 = dict(dev)
+    dev0["w_lin"] = torch.zeros_like(dev["w_lin"])
+    o0 = _plan(salad, w, dev0).run()
+    assert torch.equal(o0, o_sparse)
+    salad.check_error()
+
+
+def test_forward_is_deterministic(salad):
+    w = RAGGED128
+    dev = device_inputs(generate(w))
+    plan = _plan(salad, w, dev)
+    a = plan.run().clone()
+    b = plan.run().clone()
+    assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------ full sizes ---
+def _oracle_rows(w, inp, b, h, rows_in_order, idx_row_of, s_b, lin_cache):
+    """Oracle output rows of one head, rows given in the head's attention order."""
+    q, k, v = (to64(inp[n][b, h]) for n in ("q", "k", "v"))
+    if (b, h) not in lin_cache:
+        lin_cache[(b, h)] = oracle.linear_state(k, v)
+    Hst, Z = lin_cache[(b, h)]
+    if w.mode == "topk":
+        blocks = sorted(set(int(r) // w.block for r in rows_in_order))
+        res = oracle.topk_attention_rows(q, k, v, idx_row_of, w.block, blocks)
+        o_s = np.concatenate([res[i] for i in blocks])
+        rows = np.concatenate([np.arange(i * w.block, min(w.N, (i + 1) * w.block)) for i in blocks])
+        tok = rows
+    else:
+        sm = h in w.space_major_heads
+        perm = oracle.space_major_order(w.F, w.Hh, w.Wh) if sm else np.arange(w.N)
+        qo, ko, vo = q[perm], k[perm], v[perm]
+        rows = np.asarray(rows_in_order)
+        o_s = oracle.swa_attention_rows(qo, ko, vo, w.window, rows)
+        tok = perm[rows]
+    o_l = oracle.linear_apply(q[tok], Hst, Z, w.eps)
+    o = oracle.combine(o_s, o_l, to64(inp["w_lin"][h]), s_b)
+    return tok, o
+
+
+def _sampled_check(salad, w, n_samples, seed=0, full=False):
+    inp = generate(w)
+    dev = device_inputs(inp)
+    plan = _plan(salad, w, dev)
+    o = plan.run()
+    torch.cuda.synchronize()
+    salad.check_error()
+    s_ref = oracle.gate(inp["x"], inp["w_gate"], inp["bias"])
+    np.testing.assert_allclose(to64(plan.s_out), s_ref, rtol=0, atol=1e-5)
+    idx = _selection_used(w, inp, plan.idx_out) if w.mode == "topk" else None
+    o_cpu = o.cpu()
+    rng = np.random.default_rng(seed)
+    lin_cache = {}
+    got_all, want_all = [], []
+    if full:
+        units = [(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(w.nb)]
+    else:
+        units = [(int(rng.integers(w.B)), int(rng.integers(w.H)), int(rng.integers(w.nb)))
+                 for _ in range(n_samples)]
+        units += [(w.B - 1, w.H - 1, w.nb - 1)]  # the ragged tail is always checked
+    by_head = {}
+    for b, h, i in units:
+        by_head.setdefault((b, h), set()).add(i)
+    for (b, h), blocks in sorted(by_head.items()):
+        rows = np.concatenate([np.arange(i * w.block, min(w.N, (i + 1) * w.block))
+                               for i in sorted(blocks)])
+        tok, want = _oracle_rows(w, inp, b, h, rows, None if idx is None else idx[b, h],
+                                 s_ref[b], lin_cache)
+        got_all.append(o_cpu[b, h, torch.from_numpy(tok)])
+        want_all.append(want)
+    got = torch.cat(got_all)
+    want = np.concatenate(want_all)
+    return assert_close(got, want, f"forward {w.name} ({len(units)} query blocks)")
+
+
+def test_forward_topk480_every_output(salad):
+    _sampled_check(salad, WORKLOADS["topk480"], 0, full=True)
+
+
+def test_forward_swa480_sampled(salad):
+    _sampled_check(salad, WORKLOADS["swa480"], 96, seed=1)
+
+
+def test_forward_topk720_sampled(salad):
+    _sampled_check(salad, WORKLOADS["topk720"], 64, seed=2)
+
+
+@pytest.mark.parametrize("name", ["cfg_b2h40_s80", "cfg_b2h40_s95", "cfg_b2h40_all"])
+def test_forward_b2h40_sampled(salad, name):
+    _sampled_check(salad, WORKLOADS[name], 48, seed=3)

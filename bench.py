@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark of the SALAD hybrid-attention forward layer (one layer = one step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+gate, Top-K selection (or ST-SWA regrouping), linear-attention state, and the
+sparse attention kernel with the fused gated linear term.  The default
+workload is the 480p-like Top-K layer (B=1, H=12, d=128, N=31200, 488 blocks,
+k=49, ~90% sparsity).
+
+Metric: effective TFLOP/s counting only computed work -- 4*d*64^2 per kept
+(query block, key block) pair plus 6*N*d^2 + 4*N*d per head for the linear
+branch -- over the device time of K back-to-back steps (CUDA events, max over
+ranks).  ms per layer is reported beside it.  Inputs (Q, K, V, X: 384 MB at the
+default size) exceed the 126 MB L2, so no flush is inserted between steps.
+
+Multi-GPU (torchrun): every rank runs an independent replica of the layer on
+its own GPU (weak scaling, no collective on the data path); NCCL is used only
+for the barrier and the max-over-ranks reduction of the elapsed time.
+
+--impl reference times the CPU oracle on a bounded sample of the same
+workload (rank 0 only) and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ms/layer & effective TFLOP/s, SALAD attn fwd N=31200 90% sparse; % roofline"
+UNIT = "effective TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ work ---
+def step_flops(w) -> dict:
+    """Algorithmic work of one layer (counted, not executed, flops)."""
+    B, H, N, d, bs = w.B, w.H, w.N, w.d, w.block
+    nb = w.nb
+    if w.mode == "topk":
+        pairs = B * H * nb * w.topk
+        sparse = 4.0 * d * bs * bs * pairs
+    elif w.mode == "swa":
+        # Exact (query, key) pairs inside the window, clipped at the ends.
+        W = w.window
+        per_head = sum(min(N - 1, r + W) - max(0, r - W) + 1 for r in range(N))
+        sparse = 4.0 * d * per_head * B * H
+    else:
+        sparse = 4.0 * d * N * N * B * H
+    linear = (6.0 * N * d * d + 4.0 * N * d) * B * H
+    # The attention kernel itself: the sparse branch plus phi(Q) (H W_lin).
+    attn_kernel = sparse + 2.0 * N * d * d * B * H
+    dense = 4.0 * d * N * N * B * H
+    return {"sparse": sparse, "linear": linear, "total": sparse + linear,
+            "attn_kernel": attn_kernel, "dense": dense}
+
+
+def launches_per_step(w) -> int:
+    # gate (2) + [pool, score, topk, pair_union | gather] + linear (3) + attention (1)
+    if w.mode == "topk":
+        return 2 + 4 + 3 + 1
+    if w.mode == "swa":
+        return 2 + (1 if w.space_major_heads else 0) + 3 + 1
+    return 2 + 3 + 1
+
+
+def load_peaks() -> tuple:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("attn.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "sparse_linear_hybrid_top_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if the
+    kernel source is unchanged since it was captured; else None."""
+    p = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    ent = rec.get(workload)
+    if not ent or ent.get("attn_source_hash") != attn_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks ---
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------- distributed ---
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(backend: str, world: int):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of a float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and str(device).startswith("cuda"):
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate(world: int, flops_per_step: float, steps: int, max_ms: float) -> dict:
+    """Whole-job throughput of `world` replicas that each ran `steps` steps,
+    timed as the max over ranks."""
+    total = world * flops_per_step * steps
+    return {"value": total / (max_ms * 1e-3) / 1e12, "ms_per_step": max_ms / steps}
+
+
+# ------------------------------------------------------------ CPU oracle ---
+def cpu_sample_work(w, inp, n_heads: int, blocks_per_head: int, seed: int = 0):
+    """Runs the oracle on a bounded sample of the layer; returns (flops, seconds).
+
+    The sample: the gate over all of X, then for `n_heads` heads the block
+    selection (all query blocks), the linear state, and for `blocks_per_head`
+    query blocks the sparse attention plus the linear term of their rows.
+    Counted flops follow the metric's rule restricted to the sample."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(seed)
+    B, H, N, d, bs = w.B, w.H, w.N, w.d, w.block
+    heads = [(int(rng.integers(B)), int(h)) for h in rng.choice(H, size=min(n_heads, H), replace=False)]
+    t0 = time.perf_counter()
+    s = oracle.gate(inp["x"], inp["w_gate"], inp["bias"])
+    flops = 0.0
+    for b, h in heads:
+        q, k, v = (oracle.as64(inp[n][b, h]) for n in ("q", "k", "v"))
+        Hst, Z = oracle.linear_state(k, v)
+        flops += 2.0 * N * d * d + N * d
+        blocks = rng.choice(w.nb, size=min(blocks_per_head, w.nb), replace=False)
+        if w.mode == "topk":
+            idx = oracle.select_topk(oracle.block_scores(q, k, bs), w.topk)
+            res = oracle.topk_attention_rows(q, k, v, idx, bs, blocks)
+            kept = w.topk
+        else:
+            res = {}
+            for i in blocks:
+                rows = np.arange(i * bs, min(N, (i + 1) * bs))
+                res[i] = (oracle.swa_attention_rows(q, k, v, w.window, rows) if w.mode == "swa"
+                          else oracle.dense_attention(q[rows], k, v))
+            kept = min(w.nb, (2 * w.window) // bs + 1) if w.mode == "swa" else w.nb
+        for i in blocks:
+            rows = np.arange(i * bs, min(N, (i + 1) * bs))
+            o_l = oracle.linear_apply(q[rows], Hst, Z, w.eps)
+            oracle.combine(res[i], o_l, oracle.as64(inp["w_lin"][h]), s[b])
+            flops += 4.0 * d * bs * bs * kept + len(rows) * (4.0 * d * d + 4.0 * d)
+    return flops, time.perf_counter() - t0
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ runs ---
+def run_ours(args, w) -> int:
+    import torch
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        print(json.dumps({"error": f"WORLD_SIZE={world} but --gpus {args.gpus}"}), flush=True)
+        return 2
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist("nccl", world)
+    import sparse_linear_hybrid_top_b200 as salad
+    from synth import generate
+
+    host = generate(w)
+    dev = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
+    extra = {}
+    if w.mode == "swa":
+        extra = dict(window=w.window, space_major_heads=w.space_major_heads, F=w.F, Hh=w.Hh,
+                     Wh=w.Wh)
+    plan = salad.ForwardPlan(dev["q"], dev["k"], dev["v"], dev["x"], dev["w_gate"], dev["w_lin"],
+                             mode=w.mode, topk=w.topk, bias=w.bias, eps=w.eps, **extra)
+    stream = torch.cuda.current_stream(device)
+    fl = step_flops(w)
+
+    for _ in range(args.warmup):
+        plan.run(stream)
+    salad.check_error(stream)
+
+    # Phase events: 5 per step, recorded by the library on the launch stream.
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else local)
+    for e5 in ev:                 # create the handles before the timed region
+        for e in e5:
+            e.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    clocks.start()
+    start.record(stream)
+    for i in range(args.steps):
+        plan.set_phase_events(ev[i])
+        plan.run(stream)
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    plan.set_phase_events(None)
+    salad.check_error(stream)
+    local_ms = start.elapsed_time(end)
+    max_ms = reduce_max(local_ms, device)
+    agg = aggregate(world, fl["total"], args.steps, max_ms)
+
+    def phase(a, b):
+        return statistics.fmean(e5[a].elapsed_time(e5[b]) for e5 in ev)
+    phases = {"gate": phase(0, 1), "pattern": phase(1, 2), "linear_state": phase(2, 3),
+              "attention": phase(3, 4)}
+    attn_ms = phases["attention"]
+
+    # Dense comparator on the same Q, K, V (same library).
+    for _ in range(2):
+        salad.dense_attn(dev["q"], dev["k"], dev["v"], stream=stream)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nd = max(2, min(10, args.steps))
+    d0.record(stream)
+    for _ in range(nd):
+        salad.dense_attn(dev["q"], dev["k"], dev["v"], stream=stream)
+    d1.record(stream)
+    torch.cuda.synchronize(device)
+    dense_ms = d0.elapsed_time(d1) / nd
+
+    # End to end through the public API: pinned host inputs -> device ->
+    # salad_forward -> result back to the host, every step.
+    names = ("q", "k", "v", "x", "w_gate", "w_lin")
+    pinned = {n: host[n].pin_memory() for n in names}
+    out_host = torch.empty(plan.o.shape, dtype=plan.o.dtype).pin_memory()
+    h2d = sum(pinned[n].numel() * pinned[n].element_size() for n in names)
+    d2h = out_host.numel() * out_host.element_size()
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(2):
+        for n in names:
+            dev[n].copy_(pinned[n], non_blocking=True)
+        plan.run(stream)
+        out_host.copy_(plan.o, non_blocking=True)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for n in names:
+            dev[n].copy_(pinned[n], non_blocking=True)
+        plan.run(stream)
+        out_host.copy_(plan.o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), device)
+    e2e = aggregate(world, fl["total"], e2e_steps, e2e_ms)
+
+    peaks, peaks_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    achieved = fl["attn_kernel"] / (attn_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(agg["value"], 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "block": w.block, "mode": w.mode, "topk": w.topk, "window": w.window,
+                   "nb": w.nb, "D": w.D,
+                   "sparsity": round(1 - fl["sparse"] / fl["dense"], 4),
+                   "parallelism": f"replicas{world}",
+                   "l2": "no flush: inputs (Q,K,V,X) %.0f MB > 126 MB L2" % (h2d / 1e6)},
+        "ms_per_layer": round(agg["ms_per_step"], 5),
+        "phases_ms": {k: round(v, 5) for k, v in phases.items()},
+        "dense_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / agg["ms_per_step"], 3),
+        "flops_per_step": fl["total"],
+        "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,hybrid>",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "peak_source": f"bf16 sustained, {peaks_src}",
+                     "traffic": committed_traffic(w.name),
+                     "algorithmic_flops_per_launch": fl["attn_kernel"]},
+        "e2e": {"value": round(e2e["value"], 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "ms_per_step": round(e2e["ms_per_step"], 4)},
+        "gpu_launches": launches_per_step(w) * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        del dev
+        flops, secs = cpu_sample_work(w, host, n_heads=2, blocks_per_head=args.cpu_blocks)
+        line["cpu_baseline"] = {"value": round(flops / secs / 1e12, 6), "unit": UNIT,
+                                "cores": cpu_threads(), "kind": "oracle",
+                                "sample": f"gate over all X; 2 heads: selection, linear state, "
+                                          f"{args.cpu_blocks} query blocks each (attention + "
+                                          f"linear term); {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        barrier(device)
+        dist.destroy_process_group()
+    return 0
+
+
+def run_reference(args, w) -> int:
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    from synth import generate
+    host = generate(w)
+    for _ in range(args.warmup):
+        cpu_sample_work(w, host, n_heads=1, blocks_per_head=args.ref_blocks, seed=1000)
+    t_flops, t_secs = 0.0, 0.0
+    for i in range(args.steps):
+        f, s = cpu_sample_work(w, host, n_heads=1, blocks_per_head=args.ref_blocks, seed=i)
+        t_flops += f
+        t_secs += s
+    value = t_flops / t_secs / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "impl": "reference",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t_secs * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "block": w.block, "mode": w.mode, "topk": w.topk, "window": w.window},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cpu_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: gate over all X; 1 head: selection, linear "
+                                   f"state, {args.ref_blocks} query blocks"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="topk480")
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-blocks", type=int, default=96, help="query blocks per head in cpu_baseline")
+    ap.add_argument("--ref-blocks", type=int, default=16, help="query blocks per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    from synth import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -176,6 +176,11 @@ typedef struct salad_forward_args {
     int32_t* idx_out;           /* optional device int32 [B,H,nb,topk] (out), may be NULL */
     void* workspace;            /* device scratch, >= salad_forward_workspace_bytes() */
     size_t workspace_bytes;
+    /* Optional profiling hook: NULL, or a HOST array of 5 cudaEvent_t that
+     * are recorded on `stream` at the start, after the gate, after the
+     * sparse-pattern step (selection or regrouping), after the linear
+     * state, and after the attention kernel. */
+    void* const* phase_events;
 } salad_forward_args;
 
 size_t salad_forward_workspace_bytes(const salad_forward_args* args);

@@ -62,6 +62,7 @@ class ForwardArgs(ctypes.Structure):
         ("eps", ctypes.c_float), ("gate_override", ctypes.c_float),
         ("s_out", ctypes.c_void_p), ("idx_out", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("phase_events", ctypes.c_void_p),
     ]
 
 
@@ -290,6 +291,18 @@ class ForwardPlan:
         a.workspace = _ptr(self.workspace)
         a.workspace_bytes = need
         self.args = a
+
+    def set_phase_events(self, events: Optional[Sequence[torch.cuda.Event]]) -> None:
+        """Record these 5 events inside each run (start, gate, pattern, linear, attention)."""
+        if events is None:
+            self._events, self.args.phase_events = None, None
+            return
+        if len(events) != 5:
+            raise ValueError("need 5 events")
+        for ev in events:
+            ev.record()   # creates the underlying cudaEvent_t
+        self._events = (ctypes.c_void_p * 5)(*[ev.cuda_event for ev in events])
+        self.args.phase_events = ctypes.cast(self._events, ctypes.c_void_p)
 
     def run(self, stream=None) -> torch.Tensor:
         _check(lib.salad_forward(ctypes.byref(self.args), _stream(stream)), "salad_forward")

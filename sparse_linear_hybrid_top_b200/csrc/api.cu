@@ -415,6 +415,11 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   const int B = a->B, H = a->H, N = a->N, d = a->d;
   const int nb = nblocks(N);
   cudaError_t e;
+  auto mark = [&](int i) -> bool {
+    if (a->phase_events == nullptr || a->phase_events[i] == nullptr) return true;
+    return cudaEventRecord(static_cast<cudaEvent_t>(a->phase_events[i]), c.stream) == cudaSuccess;
+  };
+  if (!mark(0)) return SALAD_ERR_CUDA;
   // 1. gate (paper.rainbus.top 方法步骤详情 step 5)
   float* s = a->s_out != nullptr ? a->s_out : reinterpret_cast<float*>(ws + L.s);
   if (override_gate) {
@@ -422,7 +427,7 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   } else {
     e = launch_gate(c, a->x, a->w_gate, a->gate_bias, B, N, a->D, s, ws + L.gate);
   }
-  if (e != cudaSuccess) return SALAD_ERR_CUDA;
+  if (e != cudaSuccess || !mark(1)) return SALAD_ERR_CUDA;
 
   AttnArgs at;
   std::memset(&at, 0, sizeof(at));
@@ -463,6 +468,7 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   } else {
     at.mode = kModeDense;
   }
+  if (!mark(2)) return SALAD_ERR_CUDA;
   // 3. linear branch state and the folded projection G = H W_lin (steps 3-4)
   float* Hst = reinterpret_cast<float*>(ws + L.hst);
   float* Z = reinterpret_cast<float*>(ws + L.z);
@@ -470,11 +476,13 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   e = launch_linear_state(c, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin);
   if (e != cudaSuccess) return SALAD_ERR_CUDA;
   e = launch_linear_fold(c, Hst, a->w_lin, B, H, d, G);
-  if (e != cudaSuccess) return SALAD_ERR_CUDA;
+  if (e != cudaSuccess || !mark(3)) return SALAD_ERR_CUDA;
   at.G = G;
   at.Z = Z;
   // 4. sparse attention with the gated residual epilogue (steps 2, 6)
-  return from_cuda(launch_attention(c, at));
+  e = launch_attention(c, at);
+  if (e != cudaSuccess || !mark(4)) return SALAD_ERR_CUDA;
+  return SALAD_OK;
 }
 
 // ------------------------------------------------------------- errors --

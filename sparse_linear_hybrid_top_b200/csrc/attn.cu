@@ -19,6 +19,12 @@
 // P = 0 for it.  Online softmax with a lazily raised running max (the O row
 // is rescaled only when the max grows by more than 2^8).
 //
+// Barrier discipline: an mbarrier parity wait is only sound when the waiter is
+// at most one phase behind.  Every barrier here is therefore observed by each
+// of its waiters at every phase: in particular each softmax warp waits for
+// PV(t-1) once per tile (after computing and storing P(t), so the wait
+// overlaps its own work), rescales O only then, and only then releases tile t.
+//
 // Warp roles (192 threads, one CTA per SM, persistent over work items):
 //   warp 0      TMA producer: K and V tiles (64 x d, 128B swizzle) into a
 //               ring of stages.
@@ -386,6 +392,7 @@ __global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CU
         }
         const bool live = row_valid && (mask & half_bit) && lo <= hi;
         uint32_t pk[32];
+        float f = 1.0f;            // factor O must be rescaled by before PV(t)
         if (__any_sync(0xffffffffu, live)) {
           uint32_t s0[32], s1[32];
           tmem_ld32(lane_base + C::kS + sb * 64, s0);
@@ -396,29 +403,13 @@ __global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CU
             mx = (live && c >= lo && c <= hi) ? fmaxf(mx, __uint_as_float(s0[c]) * c2) : mx;
             mx = (live && c + 32 >= lo && c + 32 <= hi) ? fmaxf(mx, __uint_as_float(s1[c]) * c2) : mx;
           }
-          const bool raise = live && mx > m + 8.0f;
-          const bool rescale = raise && m != -INFINITY;
-          if (__any_sync(0xffffffffu, rescale)) {
-            // Rescale O rows (and l) once PV(t-1) has landed.  t >= 1 here.
-            const long long g = pv_base + t - 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(o_done, static_cast<uint32_t>(g & 1), wait_ns, abort_flag))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const float f = rescale ? ex2(m - mx) : 1.0f;
+          if (live && mx > m + 8.0f) {
+            // Raise the running max.  O (from PV up to t-1) is rescaled below,
+            // once PV(t-1) has landed; l is rescaled here.
+            f = (m == -INFINITY) ? 1.0f : ex2(m - mx);
             l *= f;
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t o32[32];
-              tmem_ld32(lane_base + C::kO + c0, o32);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o32[e] = __float_as_uint(__uint_as_float(o32[e]) * f);
-              tmem_st32(lane_base + C::kO + c0, o32);
-            }
-            tmem_st_wait();
+            m = mx;
           }
-          if (raise) m = mx;
           float lsum = 0.f;
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
@@ -438,6 +429,26 @@ __global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CU
           for (int e = 0; e < 32; ++e) pk[e] = 0u;
         }
         tmem_st32(lane_base + C::kS + sb * 64, pk);
+        // Observe PV(t-1) -- every warp observes every PV completion in order,
+        // so each parity wait is at most one phase behind the barrier.
+        if (t >= 1) {
+          const long long g = pv_base + t - 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(o_done, static_cast<uint32_t>(g & 1), wait_ns, abort_flag))) {
+            ok = false;
+            break;
+          }
+        }
+        if (__any_sync(0xffffffffu, f != 1.0f)) {
+          tc_fence_after();
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o32[32];
+            tmem_ld32(lane_base + C::kO + c0, o32);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o32[e] = __float_as_uint(__uint_as_float(o32[e]) * f);
+            tmem_st32(lane_base + C::kO + c0, o32);
+          }
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();

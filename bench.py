@@ -390,10 +390,10 @@ def run_ours(args, w) -> int:
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         del dev
-        flops, secs = cpu_sample_work(w, host, n_heads=2, blocks_per_head=args.cpu_blocks)
+        flops, secs = cpu_sample_work(w, host, n_heads=args.cpu_heads, blocks_per_head=args.cpu_blocks)
         line["cpu_baseline"] = {"value": round(flops / secs / 1e12, 6), "unit": UNIT,
                                 "cores": cpu_threads(), "kind": "oracle",
-                                "sample": f"gate over all X; 2 heads: selection, linear state, "
+                                "sample": f"gate over all X; {args.cpu_heads} heads: selection, linear state, "
                                           f"{args.cpu_blocks} query blocks each (attention + "
                                           f"linear term); {secs:.1f} s"}
     if rank == 0:
@@ -444,7 +444,8 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="topk480")
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--cpu-blocks", type=int, default=96, help="query blocks per head in cpu_baseline")
+    ap.add_argument("--cpu-heads", type=int, default=6, help="heads in the cpu_baseline sample")
+    ap.add_argument("--cpu-blocks", type=int, default=488, help="query blocks per head in cpu_baseline")
     ap.add_argument("--ref-blocks", type=int, default=16, help="query blocks per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

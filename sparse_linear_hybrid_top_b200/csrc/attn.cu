@@ -391,39 +391,58 @@ __global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CU
           hi = min(hi, row_pos + P.window - j * 64);
         }
         const bool live = row_valid && (mask & half_bit) && lo <= hi;
+        const bool whole = live && lo == 0 && hi == 63;
         uint32_t pk[32];
         float f = 1.0f;            // factor O must be rescaled by before PV(t)
         if (__any_sync(0xffffffffu, live)) {
-          uint32_t s0[32], s1[32];
-          tmem_ld32(lane_base + C::kS + sb * 64, s0);
-          tmem_ld32(lane_base + C::kS + sb * 64 + 32, s1);
-          float mx = -INFINITY;
+          float sv[64];
+          {
+            uint32_t s0[32], s1[32];
+            tmem_ld32(lane_base + C::kS + sb * 64, s0);
+            tmem_ld32(lane_base + C::kS + sb * 64 + 32, s1);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            mx = (live && c >= lo && c <= hi) ? fmaxf(mx, __uint_as_float(s0[c]) * c2) : mx;
-            mx = (live && c + 32 >= lo && c + 32 <= hi) ? fmaxf(mx, __uint_as_float(s1[c]) * c2) : mx;
+            for (int c = 0; c < 32; ++c) {
+              sv[c] = __uint_as_float(s0[c]);
+              sv[c + 32] = __uint_as_float(s1[c]);
+            }
           }
-          if (live && mx > m + 8.0f) {
+          // Columns outside [lo, hi] (and every column of a dead row) become
+          // -inf; only tiles with a partial row in this warp pay for it.
+          if (__any_sync(0xffffffffu, !whole)) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) sv[c] = (live && c >= lo && c <= hi) ? sv[c] : -INFINITY;
+          }
+          float t32[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) t32[c] = fmaxf(sv[c], sv[c + 32]);
+#pragma unroll
+          for (int w2 = 16; w2 >= 1; w2 >>= 1)
+#pragma unroll
+            for (int c = 0; c < w2; ++c) t32[c] = fmaxf(t32[c], t32[c + w2]);
+          const float mx = t32[0] * c2;   // c2 > 0: max of scaled = scaled max
+          if (mx > m + 8.0f) {
             // Raise the running max.  O (from PV up to t-1) is rescaled below,
             // once PV(t-1) has landed; l is rescaled here.
             f = (m == -INFINITY) ? 1.0f : ex2(m - mx);
             l *= f;
             m = mx;
           }
-          float lsum = 0.f;
+          // A row with no valid key so far keeps m = -inf: use 0 as the
+          // offset so its -inf scores give exp2(-inf) = 0, never NaN.
+          const float nm = (m == -INFINITY) ? 0.0f : -m;
+          float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            const float a0 = (live && c >= lo && c <= hi) ? ex2(fmaf(__uint_as_float(s0[c]), c2, -m)) : 0.f;
-            const float a1 = (live && c + 1 >= lo && c + 1 <= hi) ? ex2(fmaf(__uint_as_float(s0[c + 1]), c2, -m)) : 0.f;
-            const float b0 = (live && c + 32 >= lo && c + 32 <= hi) ? ex2(fmaf(__uint_as_float(s1[c]), c2, -m)) : 0.f;
-            const float b1 = (live && c + 33 >= lo && c + 33 <= hi) ? ex2(fmaf(__uint_as_float(s1[c + 1]), c2, -m)) : 0.f;
+            const float a0 = ex2(fmaf(sv[c], c2, nm));
+            const float a1 = ex2(fmaf(sv[c + 1], c2, nm));
+            const float b0 = ex2(fmaf(sv[c + 32], c2, nm));
+            const float b1 = ex2(fmaf(sv[c + 33], c2, nm));
             pk[c / 2] = pack_bf16x2(a0, a1);
             pk[16 + c / 2] = pack_bf16x2(b0, b1);
-            const float2 pa = unpack_bf16x2(pk[c / 2]);
-            const float2 pb = unpack_bf16x2(pk[16 + c / 2]);
-            lsum += (pa.x + pa.y) + (pb.x + pb.y);
+            ls0 += a0 + a1;
+            ls1 += b0 + b1;
           }
-          l += lsum;
+          l += ls0 + ls1;
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) pk[e] = 0u;

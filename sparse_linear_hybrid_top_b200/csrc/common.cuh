@@ -245,10 +245,11 @@ template <int D>
 __device__ __forceinline__ void build_b_image_hilo(const float* __restrict__ M,
                                                    unsigned char* img_hi, unsigned char* img_lo,
                                                    int tid, int nthreads) {
+  // Step e covers element pair (c, c+1) of column j, with j fastest so that
+  // consecutive threads read consecutive floats of a row of M.
   for (int e = tid; e < D * D / 2; e += nthreads) {
-    // Two consecutive c for one j per step: element pair (c, c+1).
-    const int j = e / (D / 2);
-    const int c = (e % (D / 2)) * 2;
+    const int j = e % D;
+    const int c = (e / D) * 2;
     const float m0 = __ldg(M + static_cast<long long>(c) * D + j);
     const float m1 = __ldg(M + static_cast<long long>(c + 1) * D + j);
     const __nv_bfloat16 h0 = __float2bfloat16_rn(m0), h1 = __float2bfloat16_rn(m1);

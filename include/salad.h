@@ -73,6 +73,26 @@ salad_status salad_gate(const void* x, const void* w, float bias, int B, int N, 
                         salad_stream stream);
 
 /*
+ * Gate with no scratch argument, for callers that cannot allocate device
+ * memory at all (a plug-in that receives only its input and output buffers,
+ * or code on a path where an allocator call is not permitted).  No passage of
+ * the paper corresponds to it: it computes exactly what salad_gate computes,
+ * but keeps its per-CTA partial sums in a fixed 64 KB array inside the
+ * library (present on every GPU that loads the library, until the process
+ * exits) instead of a caller workspace.
+ *   - B may be at most 256; larger batches return SALAD_ERR_INVALID_ARG
+ *     before any launch.  Other arguments as for salad_gate.
+ *   - The first call on each device looks up the array's device address;
+ *     make that first call before capturing the stream into a CUDA graph.
+ *   - All calls share the one array, and each call overwrites the slots it
+ *     reads, so no clearing is needed -- but two calls whose kernels overlap
+ *     on the GPU (different streams without ordering) race on it.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library.
+ */
+salad_status salad_gate_noalloc(const void* x, const void* w, float bias, int B, int N, int D,
+                                float* s, salad_stream stream);
+
+/*
  * Top-K block selection (ijyty.com 1.2): split tokens into blocks of `block`
  * rows, average each block over its valid rows (float64), score every
  * query-block mean against every key-block mean (float64 dot product), keep

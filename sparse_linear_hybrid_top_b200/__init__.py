@@ -16,7 +16,7 @@ import torch
 
 __all__ = [
     "SaladError", "lib", "status_string", "version",
-    "gate", "select_blocks", "linear_state", "linear_apply", "permute_tokens",
+    "gate", "gate_noalloc", "select_blocks", "linear_state", "linear_apply", "permute_tokens",
     "sparse_attn", "dense_attn", "forward", "ForwardPlan", "forward_workspace_bytes",
     "check_error", "debug_wait_timeout",
     "MODE_TOPK", "MODE_SWA", "MODE_DENSE", "EXPORTED_SYMBOLS",
@@ -38,6 +38,7 @@ EXPORTED_SYMBOLS = (
     "salad_sparse_attn_workspace_bytes", "salad_sparse_attn", "salad_dense_attn",
     "salad_forward_workspace_bytes", "salad_forward",
     "salad_check_error", "salad_debug_wait_timeout",
+    "salad_gate_noalloc",
 )
 
 
@@ -91,6 +92,7 @@ def _load() -> ctypes.CDLL:
         "salad_forward": (i, [ctypes.POINTER(ForwardArgs), vp]),
         "salad_check_error": (i, [vp]),
         "salad_debug_wait_timeout": (i, [ctypes.c_ulonglong, vp]),
+        "salad_gate_noalloc": (i, [vp, vp, f, i, i, i, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -99,7 +101,20 @@ def _load() -> ctypes.CDLL:
     return L
 
 
-lib = _load()
+class _Lib:
+    """The loaded libsalad.so, opened on first use (so that the build step can
+    import this package before the library exists).  Raises ImportError on
+    first use if the library is missing: there is no fallback."""
+
+    _cdll = None
+
+    def __getattr__(self, name):
+        if _Lib._cdll is None:
+            _Lib._cdll = _load()
+        return getattr(_Lib._cdll, name)
+
+
+lib = _Lib()
 
 
 def status_string(code: int) -> str:
@@ -168,6 +183,19 @@ def gate(x: torch.Tensor, w: torch.Tensor, bias: float = 0.0, *, s=None, workspa
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib.salad_gate(_ptr(x), _ptr(w), float(bias), B, N, D, _ptr(s), _ptr(ws), nbytes,
                           _stream(stream)), "salad_gate")
+    return s
+
+
+def gate_noalloc(x: torch.Tensor, w: torch.Tensor, bias: float = 0.0, *, s=None,
+                 stream=None) -> torch.Tensor:
+    """The gate for callers that cannot allocate scratch: same result as
+    gate(), partial sums kept in the library's own fixed device array
+    (B <= 256; calls that overlap on the GPU race on that array)."""
+    _dev_tensor(x, torch.bfloat16, "x"); _dev_tensor(w, torch.bfloat16, "w")
+    B, N, D = x.shape
+    s = torch.empty(B, dtype=torch.float32, device=x.device) if s is None else s
+    _check(lib.salad_gate_noalloc(_ptr(x), _ptr(w), float(bias), B, N, D, _ptr(s),
+                                  _stream(stream)), "salad_gate_noalloc")
     return s
 
 

@@ -131,3 +131,92 @@ cudaError_t launch_fill_f32(const Ctx& c, float* dst, float value, int n) {
 }
 
 }  // namespace salad
+
+// ---------------------------------------------------------------------------
+// Gate without caller-provided scratch.
+//
+// For callers that cannot allocate device memory at all -- code that runs
+// inside a host that owns every allocation (a plug-in handed only its input
+// and output buffers), or code on a path where an allocator call is not
+// allowed -- the gate's per-CTA partial sums live in this file-scope device
+// array instead of a workspace.  The array is part of the library image: every
+// GPU that loads the library holds it (64 KB) until the process exits.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+#include "salad.h"
+
+namespace salad {
+namespace {
+
+constexpr int kNoAllocMaxBatch = 256;        // largest B the array serves
+constexpr int kNoAllocPartsPerSample = 64;   // partial sums kept per sample
+constexpr int kNoAllocFloats = kNoAllocMaxBatch * kNoAllocPartsPerSample;
+
+static __device__ __align__(256) float g_gate_scratch[kNoAllocFloats];
+
+struct NoAllocDev {
+  bool ready = false;
+  bool supported = false;
+  int num_sms = 0;
+  float* scratch = nullptr;   // device address of g_gate_scratch on this device
+};
+NoAllocDev g_noalloc_dev[64];
+std::mutex g_noalloc_mu;
+
+// One-time set-up per device, with that device current: look up the device
+// address of the array (its host-side name is only a stand-in).
+salad_status noalloc_setup(int dev, NoAllocDev** out) {
+  if (dev < 0 || dev >= 64) return SALAD_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocDev& d = g_noalloc_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SALAD_ERR_CUDA;
+    d.supported = (major == 10 && minor == 0);
+    d.num_sms = sms;
+    if (d.supported) {
+      float* ptr = nullptr;
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_gate_scratch) != cudaSuccess)
+        return SALAD_ERR_CUDA;
+      d.scratch = ptr;
+    }
+    d.ready = true;
+  }
+  if (!d.supported) return SALAD_ERR_UNSUPPORTED;
+  *out = &d;
+  return SALAD_OK;
+}
+
+}  // namespace
+}  // namespace salad
+
+extern "C" salad_status salad_gate_noalloc(const void* x, const void* w, float bias, int B, int N,
+                                           int D, float* s, salad_stream stream) {
+  using namespace salad;
+  if (B < 1 || N < 1 || D < 8 || D % 8 != 0) return SALAD_ERR_INVALID_ARG;
+  if (B > kNoAllocMaxBatch) return SALAD_ERR_INVALID_ARG;   // beyond the array's capacity
+  const uintptr_t ax = reinterpret_cast<uintptr_t>(x), aw = reinterpret_cast<uintptr_t>(w),
+                  as = reinterpret_cast<uintptr_t>(s);
+  if (x == nullptr || w == nullptr || s == nullptr || ax % 16 || aw % 16 || as % 4)
+    return SALAD_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SALAD_ERR_CUDA;
+  NoAllocDev* d = nullptr;
+  const salad_status st = noalloc_setup(dev, &d);
+  if (st != SALAD_OK) return st;
+  int nparts = gate_ctas_per_b(B, N, D, d->num_sms < 256 ? d->num_sms : 256);
+  if (nparts > kNoAllocPartsPerSample) nparts = kNoAllocPartsPerSample;
+  // Every partial slot read by the final kernel is written first by this
+  // call's partial kernel, so nothing needs clearing between calls.
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const long long chunks_per_b = static_cast<long long>(N) * (D / 8);
+  gate_partial_kernel<<<dim3(nparts, B), kGateThreads, 0, cs>>>(
+      static_cast<const uint4*>(x), static_cast<const uint4*>(w), chunks_per_b, D / 8,
+      d->scratch);
+  gate_final_kernel<<<B, 256, 0, cs>>>(d->scratch, nparts, N, bias, s);
+  return cudaGetLastError() == cudaSuccess ? SALAD_OK : SALAD_ERR_CUDA;
+}

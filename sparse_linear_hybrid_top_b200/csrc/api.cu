@@ -162,7 +162,7 @@ static FwdLayout forward_layout(const salad_forward_args* a) {
   L.lin = take(linear_state_ws_bytes(a->B, a->H, a->N, a->d));
   L.hst = take(B * H * d * d * sizeof(float));
   L.z = take(B * H * d * sizeof(float));
-  L.g = take(B * H * d * d * sizeof(float));
+  L.g = take(B * H * d * d * 2);
   L.Hs = 0;
   for (int h = 0; h < kMaxHeads; ++h) L.slot[h] = -1;
   if (a->mode == SALAD_MODE_SWA && a->H <= kMaxHeads)
@@ -472,12 +472,12 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   // 3. linear branch state and the folded projection G = H W_lin (steps 3-4)
   float* Hst = reinterpret_cast<float*>(ws + L.hst);
   float* Z = reinterpret_cast<float*>(ws + L.z);
-  float* G = reinterpret_cast<float*>(ws + L.g);
+  void* G = ws + L.g;
   e = launch_linear_state(c, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin);
   if (e != cudaSuccess) return SALAD_ERR_CUDA;
   e = launch_linear_fold(c, Hst, a->w_lin, B, H, d, G);
   if (e != cudaSuccess || !mark(3)) return SALAD_ERR_CUDA;
-  at.G = G;
+  at.Gimg = G;
   at.Z = Z;
   // 4. sparse attention with the gated residual epilogue (steps 2, 6)
   e = launch_attention(c, at);

@@ -12,57 +12,80 @@
 // (M = 128 rows, the full tcgen05 datapath).  Its key tiles are the merged,
 // ascending list of the blocks either query block keeps (Top-K), the band of
 // blocks its rows' windows touch (ST-SWA) or all blocks (dense).  For each
-// 64-key tile:  S = Q K^T  (A = Q from TMEM, B = K tile from smem, N = 64)
-// then P = exp2(S*c - m) written back to TMEM as bf16 and O += P V
-// (A = P from TMEM, B = V tile from smem, MN-major).  Only K and V tiles are
-// read from shared memory.  Rows whose query block did not keep a tile get
-// P = 0 for it.  Online softmax with a lazily raised running max (the O row
-// is rescaled only when the max grows by more than 2^8).
+// 64-key tile:  S = Q K^T  (A = Q from TMEM, B = K tile from smem, N = 64),
+// P = exp2(S*c - m) written back over S in TMEM as bf16, O += P V
+// (A = P from TMEM, B = V tile from smem, MN-major).  Rows whose query block
+// did not keep a tile get P = 0 for it.
+//
+// S tiles hold 128 keys (two 64-key blocks of the list), so the QK MMA has
+// N = 128: a tcgen05.mma with M = 128 occupies the tensor pipe for at least
+// ~64 cycles whatever its N, which leaves an N = 64 MMA at half rate.  The K
+// ring keeps consecutive 64-key stages contiguous inside each 128-byte-
+// swizzled d-half slab, so a block pair is one B operand.
+//
+// Eight softmax warps: four row quarters (the TMEM lane groups) times two
+// column halves.  The two warps holding a row exchange their partial row max
+// every tile (through a bounded mbarrier), so both apply the same running max
+// and O stays a single accumulator; each warp exponentiates 64 of the 128
+// columns, rescales its half of O when the max grows by more than 2^8, and
+// writes its half of the output.  S is double-buffered so the QK of the next
+// tile runs during the softmax of this one.  The linear term
+// s_b * phi(Q) G / (phi(Q) Z + eps) is one more MMA (A = phi(Q) from TMEM,
+// B = the bf16 image of G streamed into the V slots of a ring stage) into the
+// S_0 columns, which are free once the last PV has run.
+//
+// Warp roles (320 threads, one CTA per SM, persistent over work items):
+//   warp 0      TMA producer: K and V blocks (64 x d, 128B swizzle), two per
+//               ring stage, and the G image.
+//   warp 1      TMEM allocator and the single MMA-issuing thread.
+//   warps 2..5  softmax, column half 0; also load Q and phi(Q).
+//   warps 6..9  softmax, column half 1.
+// TMEM columns (d = 128): O [0,128) S_0 [128,256) S_1 [256,384) Q [384,448)
+// phi(Q) [448,512); the linear term lands in S_0.
 //
 // Barrier discipline: an mbarrier parity wait is only sound when the waiter is
-// at most one phase behind.  Every barrier here is therefore observed by each
-// of its waiters at every phase: in particular each softmax warp waits for
-// PV(t-1) once per tile (after computing and storing P(t), so the wait
-// overlaps its own work), rescales O only then, and only then releases tile t.
-//
-// Warp roles (192 threads, one CTA per SM, persistent over work items):
-//   warp 0      TMA producer: K and V tiles (64 x d, 128B swizzle) into a
-//               ring of stages.
-//   warp 1      TMEM allocator and the single MMA-issuing thread.
-//   warps 2..5  one query row per thread: Q (and relu(Q)) into TMEM, softmax
-//               per tile, and the epilogue (normalise, add the gated linear
-//               term, write bf16 rows; ST-SWA rows go back to frame-major).
-// Every wait is bounded; a wait that runs out raises the device error word
-// and the CTA leaves through the common teardown (loads drained, MMAs
-// committed, TMEM freed).
+// at most one phase behind.  Every barrier is observed by each of its waiters
+// at every phase: in particular each softmax warp waits for its previous PV
+// once per tile (after computing and storing P, so the wait overlaps its own
+// work), rescales its O only then, and only then releases the tile.  Every
+// wait is bounded; a wait that runs out raises the device error word and the
+// CTA leaves through the common teardown (loads drained, MMAs committed, TMEM
+// freed).
 #include "common.cuh"
 #include "internal.h"
 
 namespace salad {
-
 namespace {
 
 constexpr int kSlab = 64 * 128;
 
 template <int D, bool HYB>
 struct AT {
-  static constexpr int kStages = (D == 128) ? 4 : 6;
-  static constexpr int kTile = (D / 64) * kSlab;
-  static constexpr int kStage = 2 * kTile;
-  static constexpr int kImg = HYB ? D * D * 2 : 0;
-  static constexpr int kZ = HYB ? D * 4 : 0;
+  static constexpr int kKS = 6;                          // 64-key stages (even: pairs never wrap)
+  static constexpr int kPairs = kKS / 2;                 // ring stages of two blocks
+  static constexpr int kHalves = D / 64;                 // 128-byte d-slabs per row
+  static constexpr int kTile = kHalves * kSlab;          // one 64-key K (or V) block
+  static constexpr int kKRingHalf = kKS * kSlab;         // one d-slab of the K ring
+  static constexpr int kKRing = kHalves * kKRingHalf;
+  static constexpr int kVRing = kKS * kTile;
+  static constexpr int kGImg = D * D * 2;                // bf16 G image bytes
+  static_assert(kGImg <= 2 * kTile, "G image must fit the V slots of a pair");
+  static constexpr int kXchg = (2 * 2 * 128 + 2 * 128) * 4;  // row max/sum per parity, den per item
   static constexpr int kBarBytes = 512;
-  static constexpr int kSmemUsed = 1024 + kStages * kStage + 2 * kImg + kZ + kBarBytes;
+  static constexpr int kSmemUsed = 1024 + kKRing + kVRing + kXchg + kBarBytes;
   // At least ~half of the SM's shared memory, so one CTA (and its 512 TMEM
   // columns) occupies each SM.
   static constexpr int kSmem = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
   // TMEM columns.
-  static constexpr uint32_t kO = 0;
-  static constexpr uint32_t kS = D;              // two 64-column S/P buffers
-  static constexpr uint32_t kQ = D + 128;        // Q as A operand (D/2 columns)
-  static constexpr uint32_t kPQ = kQ + D / 2;    // relu(Q) as A operand
-  static constexpr uint32_t kL = kPQ + D / 2;    // linear-term accumulator (D columns)
+  static constexpr uint32_t kO = 0;            // D columns
+  static constexpr uint32_t kS0 = D;           // 128 columns (P aliases the first 64)
+  static constexpr uint32_t kS1 = D + 128;     // 128 columns
+  static constexpr uint32_t kL = D;            // linear term, D columns over S_0
+  static constexpr uint32_t kQ = D + 256;      // D/2 columns (A operand)
+  static constexpr uint32_t kPQ = kQ + D / 2;  // D/2 columns (A operand)
   static constexpr uint32_t kCols = 512;
+  static_assert(kPQ + D / 2 <= kCols, "TMEM budget");
+  static_assert(D <= 128, "the linear term must fit S_0");
 };
 
 struct Params {
@@ -74,7 +97,7 @@ struct Params {
   const int32_t* lists;
   const int32_t* counts;
   int list_stride;
-  const float* G;
+  const __nv_bfloat16* Gimg;  // [B*H][d*d] bf16 B-operand images of G
   const float* Z;
   const float* s;
   float gate_override;
@@ -135,51 +158,71 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Untiled bulk copy global -> shared completing on `bar` (16-byte aligned).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 template <int D, bool HYB>
-__global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CUtensorMap mk,
+__global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CUtensorMap mk,
                                                       const __grid_constant__ CUtensorMap mv,
                                                       const __grid_constant__ CUtensorMap mkp,
                                                       const __grid_constant__ CUtensorMap mvp,
                                                       const __grid_constant__ Params P) {
   using C = AT<D, HYB>;
+  constexpr int NP = C::kPairs;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  unsigned char* stages = sm;
-  unsigned char* img_hi = sm + C::kStages * C::kStage;
-  unsigned char* img_lo = img_hi + C::kImg;
-  float* zs = reinterpret_cast<float*>(img_lo + C::kImg);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(zs) + C::kZ);
-  // bars: full[S] empty[S] s_full[2] p_full[2] o_done q_ready lin_done drain
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 8);
+  unsigned char* kring = sm;                         // [d-slab][kKS x 64 rows x 128 B]
+  unsigned char* vring = sm + C::kKRing;             // [kKS][d-slab][64 rows x 128 B]
+  float* xrow = reinterpret_cast<float*>(vring + C::kVRing);  // [parity][half][128] row max / sum
+  float* xden = xrow + 2 * 2 * 128;                            // [item parity][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(xrow) + C::kXchg);
+  // bars: full[NP] empty[NP] s_full[2] p_full[2] o_done q_ready lin_done drain x_row[4]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NP + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
-  auto full = [&](int s) { return smem_u32(bars + s); };
-  auto empty = [&](int s) { return smem_u32(bars + C::kStages + s); };
-  auto s_full = [&](int b) { return smem_u32(bars + 2 * C::kStages + b); };
-  auto p_full = [&](int b) { return smem_u32(bars + 2 * C::kStages + 2 + b); };
-  const uint32_t o_done = smem_u32(bars + 2 * C::kStages + 4);
-  const uint32_t q_ready = smem_u32(bars + 2 * C::kStages + 5);
-  const uint32_t lin_done = smem_u32(bars + 2 * C::kStages + 6);
-  const uint32_t drain = smem_u32(bars + 2 * C::kStages + 7);
+  auto full = [&](int p) { return smem_u32(bars + p); };
+  auto empty = [&](int p) { return smem_u32(bars + NP + p); };
+  auto s_full = [&](int b) { return smem_u32(bars + 2 * NP + b); };
+  auto p_full = [&](int b) { return smem_u32(bars + 2 * NP + 2 + b); };
+  const uint32_t o_done = smem_u32(bars + 2 * NP + 4);
+  const uint32_t q_ready = smem_u32(bars + 2 * NP + 5);
+  const uint32_t lin_done = smem_u32(bars + 2 * NP + 6);
+  const uint32_t drain = smem_u32(bars + 2 * NP + 7);
+  auto x_row = [&](int q) { return smem_u32(bars + 2 * NP + 8 + q); };
+  // Shared-memory addresses of the blocks of ring stage (pair) p.
+  auto k_addr = [&](int p, int half) {   // rows of block 2p (then 2p+1) of one d-slab
+    return smem_u32(kring + half * C::kKRingHalf + 2 * p * kSlab);
+  };
+  auto v_addr = [&](int p, int which) {  // V block 2p + which
+    return smem_u32(vring + (2 * p + which) * C::kTile);
+  };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const long long total = static_cast<long long>(P.B) * P.H * P.npairs;
   const unsigned long long wait_ns = P.wait_ns;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(full(s), 1);
-      mbar_init(empty(s), 1);
+    for (int p = 0; p < NP; ++p) {
+      mbar_init(full(p), 1);
+      mbar_init(empty(p), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full(b), 1);
-      mbar_init(p_full(b), 4);
+      mbar_init(p_full(b), 8);
     }
     mbar_init(o_done, 1);
-    mbar_init(q_ready, 4);
+    mbar_init(q_ready, 8);   // half 0 after writing Q, half 1 after its previous epilogue
     mbar_init(lin_done, 1);
     mbar_init(drain, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(x_row(q), 2);   // the two warps of a row quarter
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_map(&mk);
@@ -201,190 +244,214 @@ __global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CU
   if (warp == 0) {
     if (lane == 0) {
       // ================================================= TMA producer
-      long long tc = 0;
+      long long pc = 0;   // ring stages filled so far
       bool ok = true;
       for (long long w = blockIdx.x; w < total && ok; w += gridDim.x) {
         const Item it = make_item(P, w);
         const CUtensorMap* km = it.slot >= 0 ? &mkp : &mk;
         const CUtensorMap* vm = it.slot >= 0 ? &mvp : &mv;
         const int z = it.slot >= 0 ? it.b * P.Hs + it.slot : it.bh;
-        for (int t = 0; t < it.ntiles; ++t, ++tc) {
-          int j, mask;
-          tile_of(it, t, P.mode, j, mask);
-          const int s = static_cast<int>(tc % C::kStages);
-          const long long n = tc / C::kStages;
-          if (n > 0 && !mbar_wait(empty(s), static_cast<uint32_t>((n - 1) & 1), wait_ns, abort_flag)) {
+        const int npair = (it.ntiles + 1) / 2;
+        for (int u = 0; u < npair + (HYB ? 1 : 0); ++u, ++pc) {
+          const int p = static_cast<int>(pc % NP);
+          const long long n = pc / NP;
+          if (n > 0 && !mbar_wait(empty(p), static_cast<uint32_t>((n - 1) & 1), wait_ns, abort_flag)) {
             raise_timeout(P.err, abort_flag);
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full(s), C::kStage);
-          const uint32_t kdst = smem_u32(stages + s * C::kStage);
-          const uint32_t vdst = kdst + C::kTile;
+          if (u < npair) {
+            const int nblk = (2 * u + 1 < it.ntiles) ? 2 : 1;
+            mbar_arrive_expect_tx(full(p), nblk * 2 * C::kTile);
+            for (int x = 0; x < nblk; ++x) {
+              int j, mask;
+              tile_of(it, 2 * u + x, P.mode, j, mask);
 #pragma unroll
-          for (int hh = 0; hh < D / 64; ++hh) {
-            tma_load_3d(kdst + hh * kSlab, km, full(s), hh * 64, j * 64, z);
-            tma_load_3d(vdst + hh * kSlab, vm, full(s), hh * 64, j * 64, z);
+              for (int hh = 0; hh < D / 64; ++hh) {
+                tma_load_3d(k_addr(p, hh) + x * kSlab, km, full(p), hh * 64, j * 64, z);
+                tma_load_3d(v_addr(p, x) + hh * kSlab, vm, full(p), hh * 64, j * 64, z);
+              }
+            }
+          } else {
+            // The G image of the item's head, in the V slots of this stage.
+            mbar_arrive_expect_tx(full(p), C::kGImg);
+            bulk_load(v_addr(p, 0), P.Gimg + static_cast<long long>(it.bh) * D * D, C::kGImg,
+                      full(p));
           }
         }
       }
       // Drain every issued load before leaving.
-      for (int s = 0; s < C::kStages && s < tc; ++s) {
-        const long long last = s + ((tc - 1 - s) / C::kStages) * C::kStages;
-        if (!mbar_wait(full(s), static_cast<uint32_t>((last / C::kStages) & 1), wait_ns, nullptr))
+      for (int p = 0; p < NP && p < pc; ++p) {
+        const long long last = p + ((pc - 1 - p) / NP) * NP;
+        if (!mbar_wait(full(p), static_cast<uint32_t>((last / NP) & 1), wait_ns, nullptr))
           atomicOr(P.err, kErrTimeout);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ================================================= MMA issuer
-      constexpr uint32_t idesc_qk = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
       constexpr uint32_t idesc_lin = idesc_bf16(128, D, false, false);
-      long long tc = 0;
+      long long pc = 0;
       uint32_t ic = 0;
-      uint32_t pf_count[2] = {0, 0};
+      uint32_t pf[2] = {0, 0};
       bool ok = true;
+      auto wait_full = [&](long long c) -> bool {
+        return mbar_wait(full(static_cast<int>(c % NP)), static_cast<uint32_t>((c / NP) & 1),
+                         wait_ns, abort_flag);
+      };
+      auto issue_qk = [&](long long c, int b) {
+        const int p = static_cast<int>(c % NP);
+        const uint32_t sbuf = b ? C::kS1 : C::kS0;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ts(tmem + sbuf, tmem + C::kQ + ks * 8,
+                 sdesc_sw128(k_addr(p, ks / 4) + (ks % 4) * 32, 16, 1024), idesc_qk,
+                 ks > 0 ? 1u : 0u);
+        mma_commit(s_full(b));
+      };
       for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++ic) {
         const Item it = make_item(P, w);
-        if (!mbar_wait(q_ready, ic & 1, wait_ns, abort_flag)) {
-          raise_timeout(P.err, abort_flag);
-          ok = false;
-          break;
-        }
+        const int npair = (it.ntiles + 1) / 2;
+        if (!mbar_wait(q_ready, ic & 1, wait_ns, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        if constexpr (HYB) {
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks / 4) * (D * 128) + (ks % 4) * 32;
-            mma_ts(tmem + C::kL, tmem + C::kPQ + ks * 8,
-                   sdesc_sw128(smem_u32(img_hi) + off, 16, 1024), idesc_lin, ks > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks / 4) * (D * 128) + (ks % 4) * 32;
-            mma_ts(tmem + C::kL, tmem + C::kPQ + ks * 8,
-                   sdesc_sw128(smem_u32(img_lo) + off, 16, 1024), idesc_lin, 1u);
-          }
-          mma_commit(lin_done);
+        for (int u = 0; u < 2 && u < npair; ++u) {
+          if (!wait_full(pc + u)) { ok = false; break; }
+          tc_fence_after();
+          issue_qk(pc + u, u);
         }
-        const long long tc0 = tc;
-        auto issue_pv = [&](int t) -> bool {
-          const int sb = t & 1;
-          if (!mbar_wait(p_full(sb), pf_count[sb] & 1, wait_ns, abort_flag)) return false;
-          ++pf_count[sb];
+        if (!ok) break;
+        for (int u = 0; u < npair; ++u) {
+          const int b = u & 1;
+          if (!mbar_wait(p_full(b), pf[b] & 1, wait_ns, abort_flag)) { ok = false; break; }
+          ++pf[b];
           tc_fence_after();
-          const int s = static_cast<int>((tc0 + t) % C::kStages);
-          const uint32_t vaddr = smem_u32(stages + s * C::kStage) + C::kTile;
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_ts(tmem + C::kO, tmem + C::kS + sb * 64 + ks * 8,
-                   sdesc_sw128(vaddr + ks * 2048, kSlab, 1024), idesc_pv,
-                   (t > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(empty(s));
+          const int p = static_cast<int>((pc + u) % NP);
+          const uint32_t pbuf = b ? C::kS1 : C::kS0;
+          const int nks = (2 * u + 1 < it.ntiles) ? 8 : 4;   // K-steps: 16 keys each
+          for (int ks = 0; ks < nks; ++ks)
+            mma_ts(tmem + C::kO, tmem + pbuf + ks * 8,
+                   sdesc_sw128(v_addr(p, ks / 4) + (ks % 4) * 2048, kSlab, 1024), idesc_pv,
+                   (u > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(empty(p));
           mma_commit(o_done);
-          return true;
-        };
-        for (int t = 0; t < it.ntiles; ++t, ++tc) {
-          const int s = static_cast<int>(tc % C::kStages);
-          if (!mbar_wait(full(s), static_cast<uint32_t>((tc / C::kStages) & 1), wait_ns, abort_flag)) {
-            ok = false;
-            break;
+          if (u + 2 < npair) {
+            if (!wait_full(pc + u + 2)) { ok = false; break; }
+            tc_fence_after();
+            issue_qk(pc + u + 2, b);   // same S buffer: runs after this PV in issue order
           }
+        }
+        if (!ok) break;
+        pc += npair;
+        if constexpr (HYB) {
+          // Linear term into S_0 (free once the last PV has run): L = phi(Q) G.
+          if (!wait_full(pc)) { ok = false; break; }
           tc_fence_after();
-          const int sb = t & 1;
-          const uint32_t kaddr = smem_u32(stages + s * C::kStage);
+          const uint32_t gaddr = v_addr(static_cast<int>(pc % NP), 0);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
-            mma_ts(tmem + C::kS + sb * 64, tmem + C::kQ + ks * 8,
-                   sdesc_sw128(kaddr + (ks / 4) * kSlab + (ks % 4) * 32, 16, 1024), idesc_qk,
+            mma_ts(tmem + C::kL, tmem + C::kPQ + ks * 8,
+                   sdesc_sw128(gaddr + (ks / 4) * (D * 128) + (ks % 4) * 32, 16, 1024), idesc_lin,
                    ks > 0 ? 1u : 0u);
-          mma_commit(s_full(sb));
-          if (t >= 1 && !issue_pv(t - 1)) {
-            ok = false;
-            break;
-          }
+          mma_commit(empty(static_cast<int>(pc % NP)));
+          mma_commit(lin_done);
+          ++pc;
         }
-        if (ok && it.ntiles >= 1 && !issue_pv(it.ntiles - 1)) ok = false;
-        if (!ok) raise_timeout(P.err, abort_flag);
       }
+      if (!ok) raise_timeout(P.err, abort_flag);
       mma_commit(drain);
       if (!mbar_wait(drain, 0, wait_ns, nullptr)) atomicOr(P.err, kErrTimeout);
     }
   } else {
     // ================================================= softmax + epilogue
+    const int hf = (warp - 2) / 4;              // column half of S, P, O and the output
     const int quarter = warp % 4;
     const int r = quarter * 32 + lane;          // row within the pair (TMEM lane)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const int tid = threadIdx.x - 64;
-    uint32_t ic = 0;
-    uint32_t sf_count[2] = {0, 0};
+    uint32_t ic = 0, sf[2] = {0, 0}, xc = 0;
     long long pv_base = 0;                      // PVs completed before this item
-    int prev_bh = -1;
     bool ok = true;
+    // Exchange of a per-row value with the other half's warp of this quarter.
+    auto exchange = [&](float mine) -> float {
+      float* slot = xrow + (xc & 1) * 256;
+      slot[hf * 128 + r] = mine;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(x_row(quarter));
+      const bool got = __all_sync(0xffffffffu, mbar_wait(x_row(quarter), xc & 1, wait_ns, abort_flag));
+      ++xc;
+      if (!got) {
+        ok = false;
+        return mine;
+      }
+      return slot[(1 - hf) * 128 + r];
+    };
     for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++ic) {
       const Item it = make_item(P, w);
       const int row_pos = it.p * 128 + r;        // position in the head's (possibly regrouped) order
       const bool row_valid = row_pos < P.N;
-      // ---- operands of this item: Q (and relu(Q), G, Z) into TMEM / smem
-      if constexpr (HYB) {
-        if (it.bh != prev_bh) {
-          build_b_image_hilo<D>(P.G + static_cast<long long>(it.bh) * D * D, img_hi, img_lo, tid, 128);
-          for (int c = tid; c < D; c += 128) zs[c] = P.Z[static_cast<long long>(it.bh) * D + c];
-          fence_proxy_async_smem();
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-        }
-      }
-      prev_bh = it.bh;
-      const __nv_bfloat16* qsrc =
-          it.slot >= 0 ? P.qp + (static_cast<long long>(it.b) * P.Hs + it.slot) * P.N * D
-                       : P.q + static_cast<long long>(it.bh) * P.N * D;
-      const uint4* qrow = reinterpret_cast<const uint4*>(qsrc + static_cast<long long>(row_valid ? row_pos : 0) * D);
-      float den = 0.f;
+      const int npair = (it.ntiles + 1) / 2;
+      if (hf == 1) {
+        // This warp's previous epilogue is complete: O, S and the linear
+        // term may be overwritten by this item's MMAs.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_ready);
+      } else {
+        // ---- Q and phi(Q) into TMEM (A operands); den = phi(q) . Z + eps
+        const __nv_bfloat16* qsrc =
+            it.slot >= 0 ? P.qp + (static_cast<long long>(it.b) * P.Hs + it.slot) * P.N * D
+                         : P.q + static_cast<long long>(it.bh) * P.N * D;
+        const uint4* qrow = reinterpret_cast<const uint4*>(
+            qsrc + static_cast<long long>(row_valid ? row_pos : 0) * D);
+        const float* zrow = HYB ? P.Z + static_cast<long long>(it.bh) * D : nullptr;
+        float den = 0.f;
 #pragma unroll
-      for (int c0 = 0; c0 < D / 2; c0 += 16) {
-        uint32_t pk[16], pr[16];
+        for (int c0 = 0; c0 < D / 2; c0 += 16) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint4 v = row_valid ? __ldg(qrow + c0 / 4 + u) : make_uint4(0, 0, 0, 0);
-          pk[4 * u + 0] = v.x; pk[4 * u + 1] = v.y; pk[4 * u + 2] = v.z; pk[4 * u + 3] = v.w;
-        }
-        tmem_st16(lane_base + C::kQ + c0, pk);
-        if constexpr (HYB) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            pr[e] = relu_bf16x2(pk[e]);
-            const float2 f = unpack_bf16x2(pr[e]);
-            den = fmaf(f.x, zs[2 * (c0 + e)], den);
-            den = fmaf(f.y, zs[2 * (c0 + e) + 1], den);
+          for (int u = 0; u < 4; ++u) {
+            const uint4 v = row_valid ? __ldg(qrow + c0 / 4 + u) : make_uint4(0, 0, 0, 0);
+            pk[4 * u + 0] = v.x; pk[4 * u + 1] = v.y; pk[4 * u + 2] = v.z; pk[4 * u + 3] = v.w;
           }
-          tmem_st16(lane_base + C::kPQ + c0, pr);
+          tmem_st16(lane_base + C::kQ + c0, pk);
+          if constexpr (HYB) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              pk[e] = relu_bf16x2(pk[e]);
+              const float2 f = unpack_bf16x2(pk[e]);
+              den = fmaf(f.x, __ldg(zrow + 2 * (c0 + e)), den);
+              den = fmaf(f.y, __ldg(zrow + 2 * (c0 + e) + 1), den);
+            }
+            tmem_st16(lane_base + C::kPQ + c0, pk);
+          }
         }
+        xden[(ic & 1) * 128 + r] = den + P.eps;
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_ready);
       }
-      den += P.eps;
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_ready);
 
-      // ---- softmax over the key tiles
+      // ---- softmax over the item's S tiles (128 keys each)
       const float c2 = P.scale_log2;
-      float m = -INFINITY;   // running max in the exp2 domain
-      float l = 0.f;
+      float m = -INFINITY;   // running max of the row in the exp2 domain (same in both halves)
+      float l = 0.f;         // this half's share of the row sum
       const int half_bit = r >= 64 ? 2 : 1;
-      for (int t = 0; t < it.ntiles; ++t) {
-        const int sb = t & 1;
+      for (int u = 0; u < npair; ++u) {
+        const int b = u & 1;
+        const uint32_t sbuf = b ? C::kS1 : C::kS0;
         // Waits and TMEM accesses are warp-collective: every decision that
         // guards one is made uniform across the warp first.
-        if (!__all_sync(0xffffffffu, mbar_wait(s_full(sb), sf_count[sb] & 1, wait_ns, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(s_full(b), sf[b] & 1, wait_ns, abort_flag))) {
           ok = false;
           break;
         }
-        ++sf_count[sb];
+        ++sf[b];
         tc_fence_after();
-        int j, mask;
-        tile_of(it, t, P.mode, j, mask);
-        // Valid key columns of this tile form one contiguous range [lo, hi].
+        const int t = 2 * u + hf;                  // this half's key block
+        int j = 0, mask = 0;
+        if (t < it.ntiles) tile_of(it, t, P.mode, j, mask);
+        // Valid key columns of the block form one contiguous range [lo, hi].
         int lo = 0, hi = min(63, P.N - 1 - j * 64);
         if (P.mode == kModeBand) {
           lo = max(lo, row_pos - P.window - j * 64);
@@ -392,14 +459,14 @@ __global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CU
         }
         const bool live = row_valid && (mask & half_bit) && lo <= hi;
         const bool whole = live && lo == 0 && hi == 63;
-        uint32_t pk[32];
-        float f = 1.0f;            // factor O must be rescaled by before PV(t)
-        if (__any_sync(0xffffffffu, live)) {
-          float sv[64];
+        const bool any_live = __any_sync(0xffffffffu, live);
+        float sv[64];
+        float pm = -INFINITY;
+        if (any_live) {
           {
             uint32_t s0[32], s1[32];
-            tmem_ld32(lane_base + C::kS + sb * 64, s0);
-            tmem_ld32(lane_base + C::kS + sb * 64 + 32, s1);
+            tmem_ld32(lane_base + sbuf + hf * 64, s0);
+            tmem_ld32(lane_base + sbuf + hf * 64 + 32, s1);
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               sv[c] = __uint_as_float(s0[c]);
@@ -407,7 +474,7 @@ __global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CU
             }
           }
           // Columns outside [lo, hi] (and every column of a dead row) become
-          // -inf; only tiles with a partial row in this warp pay for it.
+          // -inf; only blocks with a partial row in this warp pay for it.
           if (__any_sync(0xffffffffu, !whole)) {
 #pragma unroll
             for (int c = 0; c < 64; ++c) sv[c] = (live && c >= lo && c <= hi) ? sv[c] : -INFINITY;
@@ -419,14 +486,22 @@ __global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CU
           for (int w2 = 16; w2 >= 1; w2 >>= 1)
 #pragma unroll
             for (int c = 0; c < w2; ++c) t32[c] = fmaxf(t32[c], t32[c + w2]);
-          const float mx = t32[0] * c2;   // c2 > 0: max of scaled = scaled max
-          if (mx > m + 8.0f) {
-            // Raise the running max.  O (from PV up to t-1) is rescaled below,
-            // once PV(t-1) has landed; l is rescaled here.
-            f = (m == -INFINITY) ? 1.0f : ex2(m - mx);
-            l *= f;
-            m = mx;
-          }
+          pm = t32[0] * c2;   // c2 > 0: max of scaled = scaled max
+        }
+        // Both halves have loaded their S columns once the exchange completes,
+        // so P may now be written over S.
+        const float mx = fmaxf(pm, exchange(pm));
+        if (!ok) break;
+        float f = 1.0f;            // factor O must be rescaled by before this PV
+        if (mx > m + 8.0f) {
+          // Raise the running max.  O (earlier PVs) is rescaled below, once
+          // the previous PV has landed; l is rescaled here.
+          f = (m == -INFINITY) ? 1.0f : ex2(m - mx);
+          l *= f;
+          m = mx;
+        }
+        uint32_t pk[32];
+        if (any_live) {
           // A row with no valid key so far keeps m = -inf: use 0 as the
           // offset so its -inf scores give exp2(-inf) = 0, never NaN.
           const float nm = (m == -INFINITY) ? 0.0f : -m;
@@ -447,11 +522,11 @@ __global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CU
 #pragma unroll
           for (int e = 0; e < 32; ++e) pk[e] = 0u;
         }
-        tmem_st32(lane_base + C::kS + sb * 64, pk);
-        // Observe PV(t-1) -- every warp observes every PV completion in order,
+        tmem_st32(lane_base + sbuf + hf * 32, pk);
+        // Observe PV(u-1): every warp observes every PV completion in order,
         // so each parity wait is at most one phase behind the barrier.
-        if (t >= 1) {
-          const long long g = pv_base + t - 1;
+        if (u >= 1) {
+          const long long g = pv_base + u - 1;
           if (!__all_sync(0xffffffffu, mbar_wait(o_done, static_cast<uint32_t>(g & 1), wait_ns, abort_flag))) {
             ok = false;
             break;
@@ -460,7 +535,7 @@ __global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CU
         if (__any_sync(0xffffffffu, f != 1.0f)) {
           tc_fence_after();
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
+          for (int c0 = hf * (D / 2); c0 < (hf + 1) * (D / 2); c0 += 32) {
             uint32_t o32[32];
             tmem_ld32(lane_base + C::kO + c0, o32);
 #pragma unroll
@@ -471,32 +546,44 @@ __global__ void __launch_bounds__(192, 1) attn_kernel(const __grid_constant__ CU
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full(sb));
+        if (lane == 0) mbar_arrive(p_full(b));
       }
       if (!ok) break;
-      // ---- epilogue
-      if (it.ntiles >= 1) {
-        const long long g = pv_base + it.ntiles - 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(o_done, static_cast<uint32_t>(g & 1), wait_ns, abort_flag))) { ok = false; break; }
+      {
+        // The item's last PV has landed.
+        const long long g = pv_base + npair - 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(o_done, static_cast<uint32_t>(g & 1), wait_ns, abort_flag))) {
+          ok = false;
+          break;
+        }
+        pv_base += npair;
       }
+      // ---- row sum over both halves
+      const float L = l + exchange(l);
+      if (!ok) break;
+      const float inv_l = 1.0f / L;
+      float lin_scale = 0.f;
       if constexpr (HYB) {
-        if (!__all_sync(0xffffffffu, mbar_wait(lin_done, ic & 1, wait_ns, abort_flag))) { ok = false; break; }
+        const float gate = P.s != nullptr ? __ldg(P.s + it.b) : P.gate_override;
+        const float den = xden[(ic & 1) * 128 + r];
+        lin_scale = den > 0.f ? gate / den : 0.f;
+        if (!__all_sync(0xffffffffu, mbar_wait(lin_done, ic & 1, wait_ns, abort_flag))) {
+          ok = false;
+          break;
+        }
       }
       tc_fence_after();
-      pv_base += it.ntiles;
-      float gate = 0.f;
-      if constexpr (HYB) gate = P.s != nullptr ? __ldg(P.s + it.b) : P.gate_override;
-      const float inv_l = 1.0f / l;
-      const float lin_scale = gate / den;
+      // ---- epilogue: this warp writes columns [hf*D/2, (hf+1)*D/2) of the row
       long long out_row = row_pos;
       if (it.slot >= 0 && row_valid) {
-        const int f = row_pos % P.F, pos = row_pos / P.F;
+        const int fr = row_pos % P.F, pos = row_pos / P.F;
         const int y = pos / P.Wh, x = pos % P.Wh;
-        out_row = (static_cast<long long>(f) * P.Hh + y) * P.Wh + x;
+        out_row = (static_cast<long long>(fr) * P.Hh + y) * P.Wh + x;
       }
-      uint4* orow = reinterpret_cast<uint4*>(P.o + (static_cast<long long>(it.bh) * P.N + (row_valid ? out_row : 0)) * D);
+      uint4* orow = reinterpret_cast<uint4*>(
+          P.o + (static_cast<long long>(it.bh) * P.N + (row_valid ? out_row : 0)) * D);
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = hf * (D / 2); c0 < (hf + 1) * (D / 2); c0 += 32) {
         uint32_t o32[32];
         tmem_ld32(lane_base + C::kO + c0, o32);
         float v[32];
@@ -561,8 +648,9 @@ cudaError_t launch_attn_t(const Ctx& c, const AttnArgs& a, const Params& P) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const long long items = static_cast<long long>(BH) * P.npairs;
-  const int grid = static_cast<int>(items < c.num_sms ? items : c.num_sms);
-  attn_kernel<D, HYB><<<grid, 192, C::kSmem, c.stream>>>(mk, mv, mkp, mvp, P);
+  long long grid = items < c.num_sms ? items : c.num_sms;
+  if (grid < 1) grid = 1;
+  attn_kernel<D, HYB><<<static_cast<int>(grid), 320, C::kSmem, c.stream>>>(mk, mv, mkp, mvp, P);
   return cudaGetLastError();
 }
 
@@ -589,7 +677,7 @@ cudaError_t launch_attention(const Ctx& c, const AttnArgs& a) {
   P.lists = a.lists;
   P.counts = a.counts;
   P.list_stride = a.list_stride;
-  P.G = a.G;
+  P.Gimg = static_cast<const __nv_bfloat16*>(a.Gimg);
   P.Z = a.Z;
   P.s = a.s;
   P.gate_override = a.gate_override;
@@ -598,7 +686,7 @@ cudaError_t launch_attention(const Ctx& c, const AttnArgs& a) {
   P.o = static_cast<__nv_bfloat16*>(a.o);
   P.err = c.err;
   P.wait_ns = c.wait_ns;
-  const bool hyb = a.G != nullptr;
+  const bool hyb = a.Gimg != nullptr;
   if (a.d == 128) return hyb ? launch_attn_t<128, true>(c, a, P) : launch_attn_t<128, false>(c, a, P);
   return hyb ? launch_attn_t<64, true>(c, a, P) : launch_attn_t<64, false>(c, a, P);
 }

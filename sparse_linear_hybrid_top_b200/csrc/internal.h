@@ -39,9 +39,10 @@ cudaError_t launch_pair_union(const Ctx& c, const int32_t* idx, int BH, int nb, 
 size_t linear_state_ws_bytes(int B, int H, int N, int d);
 cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int B, int H, int N,
                                 int d, float* Hst, float* Z, void* ws);
-// G[b,h] = Hst[b,h] W_lin[h]  (float32 [B,H,d,d])
+// G[b,h] = Hst[b,h] W_lin[h], written as bf16 MMA B-operand images
+// [B*H][d*d] (K-major over the row index of G, 128-byte swizzle).
 cudaError_t launch_linear_fold(const Ctx& c, const float* Hst, const void* w_lin, int B, int H,
-                               int d, float* G);
+                               int d, void* Gimg);
 cudaError_t launch_linear_apply(const Ctx& c, const void* q, const float* Hst, const float* Z,
                                 float eps, int B, int H, int N, int d, void* o);
 
@@ -75,8 +76,8 @@ struct AttnArgs {
   const int32_t* lists;       // topk: [B*H*npairs][2*topk] entries j | mask<<16
   const int32_t* counts;      // topk: [B*H*npairs]
   int list_stride;            // 2*topk
-  // Hybrid epilogue (null G = plain normalised attention output).
-  const float* G;             // [B,H,d,d] float32: Hst W_lin
+  // Hybrid epilogue (null Gimg = plain normalised attention output).
+  const void* Gimg;           // bf16 images [B*H][d*d] of Hst W_lin (see launch_linear_fold)
   const float* Z;             // [B,H,d]
   const float* s;             // [B] gate values (device)
   float gate_override;        // used when s is null

@@ -248,10 +248,13 @@ __global__ void linear_reduce_kernel(const float* __restrict__ partH,
   }
 }
 
-// G[bh] = Hst[bh] W_lin[h]  (float32, W_lin in bf16).  16 rows per CTA.
+// G[bh] = Hst[bh] W_lin[h] (float32 accumulation, W_lin in bf16), written as
+// the bf16 B-operand image of D[row][j] += A[row][c] G[c][j]: K-major (K = c),
+// 128-byte swizzle, slab c/64 of d rows x 128 bytes.  16 rows c per CTA.
 __global__ void __launch_bounds__(256) linear_fold_kernel(const float* __restrict__ Hst,
                                                           const __nv_bfloat16* __restrict__ W,
-                                                          int H, int D, float* __restrict__ G) {
+                                                          int H, int D,
+                                                          __nv_bfloat16* __restrict__ Gimg) {
   extern __shared__ float fold_sm[];
   float* hrows = fold_sm;             // [16][D]
   float* wsm = fold_sm + 16 * D;      // [D][D]
@@ -267,7 +270,9 @@ __global__ void __launch_bounds__(256) linear_fold_kernel(const float* __restric
     const int r = e / D, j = e % D;
     float acc = 0.f;
     for (int m = 0; m < D; ++m) acc = fmaf(hrows[r * D + m], wsm[m * D + j], acc);
-    G[bh * D * D + static_cast<long long>(r0 + r) * D + j] = acc;
+    const int c = r0 + r;
+    const uint32_t off = (c / 64) * (D * 128) + sw128_offset(j, c % 64);
+    Gimg[bh * D * D + off / 2] = __float2bfloat16_rn(acc);
   }
 }
 
@@ -452,14 +457,14 @@ cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int 
 }
 
 cudaError_t launch_linear_fold(const Ctx& c, const float* Hst, const void* w_lin, int B, int H,
-                               int d, float* G) {
+                               int d, void* Gimg) {
   const size_t smem = (16 * d + d * d) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(linear_fold_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   linear_fold_kernel<<<dim3(d / 16, B * H), 256, smem, c.stream>>>(
-      Hst, static_cast<const __nv_bfloat16*>(w_lin), H, d, G);
+      Hst, static_cast<const __nv_bfloat16*>(w_lin), H, d, static_cast<__nv_bfloat16*>(Gimg));
   return cudaGetLastError();
 }
 

@@ -209,7 +209,9 @@ salad_status salad_forward(const salad_forward_args* args, salad_stream stream);
 /*
  * Reads and clears the device-side error word after synchronising `stream`.
  * Returns SALAD_ERR_TIMEOUT if any kernel gave up a bounded wait since the
- * last check, SALAD_ERR_CUDA if the stream reports an error, else SALAD_OK.
+ * last check; SALAD_ERR_CUDA if the stream reports an error or a kernel
+ * refused to run (the attention kernel does when its dynamic shared memory
+ * is not 1024-byte aligned); else SALAD_OK.
  */
 salad_status salad_check_error(salad_stream stream);
 

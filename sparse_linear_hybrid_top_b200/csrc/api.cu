@@ -498,7 +498,7 @@ salad_status salad_check_error(salad_stream stream) {
     const unsigned zero = 0;
     if (cudaMemcpy(c.err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
       return SALAD_ERR_CUDA;
-    return SALAD_ERR_TIMEOUT;
+    return (word & kErrTimeout) ? SALAD_ERR_TIMEOUT : SALAD_ERR_CUDA;
   }
   return SALAD_OK;
 }

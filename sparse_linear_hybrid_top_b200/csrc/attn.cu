@@ -68,11 +68,13 @@ struct AT {
   static constexpr int kKRingHalf = kKS * kSlab;         // one d-slab of the K ring
   static constexpr int kKRing = kHalves * kKRingHalf;
   static constexpr int kVRing = kKS * kTile;
-  static constexpr int kGImg = D * D * 2;                // bf16 G image bytes
-  static_assert(kGImg <= 2 * kTile, "G image must fit the V slots of a pair");
-  static constexpr int kXchg = (2 * 2 * 128 + 2 * 128) * 4;  // row max/sum per parity, den per item
-  static constexpr int kBarBytes = 512;
-  static constexpr int kSmemUsed = 1024 + kKRing + kVRing + kXchg + kBarBytes;
+  static constexpr int kGImg = D * D * 2;                // bf16 G image bytes (own buffer)
+  static constexpr int kXchg = (2 * 2 * 128 + 128) * 4;  // row max/sum per parity, den
+  static constexpr int kBarBytes = 256;
+  // The dynamic shared memory is declared 1024-byte aligned (the 128-byte
+  // swizzle atoms need it), so no slack is reserved for aligning it.
+  static constexpr int kSmemUsed = kKRing + kVRing + kGImg + kXchg + kBarBytes;
+  static_assert(kSmemUsed <= 227 * 1024, "shared memory budget");
   // At least ~half of the SM's shared memory, so one CTA (and its 512 TMEM
   // columns) occupies each SM.
   static constexpr int kSmem = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
@@ -152,10 +154,28 @@ __device__ __forceinline__ void tile_of(const Item& it, int t, int mode, int& j,
   }
 }
 
+// Maximum of 64 values by a tree of three-input maxima (64 -> 22 -> 8 -> 3 -> 1).
+__device__ __forceinline__ float max64(const float* v) {
+  float a[22];
+#pragma unroll
+  for (int i = 0; i < 21; ++i) a[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  a[21] = v[63];
+  float b[8];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) b[i] = fmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  b[7] = a[21];
+  return fmax3(fmax3(b[0], b[1], b[2]), fmax3(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Bulk prefetch of [src, src + bytes) into L2 (16-byte aligned, multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // Untiled bulk copy global -> shared completing on `bar` (16-byte aligned).
@@ -176,16 +196,22 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
                                                       const __grid_constant__ Params P) {
   using C = AT<D, HYB>;
   constexpr int NP = C::kPairs;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* sm = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // The layout below assumes the declared alignment; refuse to run without it.
+  if (reinterpret_cast<uintptr_t>(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(P.err, kErrLayout);
+    return;
+  }
+  unsigned char* sm = smem_raw;
   unsigned char* kring = sm;                         // [d-slab][kKS x 64 rows x 128 B]
   unsigned char* vring = sm + C::kKRing;             // [kKS][d-slab][64 rows x 128 B]
-  float* xrow = reinterpret_cast<float*>(vring + C::kVRing);  // [parity][half][128] row max / sum
-  float* xden = xrow + 2 * 2 * 128;                            // [item parity][128]
+  unsigned char* gbuf = vring + C::kVRing;           // G image of the current item's head
+  float* xrow = reinterpret_cast<float*>(gbuf + C::kGImg);    // [parity][half][128] row max / sum
+  float* xden = xrow + 2 * 2 * 128;                            // [128] phi(q) . Z + eps
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(xrow) + C::kXchg);
-  // bars: full[NP] empty[NP] s_full[2] p_full[2] o_done q_ready lin_done drain x_row[4]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NP + 12);
+  // bars: full[NP] empty[NP] s_full[2] p_full[2] o_done q_ready lin_done drain x_row[4] g_full
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NP + 13);
+  static_assert((2 * NP + 13) * 8 + 8 <= C::kBarBytes, "barrier region");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   auto full = [&](int p) { return smem_u32(bars + p); };
@@ -197,6 +223,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
   const uint32_t lin_done = smem_u32(bars + 2 * NP + 6);
   const uint32_t drain = smem_u32(bars + 2 * NP + 7);
   auto x_row = [&](int q) { return smem_u32(bars + 2 * NP + 8 + q); };
+  const uint32_t g_full = smem_u32(bars + 2 * NP + 12);
   // Shared-memory addresses of the blocks of ring stage (pair) p.
   auto k_addr = [&](int p, int half) {   // rows of block 2p (then 2p+1) of one d-slab
     return smem_u32(kring + half * C::kKRingHalf + 2 * p * kSlab);
@@ -223,6 +250,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
     mbar_init(lin_done, 1);
     mbar_init(drain, 1);
     for (int q = 0; q < 4; ++q) mbar_init(x_row(q), 2);   // the two warps of a row quarter
+    mbar_init(g_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_map(&mk);
@@ -252,7 +280,18 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         const CUtensorMap* vm = it.slot >= 0 ? &mvp : &mv;
         const int z = it.slot >= 0 ? it.b * P.Hs + it.slot : it.bh;
         const int npair = (it.ntiles + 1) / 2;
-        for (int u = 0; u < npair + (HYB ? 1 : 0); ++u, ++pc) {
+        if (w + gridDim.x < total) {
+          // The next item's rows of Q into L2 (one contiguous run), an item
+          // ahead of the softmax warps that load them.
+          const Item nx = make_item(P, w + gridDim.x);
+          const __nv_bfloat16* qsrc =
+              nx.slot >= 0 ? P.qp + (static_cast<long long>(nx.b) * P.Hs + nx.slot) * P.N * D
+                           : P.q + static_cast<long long>(nx.bh) * P.N * D;
+          const int rows = min(128, P.N - nx.p * 128);
+          prefetch_l2(qsrc + static_cast<long long>(nx.p) * 128 * D,
+                      static_cast<uint32_t>(rows) * D * 2);
+        }
+        for (int u = 0; u < npair; ++u, ++pc) {
           const int p = static_cast<int>(pc % NP);
           const long long n = pc / NP;
           if (n > 0 && !mbar_wait(empty(p), static_cast<uint32_t>((n - 1) & 1), wait_ns, abort_flag)) {
@@ -272,11 +311,6 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
                 tma_load_3d(v_addr(p, x) + hh * kSlab, vm, full(p), hh * 64, j * 64, z);
               }
             }
-          } else {
-            // The G image of the item's head, in the V slots of this stage.
-            mbar_arrive_expect_tx(full(p), C::kGImg);
-            bulk_load(v_addr(p, 0), P.Gimg + static_cast<long long>(it.bh) * D * D, C::kGImg,
-                      full(p));
           }
         }
       }
@@ -345,18 +379,17 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         if (!ok) break;
         pc += npair;
         if constexpr (HYB) {
-          // Linear term into S_0 (free once the last PV has run): L = phi(Q) G.
-          if (!wait_full(pc)) { ok = false; break; }
+          // Linear term into S_0 (free once the last PV has run): L = phi(Q) G,
+          // B = the item's G image in its own buffer.
+          if (!mbar_wait(g_full, ic & 1, wait_ns, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t gaddr = v_addr(static_cast<int>(pc % NP), 0);
+          const uint32_t gaddr = smem_u32(gbuf);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
             mma_ts(tmem + C::kL, tmem + C::kPQ + ks * 8,
                    sdesc_sw128(gaddr + (ks / 4) * (D * 128) + (ks % 4) * 32, 16, 1024), idesc_lin,
                    ks > 0 ? 1u : 0u);
-          mma_commit(empty(static_cast<int>(pc % NP)));
           mma_commit(lin_done);
-          ++pc;
         }
       }
       if (!ok) raise_timeout(P.err, abort_flag);
@@ -372,6 +405,17 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
     uint32_t ic = 0, sf[2] = {0, 0}, xc = 0;
     long long pv_base = 0;                      // PVs completed before this item
     bool ok = true;
+    // One thread streams each item's G image into its buffer: the first now,
+    // each next one as soon as the linear term of the current item is done.
+    const bool g_loader = HYB && warp == 2 && lane == 0;
+    long long g_issued = 0;
+    auto load_g = [&](long long w) {
+      const Item nx = make_item(P, w);
+      mbar_arrive_expect_tx(g_full, C::kGImg);
+      bulk_load(smem_u32(gbuf), P.Gimg + static_cast<long long>(nx.bh) * D * D, C::kGImg, g_full);
+      ++g_issued;
+    };
+    if (g_loader && blockIdx.x < total) load_g(blockIdx.x);
     // Exchange of a per-row value with the other half's warp of this quarter.
     auto exchange = [&](float mine) -> float {
       float* slot = xrow + (xc & 1) * 256;
@@ -391,11 +435,20 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
       const int row_pos = it.p * 128 + r;        // position in the head's (possibly regrouped) order
       const bool row_valid = row_pos < P.N;
       const int npair = (it.ntiles + 1) / 2;
+      float den_row = 0.f;   // phi(q) . Z + eps of the row
       if (hf == 1) {
         // This warp's previous epilogue is complete: O, S and the linear
         // term may be overwritten by this item's MMAs.
         __syncwarp();
         if (lane == 0) mbar_arrive(q_ready);
+        // Half 0 has written den for this item once q_ready completes; it
+        // writes the next one only after this item's last PV, which needs
+        // this warp's P, so the single slot is safe to read here.
+        if (!__all_sync(0xffffffffu, mbar_wait(q_ready, ic & 1, wait_ns, abort_flag))) {
+          ok = false;
+          break;
+        }
+        if constexpr (HYB) den_row = xden[r];
       } else {
         // ---- Q and phi(Q) into TMEM (A operands); den = phi(q) . Z + eps
         const __nv_bfloat16* qsrc =
@@ -425,7 +478,8 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
             tmem_st16(lane_base + C::kPQ + c0, pk);
           }
         }
-        xden[(ic & 1) * 128 + r] = den + P.eps;
+        den_row = den + P.eps;
+        xden[r] = den_row;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -464,14 +518,10 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         float pm = -INFINITY;
         if (any_live) {
           {
-            uint32_t s0[32], s1[32];
-            tmem_ld32(lane_base + sbuf + hf * 64, s0);
-            tmem_ld32(lane_base + sbuf + hf * 64 + 32, s1);
+            uint32_t s64[64];
+            tmem_ld64(lane_base + sbuf + hf * 64, s64);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              sv[c] = __uint_as_float(s0[c]);
-              sv[c + 32] = __uint_as_float(s1[c]);
-            }
+            for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(s64[c]);
           }
           // Columns outside [lo, hi] (and every column of a dead row) become
           // -inf; only blocks with a partial row in this warp pay for it.
@@ -479,14 +529,8 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
 #pragma unroll
             for (int c = 0; c < 64; ++c) sv[c] = (live && c >= lo && c <= hi) ? sv[c] : -INFINITY;
           }
-          float t32[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) t32[c] = fmaxf(sv[c], sv[c + 32]);
-#pragma unroll
-          for (int w2 = 16; w2 >= 1; w2 >>= 1)
-#pragma unroll
-            for (int c = 0; c < w2; ++c) t32[c] = fmaxf(t32[c], t32[c + w2]);
-          pm = t32[0] * c2;   // c2 > 0: max of scaled = scaled max
+          // Row max by a tree of three-input maxima (64 -> 22 -> 8 -> 3 -> 1).
+          pm = max64(sv) * c2;   // c2 > 0: max of scaled = scaled max
         }
         // Both halves have loaded their S columns once the exchange completes,
         // so P may now be written over S.
@@ -565,12 +609,14 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
       float lin_scale = 0.f;
       if constexpr (HYB) {
         const float gate = P.s != nullptr ? __ldg(P.s + it.b) : P.gate_override;
-        const float den = xden[(ic & 1) * 128 + r];
+        const float den = den_row;
         lin_scale = den > 0.f ? gate / den : 0.f;
         if (!__all_sync(0xffffffffu, mbar_wait(lin_done, ic & 1, wait_ns, abort_flag))) {
           ok = false;
           break;
         }
+        // The linear term has read G: the next item's image may replace it.
+        if (g_loader && w + gridDim.x < total) load_g(w + gridDim.x);
       }
       tc_fence_after();
       // ---- epilogue: this warp writes columns [hf*D/2, (hf+1)*D/2) of the row
@@ -610,6 +656,11 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
       tc_fence_before();
     }
     if (!ok) raise_timeout(P.err, abort_flag);
+    // Drain the last G load before the CTA leaves (it has landed already
+    // unless a wait above ran out).
+    if (g_loader && g_issued > 0 &&
+        !mbar_wait(g_full, static_cast<uint32_t>((g_issued - 1) & 1), wait_ns, nullptr))
+      atomicOr(P.err, kErrTimeout);
   }
   tc_fence_before();
   __syncthreads();

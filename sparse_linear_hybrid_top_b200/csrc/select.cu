@@ -67,55 +67,68 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
 }
 
 // ----------------------------------------------------------------- score --
-// S[bh][i][j] = sum_c qbar[bh][i][c] * kbar[bh][j][c]; 64 x 64 tile per CTA,
-// 4 x 4 outputs per thread, float64.
-constexpr int kST = 64;   // tile edge
-constexpr int kSK = 16;   // c-chunk
-__global__ void __launch_bounds__(256) score_kernel(const double* __restrict__ qbar,
+// S[bh][i][j] = sum_c qbar[bh][i][c] * kbar[bh][j][c] in float64, each sum
+// taken in ascending c.  64 (i) x 128 (j) tile per CTA of 128 threads, 8 x 8
+// outputs per thread: rows 2*ty + {0,1} + 16a, columns 2*tx + {0,1} + 32b, so
+// the 16-byte shared loads of a warp cover contiguous banks.
+constexpr int kSI = 64;    // tile rows (query blocks)
+constexpr int kSJ = 128;   // tile columns (key blocks)
+constexpr int kSK = 16;    // c-chunk staged per step
+constexpr int kSPad = 2;   // row padding (keeps 16-byte alignment, spreads banks)
+__global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ qbar,
                                                     const double* __restrict__ kbar, int nb,
                                                     int D, double* __restrict__ S) {
-  __shared__ __align__(16) double qs[kSK][kST + 2];
-  __shared__ __align__(16) double ks[kSK][kST + 2];
+  __shared__ __align__(16) double qs[kSK][kSI + kSPad];
+  __shared__ __align__(16) double ks[kSK][kSJ + kSPad];
   const long long bh = blockIdx.z;
-  const int i0 = blockIdx.y * kST, j0 = blockIdx.x * kST;
+  const int i0 = blockIdx.y * kSI, j0 = blockIdx.x * kSJ;
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   const double* qb = qbar + bh * nb * D;
   const double* kb = kbar + bh * nb * D;
-  double acc[4][4];
+  double acc[8][8];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
   for (int c0 = 0; c0 < D; c0 += kSK) {
-    // 64 rows x 16 cols of each operand: 1024 values, 4 per thread.
-    for (int e = threadIdx.x; e < kST * kSK; e += 256) {
+    // Rows of each operand, 16 consecutive c per row (128-byte reads).
+    for (int e = threadIdx.x; e < kSI * kSK; e += 128) {
       const int r = e / kSK, cc = e % kSK;
       qs[cc][r] = (i0 + r < nb) ? qb[static_cast<long long>(i0 + r) * D + c0 + cc] : 0.0;
+    }
+    for (int e = threadIdx.x; e < kSJ * kSK; e += 128) {
+      const int r = e / kSK, cc = e % kSK;
       ks[cc][r] = (j0 + r < nb) ? kb[static_cast<long long>(j0 + r) * D + c0 + cc] : 0.0;
     }
     __syncthreads();
 #pragma unroll
     for (int cc = 0; cc < kSK; ++cc) {
-      double qa[4], kk[4];
+      double2 qa[4], kk[4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) qa[a] = qs[cc][ty * 4 + a];
+      for (int a = 0; a < 4; ++a) qa[a] = *reinterpret_cast<const double2*>(&qs[cc][2 * ty + 16 * a]);
 #pragma unroll
-      for (int b = 0; b < 4; ++b) kk[b] = ks[cc][tx * 4 + b];
+      for (int b = 0; b < 4; ++b) kk[b] = *reinterpret_cast<const double2*>(&ks[cc][2 * tx + 32 * b]);
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fma(qa[a], kk[b], acc[a][b]);
+        for (int b = 0; b < 4; ++b) {
+          acc[2 * a][2 * b] = fma(qa[a].x, kk[b].x, acc[2 * a][2 * b]);
+          acc[2 * a][2 * b + 1] = fma(qa[a].x, kk[b].y, acc[2 * a][2 * b + 1]);
+          acc[2 * a + 1][2 * b] = fma(qa[a].y, kk[b].x, acc[2 * a + 1][2 * b]);
+          acc[2 * a + 1][2 * b + 1] = fma(qa[a].y, kk[b].y, acc[2 * a + 1][2 * b + 1]);
+        }
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int i = i0 + ty * 4 + a;
+  for (int a = 0; a < 8; ++a) {
+    const int i = i0 + 2 * ty + 16 * (a / 2) + (a % 2);
     if (i >= nb) continue;
+    double* srow = S + (bh * nb + i) * nb;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int j = j0 + tx * 4 + b;
-      if (j < nb) S[(bh * nb + i) * nb + j] = acc[a][b];
+    for (int b = 0; b < 8; ++b) {
+      const int j = j0 + 2 * tx + 32 * (b / 2) + (b % 2);
+      if (j < nb) srow[j] = acc[a][b];
     }
   }
 }
@@ -304,8 +317,8 @@ cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int
   else
     pool_kernel<64><<<pg, 128, 0, c.stream>>>(static_cast<const uint4*>(q),
                                                static_cast<const uint4*>(k), N, nb, qbar, kbar);
-  dim3 sg((nb + kST - 1) / kST, (nb + kST - 1) / kST, BH);
-  score_kernel<<<sg, 256, 0, c.stream>>>(qbar, kbar, nb, d, S);
+  dim3 sg((nb + kSJ - 1) / kSJ, (nb + kSI - 1) / kSI, BH);
+  score_kernel<<<sg, 128, 0, c.stream>>>(qbar, kbar, nb, d, S);
   // topk: as many warps per CTA as fit 192 KB of staged keys (>= 1).
   const size_t per_warp = static_cast<size_t>(nb) * 8 + 256 * 4;
   int warps = static_cast<int>((192 * 1024) / per_warp);

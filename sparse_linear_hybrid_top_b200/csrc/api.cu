@@ -473,9 +473,7 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   float* Hst = reinterpret_cast<float*>(ws + L.hst);
   float* Z = reinterpret_cast<float*>(ws + L.z);
   void* G = ws + L.g;
-  e = launch_linear_state(c, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin);
-  if (e != cudaSuccess) return SALAD_ERR_CUDA;
-  e = launch_linear_fold(c, Hst, a->w_lin, B, H, d, G);
+  e = launch_linear_state(c, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, a->w_lin, G);
   if (e != cudaSuccess || !mark(3)) return SALAD_ERR_CUDA;
   at.Gimg = G;
   at.Z = Z;

@@ -215,69 +215,6 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
       : "r"(taddr)
       : "memory");
 }
-// A thread's full 128 columns in one load (and one wait).
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x128.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
-      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,"
-      "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
-      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
-      "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
-      "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, "
-      "[%128];\n\t"
-      "tcgen05.wait::ld.sync.aligned;\n"
-      : SALAD_R8(r, 0), SALAD_R8(r, 8), SALAD_R8(r, 16), SALAD_R8(r, 24), SALAD_R8(r, 32),
-        SALAD_R8(r, 40), SALAD_R8(r, 48), SALAD_R8(r, 56), SALAD_R8(r, 64), SALAD_R8(r, 72),
-        SALAD_R8(r, 80), SALAD_R8(r, 88), SALAD_R8(r, 96), SALAD_R8(r, 104), SALAD_R8(r, 112),
-        SALAD_R8(r, 120)
-      : "r"(taddr)
-      : "memory");
-}
-// The same load without its wait: the registers are valid only after
-// tmem_wait_ld128 on the same array, which names them as operands so that no
-// use can be scheduled before the wait.
-__device__ __forceinline__ void tmem_ld128_async(uint32_t taddr, uint32_t (&r)[128]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x128.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
-      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,"
-      "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
-      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
-      "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
-      "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, "
-      "[%128];\n"
-      : SALAD_R8(r, 0), SALAD_R8(r, 8), SALAD_R8(r, 16), SALAD_R8(r, 24), SALAD_R8(r, 32),
-        SALAD_R8(r, 40), SALAD_R8(r, 48), SALAD_R8(r, 56), SALAD_R8(r, 64), SALAD_R8(r, 72),
-        SALAD_R8(r, 80), SALAD_R8(r, 88), SALAD_R8(r, 96), SALAD_R8(r, 104), SALAD_R8(r, 112),
-        SALAD_R8(r, 120)
-      : "r"(taddr)
-      : "memory");
-}
-#define SALAD_RW8(a, o) "+r"(a[o + 0]), "+r"(a[o + 1]), "+r"(a[o + 2]), "+r"(a[o + 3]), \
-                        "+r"(a[o + 4]), "+r"(a[o + 5]), "+r"(a[o + 6]), "+r"(a[o + 7])
-__device__ __forceinline__ void tmem_wait_ld128(uint32_t (&r)[128]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
-               : SALAD_RW8(r, 0), SALAD_RW8(r, 8), SALAD_RW8(r, 16), SALAD_RW8(r, 24),
-                 SALAD_RW8(r, 32), SALAD_RW8(r, 40), SALAD_RW8(r, 48), SALAD_RW8(r, 56),
-                 SALAD_RW8(r, 64), SALAD_RW8(r, 72), SALAD_RW8(r, 80), SALAD_RW8(r, 88),
-                 SALAD_RW8(r, 96), SALAD_RW8(r, 104), SALAD_RW8(r, 112), SALAD_RW8(r, 120)
-               :
-               : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
-      "tcgen05.wait::ld.sync.aligned;\n"
-      : SALAD_R8(r, 0), SALAD_R8(r, 8)
-      : "r"(taddr)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -286,29 +223,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       SALAD_W8(r, 0), SALAD_W8(r, 8), SALAD_W8(r, 16), SALAD_W8(r, 24)
       : "memory");
 }
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
-      "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
-      "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};\n" ::"r"(taddr),
-      SALAD_W8(r, 0), SALAD_W8(r, 8), SALAD_W8(r, 16), SALAD_W8(r, 24), SALAD_W8(r, 32),
-      SALAD_W8(r, 40), SALAD_W8(r, 48), SALAD_W8(r, 56)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(taddr),
       SALAD_W8(r, 0), SALAD_W8(r, 8)
       : "memory");
-}
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(
-                   taddr),
-               SALAD_W8(r, 0)
-               : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");

@@ -5,7 +5,8 @@
 // and a sigmoid:  s_b = sigmoid(w . mean_n X[b, n, :] + bias).
 // Because the map is linear, w . mean_n X = (1/N) sum_{n,c} w_c X[b,n,c]: one
 // streaming pass over X (the only HBM traffic), a per-CTA partial in float32,
-// then a fixed-order float64 sum of the partials (deterministic).
+// then a fixed-order float64 sum of the partials (deterministic: the
+// partition depends only on B, N, D and the SM count).
 #include "common.cuh"
 #include "internal.h"
 
@@ -73,6 +74,57 @@ __global__ void __launch_bounds__(kGateThreads) gate_partial_kernel(
   }
 }
 
+// Column-resident variant, used when D/8 is a multiple of 32 and at most
+// 1024: thread c owns 16-byte column chunk c of every row, so its 8 weights
+// stay in registers; CTA (part, b) streams rows [part*rows_per, ...) of X[b]
+// with kGateRowUnroll independent 16-byte loads in flight per thread.
+constexpr int kGateRowUnroll = 8;
+__global__ void gate_rows_kernel(const uint4* __restrict__ x, const uint4* __restrict__ w, int N,
+                                 int rows_per, float* __restrict__ partial) {
+  const int CD = blockDim.x;
+  const int b = blockIdx.y;
+  const int c = threadIdx.x;
+  const uint4 wv = __ldg(w + c);
+  const int r0 = blockIdx.x * rows_per;
+  const int r1 = min(N, r0 + rows_per);
+  const uint4* xb = x + (static_cast<long long>(b) * N) * CD + c;
+  float acc = 0.f;
+  int r = r0;
+  for (; r + kGateRowUnroll <= r1; r += kGateRowUnroll) {
+    uint4 xv[kGateRowUnroll];
+#pragma unroll
+    for (int u = 0; u < kGateRowUnroll; ++u)
+      xv[u] = __ldcs(xb + static_cast<long long>(r + u) * CD);
+#pragma unroll
+    for (int u = 0; u < kGateRowUnroll; ++u) acc += dot8(xv[u], wv);
+  }
+  for (; r < r1; ++r) acc += dot8(__ldcs(xb + static_cast<long long>(r) * CD), wv);
+  // Block reduction (fixed order).
+  __shared__ float red[32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int i = 0; i < CD / 32; ++i) t += red[i];
+    partial[static_cast<long long>(b) * gridDim.x + blockIdx.x] = t;
+  }
+}
+
+bool gate_rows_ok(int D) { return D % 256 == 0 && D / 8 <= 1024; }
+
+// Row-split CTAs per sample for gate_rows_kernel: about as many CTAs as fit
+// on the device at once, at least 8 rows each.
+int gate_rows_parts(int B, int N, int D, int num_sms) {
+  const int per_sm = 2048 / (D / 8);
+  long long want = (static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1) + B - 1) / B;
+  const long long cap = (N + 7) / 8;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  return static_cast<int>(want);
+}
+
 __global__ void gate_final_kernel(const float* __restrict__ partial, int nparts, int N,
                                   float bias, float* __restrict__ s) {
   const int b = blockIdx.x;
@@ -109,18 +161,30 @@ int gate_ctas_per_b(int B, int N, int D, int num_sms) {
 }  // namespace
 
 size_t gate_ws_bytes(int B, int N, int D) {
-  // Sized for the largest grid the launch can pick (up to 8 CTAs per SM on a
-  // 256-SM part), independent of the device.
-  return align256(static_cast<size_t>(B) * gate_ctas_per_b(B, N, D, 256) * sizeof(float));
+  // Sized for the largest grid either kernel can pick on a part with up to
+  // 256 SMs, independent of the device.
+  const int parts = gate_rows_ok(D) ? gate_rows_parts(B, N, D, 256) : gate_ctas_per_b(B, N, D, 256);
+  return align256(static_cast<size_t>(B) * parts * sizeof(float));
 }
 
 cudaError_t launch_gate(const Ctx& c, const void* x, const void* w, float bias, int B, int N,
                         int D, float* s, void* ws) {
-  const int nparts = gate_ctas_per_b(B, N, D, c.num_sms < 256 ? c.num_sms : 256);
-  const long long chunks_per_b = static_cast<long long>(N) * (D / 8);
+  const int sms = c.num_sms < 256 ? c.num_sms : 256;
   float* partial = static_cast<float*>(ws);
-  gate_partial_kernel<<<dim3(nparts, B), kGateThreads, 0, c.stream>>>(
-      static_cast<const uint4*>(x), static_cast<const uint4*>(w), chunks_per_b, D / 8, partial);
+  int nparts;
+  if (gate_rows_ok(D)) {
+    nparts = gate_rows_parts(B, N, D, sms);
+    // Whole unrolled groups per CTA; no empty CTA.
+    const int rows_per = ((N + nparts - 1) / nparts + kGateRowUnroll - 1) / kGateRowUnroll * kGateRowUnroll;
+    nparts = (N + rows_per - 1) / rows_per;
+    gate_rows_kernel<<<dim3(nparts, B), D / 8, 0, c.stream>>>(
+        static_cast<const uint4*>(x), static_cast<const uint4*>(w), N, rows_per, partial);
+  } else {
+    nparts = gate_ctas_per_b(B, N, D, sms);
+    const long long chunks_per_b = static_cast<long long>(N) * (D / 8);
+    gate_partial_kernel<<<dim3(nparts, B), kGateThreads, 0, c.stream>>>(
+        static_cast<const uint4*>(x), static_cast<const uint4*>(w), chunks_per_b, D / 8, partial);
+  }
   gate_final_kernel<<<B, 256, 0, c.stream>>>(partial, nparts, N, bias, s);
   return cudaGetLastError();
 }

@@ -37,12 +37,12 @@ cudaError_t launch_pair_union(const Ctx& c, const int32_t* idx, int BH, int nb, 
 
 // ---- linear branch (linear.cu)
 size_t linear_state_ws_bytes(int B, int H, int N, int d);
-cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int B, int H, int N,
-                                int d, float* Hst, float* Z, void* ws);
+// Hst = phi(K)^T V and Z = phi(K)^T 1 per (b, h).  With w_lin given, also
 // G[b,h] = Hst[b,h] W_lin[h], written as bf16 MMA B-operand images
-// [B*H][d*d] (K-major over the row index of G, 128-byte swizzle).
-cudaError_t launch_linear_fold(const Ctx& c, const float* Hst, const void* w_lin, int B, int H,
-                               int d, void* Gimg);
+// [B*H][d*d] (K-major over the row index of G, 128-byte swizzle) into Gimg.
+cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int B, int H, int N,
+                                int d, float* Hst, float* Z, void* ws,
+                                const void* w_lin = nullptr, void* Gimg = nullptr);
 cudaError_t launch_linear_apply(const Ctx& c, const void* q, const float* Hst, const float* Z,
                                 float eps, int B, int H, int N, int d, void* o);
 
@@ -77,7 +77,7 @@ struct AttnArgs {
   const int32_t* counts;      // topk: [B*H*npairs]
   int list_stride;            // 2*topk
   // Hybrid epilogue (null Gimg = plain normalised attention output).
-  const void* Gimg;           // bf16 images [B*H][d*d] of Hst W_lin (see launch_linear_fold)
+  const void* Gimg;           // bf16 images [B*H][d*d] of Hst W_lin (see launch_linear_state)
   const float* Z;             // [B,H,d]
   const float* s;             // [B] gate values (device)
   float gate_override;        // used when s is null

@@ -248,31 +248,50 @@ __global__ void linear_reduce_kernel(const float* __restrict__ partH,
   }
 }
 
-// G[bh] = Hst[bh] W_lin[h] (float32 accumulation, W_lin in bf16), written as
-// the bf16 B-operand image of D[row][j] += A[row][c] G[c][j]: K-major (K = c),
-// 128-byte swizzle, slab c/64 of d rows x 128 bytes.  16 rows c per CTA.
-__global__ void __launch_bounds__(256) linear_fold_kernel(const float* __restrict__ Hst,
-                                                          const __nv_bfloat16* __restrict__ W,
-                                                          int H, int D,
-                                                          __nv_bfloat16* __restrict__ Gimg) {
-  extern __shared__ float fold_sm[];
-  float* hrows = fold_sm;             // [16][D]
-  float* wsm = fold_sm + 16 * D;      // [D][D]
+// The linear state's reduction fused with the fold of W_lin, for the forward
+// pass.  CTA (x, bh): rows [4x, 4x + 4) of Hst[bh] = sum of the per-CTA
+// partials in ascending order (written out, as by linear_reduce_kernel), Z[bh]
+// in CTA x = 0, then rows [4x, 4x + 4) of G[bh] = Hst[bh] W_lin[h] (float32
+// accumulation in ascending m, W_lin in bf16) written as the bf16 B-operand
+// image of D[row][j] += A[row][c] G[c][j]: K-major (K = c), 128-byte swizzle,
+// slab c/64 of d rows x 128 bytes.
+constexpr int kFoldRows = 4;
+__global__ void __launch_bounds__(256) linear_reduce_fold_kernel(
+    const float* __restrict__ partH, const float* __restrict__ partZ, int H, int D, int cph,
+    const __nv_bfloat16* __restrict__ W, float* __restrict__ Hst, float* __restrict__ Z,
+    __nv_bfloat16* __restrict__ Gimg) {
+  extern __shared__ __align__(16) float fold_sm[];
+  float* hrows = fold_sm;                                                       // [4][D]
+  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(fold_sm + kFoldRows * D);  // [D][D]
   const long long bh = blockIdx.y;
   const int h = static_cast<int>(bh % H);
-  const int r0 = blockIdx.x * 16;
-  for (int e = threadIdx.x; e < 16 * D; e += 256)
-    hrows[e] = Hst[bh * D * D + static_cast<long long>(r0) * D + e];
-  for (int e = threadIdx.x; e < D * D; e += 256)
-    wsm[e] = __bfloat162float(W[static_cast<long long>(h) * D * D + e]);
+  const int r0 = blockIdx.x * kFoldRows;
+  const int DD = D * D;
+  const uint4* wsrc = reinterpret_cast<const uint4*>(W + static_cast<long long>(h) * DD);
+  for (int e = threadIdx.x; e < DD / 8; e += blockDim.x)
+    reinterpret_cast<uint4*>(wsm)[e] = __ldg(wsrc + e);
+  for (int e = threadIdx.x; e < kFoldRows * D; e += blockDim.x) {
+    const long long off = static_cast<long long>(r0) * D + e;
+    float acc = 0.f;
+    for (int c = 0; c < cph; ++c) acc += partH[(bh * cph + c) * DD + off];
+    hrows[e] = acc;
+    Hst[bh * DD + off] = acc;
+  }
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e < D; e += blockDim.x) {
+      float acc = 0.f;
+      for (int c = 0; c < cph; ++c) acc += partZ[(bh * cph + c) * D + e];
+      Z[bh * D + e] = acc;
+    }
+  }
   __syncthreads();
-  for (int e = threadIdx.x; e < 16 * D; e += 256) {
+  for (int e = threadIdx.x; e < kFoldRows * D; e += blockDim.x) {
     const int r = e / D, j = e % D;
     float acc = 0.f;
-    for (int m = 0; m < D; ++m) acc = fmaf(hrows[r * D + m], wsm[m * D + j], acc);
+    for (int m = 0; m < D; ++m) acc = fmaf(hrows[r * D + m], __bfloat162float(wsm[m * D + j]), acc);
     const int c = r0 + r;
     const uint32_t off = (c / 64) * (D * 128) + sw128_offset(j, c % 64);
-    Gimg[bh * D * D + off / 2] = __float2bfloat16_rn(acc);
+    Gimg[bh * DD + off / 2] = __float2bfloat16_rn(acc);
   }
 }
 
@@ -424,7 +443,8 @@ size_t linear_state_ws_bytes(int B, int H, int N, int d) {
 }
 
 cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int B, int H, int N,
-                                int d, float* Hst, float* Z, void* ws) {
+                                int d, float* Hst, float* Z, void* ws, const void* w_lin,
+                                void* Gimg) {
   const LSPlan p = ls_plan(B, H, N, c.num_sms < 256 ? c.num_sms : 256);
   const int BH = B * H;
   const size_t parts = static_cast<size_t>(BH) * p.ctas_per_head;
@@ -451,20 +471,18 @@ cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int 
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  linear_reduce_kernel<<<dim3((d * d + 255) / 256, BH), 256, 0, c.stream>>>(
-      partH, partZ, d, p.ctas_per_head, Hst, Z);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_linear_fold(const Ctx& c, const float* Hst, const void* w_lin, int B, int H,
-                               int d, void* Gimg) {
-  const size_t smem = (16 * d + d * d) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(linear_fold_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  if (w_lin == nullptr) {
+    linear_reduce_kernel<<<dim3((d * d + 255) / 256, BH), 256, 0, c.stream>>>(
+        partH, partZ, d, p.ctas_per_head, Hst, Z);
+    return cudaGetLastError();
+  }
+  const size_t smem = kFoldRows * d * sizeof(float) + static_cast<size_t>(d) * d * 2;
+  e = cudaFuncSetAttribute(linear_reduce_fold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  linear_fold_kernel<<<dim3(d / 16, B * H), 256, smem, c.stream>>>(
-      Hst, static_cast<const __nv_bfloat16*>(w_lin), H, d, static_cast<__nv_bfloat16*>(Gimg));
+  linear_reduce_fold_kernel<<<dim3(d / kFoldRows, BH), 256, smem, c.stream>>>(
+      partH, partZ, H, d, p.ctas_per_head, static_cast<const __nv_bfloat16*>(w_lin), Hst, Z,
+      static_cast<__nv_bfloat16*>(Gimg));
   return cudaGetLastError();
 }
 

@@ -68,56 +68,82 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
 
 // ----------------------------------------------------------------- score --
 // S[bh][i][j] = sum_c qbar[bh][i][c] * kbar[bh][j][c] in float64, each sum
-// taken in ascending c.  64 (i) x 128 (j) tile per CTA of 128 threads, 8 x 8
-// outputs per thread: rows 2*ty + {0,1} + 16a, columns 2*tx + {0,1} + 32b, so
-// the 16-byte shared loads of a warp cover contiguous banks.
-constexpr int kSI = 64;    // tile rows (query blocks)
-constexpr int kSJ = 128;   // tile columns (key blocks)
+// taken in ascending c.  64 x 64 tile per CTA of 128 threads, 8 (rows) x 4
+// (columns) outputs per thread: rows 2*ty + {0,1} + 16a, columns 2*tx +
+// {0,1} + 32b, so each 16-byte shared load of a half-warp covers contiguous
+// banks.  The c dimension is staged 16 at a time through two shared buffers;
+// the next chunk is read from global memory into registers while the current
+// one is multiplied.
+constexpr int kST = 64;    // tile edge
 constexpr int kSK = 16;    // c-chunk staged per step
 constexpr int kSPad = 2;   // row padding (keeps 16-byte alignment, spreads banks)
-__global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ qbar,
+__global__ void __launch_bounds__(128, 4) score_kernel(const double* __restrict__ qbar,
                                                     const double* __restrict__ kbar, int nb,
                                                     int D, double* __restrict__ S) {
-  __shared__ __align__(16) double qs[kSK][kSI + kSPad];
-  __shared__ __align__(16) double ks[kSK][kSJ + kSPad];
+  __shared__ __align__(16) double qs[2][kSK][kST + kSPad];
+  __shared__ __align__(16) double ks[2][kSK][kST + kSPad];
   const long long bh = blockIdx.z;
-  const int i0 = blockIdx.y * kSI, j0 = blockIdx.x * kSJ;
+  const int i0 = blockIdx.y * kST, j0 = blockIdx.x * kST;
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   const double* qb = qbar + bh * nb * D;
   const double* kb = kbar + bh * nb * D;
-  double acc[8][8];
+  // Staging: thread t moves elements (row t/8 + 16v, c-pair t%8) of each
+  // operand, v = 0..3: 16-byte reads, 128 bytes per row.
+  const int sr = threadIdx.x / 8, sc = 2 * (threadIdx.x % 8);
+  double2 gq[4], gk[4];
+  auto fetch = [&](int c0) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int r = sr + 16 * v;
+      gq[v] = (i0 + r < nb) ? *reinterpret_cast<const double2*>(qb + static_cast<long long>(i0 + r) * D + c0 + sc)
+                            : make_double2(0.0, 0.0);
+      gk[v] = (j0 + r < nb) ? *reinterpret_cast<const double2*>(kb + static_cast<long long>(j0 + r) * D + c0 + sc)
+                            : make_double2(0.0, 0.0);
+    }
+  };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int r = sr + 16 * v;
+      qs[buf][sc][r] = gq[v].x;
+      qs[buf][sc + 1][r] = gq[v].y;
+      ks[buf][sc][r] = gk[v].x;
+      ks[buf][sc + 1][r] = gk[v].y;
+    }
+  };
+  double acc[8][4];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
-  for (int c0 = 0; c0 < D; c0 += kSK) {
-    // Rows of each operand, 16 consecutive c per row (128-byte reads).
-    for (int e = threadIdx.x; e < kSI * kSK; e += 128) {
-      const int r = e / kSK, cc = e % kSK;
-      qs[cc][r] = (i0 + r < nb) ? qb[static_cast<long long>(i0 + r) * D + c0 + cc] : 0.0;
-    }
-    for (int e = threadIdx.x; e < kSJ * kSK; e += 128) {
-      const int r = e / kSK, cc = e % kSK;
-      ks[cc][r] = (j0 + r < nb) ? kb[static_cast<long long>(j0 + r) * D + c0 + cc] : 0.0;
-    }
-    __syncthreads();
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+  const int nchunks = D / kSK;
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  for (int ch = 0; ch < nchunks; ++ch) {
+    const int buf = ch & 1;
+    if (ch + 1 < nchunks) fetch((ch + 1) * kSK);
 #pragma unroll
     for (int cc = 0; cc < kSK; ++cc) {
-      double2 qa[4], kk[4];
+      double2 qa[4], kk[2];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) qa[a] = *reinterpret_cast<const double2*>(&qs[cc][2 * ty + 16 * a]);
+      for (int a = 0; a < 4; ++a)
+        qa[a] = *reinterpret_cast<const double2*>(&qs[buf][cc][2 * ty + 16 * a]);
 #pragma unroll
-      for (int b = 0; b < 4; ++b) kk[b] = *reinterpret_cast<const double2*>(&ks[cc][2 * tx + 32 * b]);
+      for (int b = 0; b < 2; ++b)
+        kk[b] = *reinterpret_cast<const double2*>(&ks[buf][cc][2 * tx + 32 * b]);
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
+        for (int b = 0; b < 2; ++b) {
           acc[2 * a][2 * b] = fma(qa[a].x, kk[b].x, acc[2 * a][2 * b]);
           acc[2 * a][2 * b + 1] = fma(qa[a].x, kk[b].y, acc[2 * a][2 * b + 1]);
           acc[2 * a + 1][2 * b] = fma(qa[a].y, kk[b].x, acc[2 * a + 1][2 * b]);
           acc[2 * a + 1][2 * b + 1] = fma(qa[a].y, kk[b].y, acc[2 * a + 1][2 * b + 1]);
         }
     }
+    // The other buffer was last read before the previous barrier.
+    if (ch + 1 < nchunks) stash(buf ^ 1);
     __syncthreads();
   }
 #pragma unroll
@@ -126,7 +152,7 @@ __global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ q
     if (i >= nb) continue;
     double* srow = S + (bh * nb + i) * nb;
 #pragma unroll
-    for (int b = 0; b < 8; ++b) {
+    for (int b = 0; b < 4; ++b) {
       const int j = j0 + 2 * tx + 32 * (b / 2) + (b % 2);
       if (j < nb) srow[j] = acc[a][b];
     }
@@ -202,15 +228,24 @@ __global__ void topk_kernel(const double* __restrict__ S, int nrows, int nb, int
     want -= static_cast<int>(above);
     prefix |= static_cast<unsigned long long>(digit) << shift;
     pmask |= 0xFFull << shift;
+    // Every key that shares the prefix so far is kept: the set is decided
+    // (no tie among kept and dropped keys is left to break).
+    const bool settled = hist[digit] == static_cast<unsigned>(want);
     __syncwarp();
+    if (settled) {
+      want = 0x7fffffff;
+      break;
+    }
   }
-  // prefix is the exact key of the topk-th largest score; keep every larger
-  // key and the first `want` equal keys in index order.
+  // Keep every key whose masked value exceeds the prefix and the first
+  // `want` whose masked value equals it, in index order.  After all eight
+  // passes the mask is full and `prefix` is the exact key of the topk-th
+  // largest score; after an early stop every equal key is kept.
   int32_t* out = idx + row * topk;
   int written = 0, eq_seen = 0;
   for (int j0 = 0; j0 < nb; j0 += 32) {
     const int j = j0 + lane;
-    const unsigned long long key = j < nb ? keys[j] : 0ull;
+    const unsigned long long key = j < nb ? (keys[j] & pmask) : 0ull;
     const bool gt = j < nb && key > prefix;
     const bool eq = j < nb && key == prefix;
     const unsigned eq_ballot = __ballot_sync(0xffffffffu, eq);
@@ -317,7 +352,7 @@ cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int
   else
     pool_kernel<64><<<pg, 128, 0, c.stream>>>(static_cast<const uint4*>(q),
                                                static_cast<const uint4*>(k), N, nb, qbar, kbar);
-  dim3 sg((nb + kSJ - 1) / kSJ, (nb + kSI - 1) / kSI, BH);
+  dim3 sg((nb + kST - 1) / kST, (nb + kST - 1) / kST, BH);
   score_kernel<<<sg, 128, 0, c.stream>>>(qbar, kbar, nb, d, S);
   // topk: as many warps per CTA as fit 192 KB of staged keys (>= 1).
   const size_t per_warp = static_cast<size_t>(nb) * 8 + 256 * 4;

@@ -192,6 +192,13 @@ typedef struct salad_forward_args {
     int F, Hh, Wh;              /* SWA mode: latent grid, F*Hh*Wh == N */
     float eps;                  /* linear-attention denominator eps (1e-6) */
     float gate_override;        /* NaN: use the gate; otherwise s_b = this value */
+    /* Post-training branch dropping ("SALAD ... (paper.rainbus.top)" 方法步骤详情
+     * step 8; "视频扩散模型中的稀疏注意力机制解析" 3.1-3.2): the linear branch
+     * of sample b (state, fold and linear term) is skipped, on the device,
+     * when s_b < drop_threshold; that sample's output is then O_sparse.  The
+     * threshold is calibrated offline (a percentile of gate values).  0 or
+     * NaN: never drop.  +-inf is rejected. */
+    float drop_threshold;
     float* s_out;               /* optional device float32 [B] (out), may be NULL */
     int32_t* idx_out;           /* optional device int32 [B,H,nb,topk] (out), may be NULL */
     void* workspace;            /* device scratch, >= salad_forward_workspace_bytes() */

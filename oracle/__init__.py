@@ -11,12 +11,14 @@ Sources (page title, then section):
     M in {-inf, 0}^{N x N}), Linear Attention (H = phi(K)^T V, Z = phi(K)^T 1,
     O = phi(Q) H / (phi(Q) Z), phi = ReLU); 方法步骤详情 steps 2-6 (sparse branch
     O_s, linear branch O_l, zero-init projection O_l' = ZeroInitProj(O_l),
-    sigmoid gate s, residual O~ = O_s + s * O_l').
+    sigmoid gate s, residual O~ = O_s + s * O_l'), step 8 (optional dropping
+    of linear branches whose gate value is small).
   * "视频扩散模型中的稀疏注意力机制解析 (ijyty.com)": 1.1 (ST-SWA: frame-major
     flattening, per-head regrouping by spatial position, 1-D sliding window),
     1.2 (Top-K: block partition, block mean vectors, similarity to key-block
     means, keep Top-K blocks, attend only to them), 2.3 (gate: token mean ->
-    linear -> sigmoid).
+    linear -> sigmoid), 3.1-3.2 (post-training branch pruning below a
+    gate-value threshold).
 Readings where the pages are silent (each is listed in the design notes):
   softmax scale 1/sqrt(d); query side of the selection pooled per query block;
   block means over valid rows only; no forced blocks; ties broken towards the
@@ -251,13 +253,19 @@ def combine(o_sparse, o_lin, w_lin_h, s: float) -> np.ndarray:
 def forward(inp: Dict, *, mode: str, block: int = 64, topk: int = 0, window: int = 0,
             space_major_heads: Sequence[int] = (), F: int = 0, Hh: int = 0, Wh: int = 0,
             eps: float = 1e-6, gate_override: Optional[float] = None,
-            idx_override: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+            idx_override: Optional[np.ndarray] = None,
+            drop_threshold: float = 0.0) -> Dict[str, np.ndarray]:
     """The whole hybrid layer, in the step order of the method.
 
     inp: q, k, v [B, H, N, d]; x [B, N, D]; w_gate [D]; bias; w_lin [H, d, d].
     mode: "topk" | "swa" | "dense".  ``idx_override`` replaces the selection
     (used when another correct selection is compared at a near tie).
-    Returns s [B], idx [B, H, nb, topk] (topk mode), scores, o_sparse, o_lin, o.
+    ``drop_threshold``: post-training branch dropping ("SALAD ...
+    (paper.rainbus.top)" 方法步骤详情 step 8; "视频扩散模型中的稀疏注意力机制解析"
+    3.1-3.2): a sample whose gate value s_b is below the threshold keeps only
+    its sparse branch, O = O_sparse (0 never drops, since s_b > 0).
+    Returns s [B], idx [B, H, nb, topk] (topk mode), scores, o_sparse, o_lin,
+    o and dropped [B].
     """
     q, k, v = as64(inp["q"]), as64(inp["k"]), as64(inp["v"])
     B, H, N, d = q.shape
@@ -286,9 +294,12 @@ def forward(inp: Dict, *, mode: str, block: int = 64, topk: int = 0, window: int
                 raise ValueError(mode)
             Hst, Z = linear_state(k[b, h], v[b, h])
             o_lin[b, h] = linear_apply(q[b, h], Hst, Z, eps)
-            o[b, h] = combine(o_sparse[b, h], o_lin[b, h], w_lin[h], s[b])
+            if s[b] < drop_threshold:
+                o[b, h] = o_sparse[b, h]
+            else:
+                o[b, h] = combine(o_sparse[b, h], o_lin[b, h], w_lin[h], s[b])
     return {"s": s, "idx": idx, "scores": scores, "o_sparse": o_sparse,
-            "o_lin": o_lin, "o": o}
+            "o_lin": o_lin, "o": o, "dropped": s < drop_threshold}
 
 
 # ------------------------------------------------- selection comparison ---

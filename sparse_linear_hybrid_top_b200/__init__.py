@@ -61,6 +61,7 @@ class ForwardArgs(ctypes.Structure):
         ("space_major_heads", ctypes.c_void_p),
         ("F", ctypes.c_int), ("Hh", ctypes.c_int), ("Wh", ctypes.c_int),
         ("eps", ctypes.c_float), ("gate_override", ctypes.c_float),
+        ("drop_threshold", ctypes.c_float),
         ("s_out", ctypes.c_void_p), ("idx_out", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("phase_events", ctypes.c_void_p),
@@ -290,8 +291,8 @@ class ForwardPlan:
     def __init__(self, q, k, v, x, w_gate, w_lin, *, mode: str = "topk", topk: int = 0,
                  window: int = 0, space_major_heads: Optional[Sequence[int]] = None,
                  F: int = 0, Hh: int = 0, Wh: int = 0, bias: float = 0.0, eps: float = 1e-6,
-                 gate_override: Optional[float] = None, o=None, s_out=None, idx_out=None,
-                 block: int = 64):
+                 gate_override: Optional[float] = None, drop_threshold: float = 0.0, o=None,
+                 s_out=None, idx_out=None, block: int = 64):
         for n, t in (("q", q), ("k", k), ("v", v), ("x", x), ("w_gate", w_gate),
                      ("w_lin", w_lin)):
             _dev_tensor(t, torch.bfloat16, n)
@@ -310,6 +311,9 @@ class ForwardPlan:
         a.F, a.Hh, a.Wh = F, Hh, Wh
         a.eps = float(eps)
         a.gate_override = float("nan") if gate_override is None else float(gate_override)
+        # Post-training branch dropping: sample b's linear branch is skipped
+        # (on the device) when s_b < drop_threshold; 0 never drops.
+        a.drop_threshold = float(drop_threshold)
         a.s_out = _ptr(s_out)
         a.idx_out = _ptr(idx_out)
         need = lib.salad_forward_workspace_bytes(ctypes.byref(a))

@@ -195,7 +195,7 @@ const char* salad_status_string(salad_status s) {
   }
 }
 
-int salad_version(void) { return 100; }
+int salad_version(void) { return 200; }
 
 // ------------------------------------------------------------------ gate --
 size_t salad_gate_workspace_bytes(int B, int N, int D) {
@@ -400,6 +400,7 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   if (a->idx_out != nullptr && !aligned(a->idx_out, 4)) return SALAD_ERR_INVALID_ARG;
   const bool override_gate = !std::isnan(a->gate_override);
   if (override_gate && !std::isfinite(a->gate_override)) return SALAD_ERR_INVALID_ARG;
+  if (std::isinf(a->drop_threshold)) return SALAD_ERR_INVALID_ARG;
   if (a->mode == SALAD_MODE_TOPK && (a->topk < 1 || a->topk > nblocks(a->N)))
     return SALAD_ERR_INVALID_ARG;
   if (a->mode == SALAD_MODE_SWA && a->window < 0) return SALAD_ERR_INVALID_ARG;
@@ -437,6 +438,8 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   at.o = a->o;
   at.eps = a->eps;
   at.s = s;
+  // NaN compares false: never drop.
+  at.drop = std::isnan(a->drop_threshold) ? 0.0f : a->drop_threshold;
   // 2. sparse-branch pattern (ijyty.com 1.1 / 1.2)
   if (a->mode == SALAD_MODE_TOPK) {
     int32_t* idx = a->idx_out != nullptr ? a->idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
@@ -473,7 +476,10 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   float* Hst = reinterpret_cast<float*>(ws + L.hst);
   float* Z = reinterpret_cast<float*>(ws + L.z);
   void* G = ws + L.g;
-  e = launch_linear_state(c, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, a->w_lin, G);
+  BranchDrop drop;
+  drop.s = s;
+  drop.thr = at.drop;
+  e = launch_linear_state(c, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, a->w_lin, G, drop);
   if (e != cudaSuccess || !mark(3)) return SALAD_ERR_CUDA;
   at.Gimg = G;
   at.Z = Z;

@@ -103,6 +103,7 @@ struct Params {
   const float* Z;
   const float* s;
   float gate_override;
+  float drop;                 // the linear term of sample b is skipped when s_b < drop
   float eps;
   float scale_log2;
   __nv_bfloat16* o;
@@ -141,6 +142,13 @@ __device__ __forceinline__ Item make_item(const Params& P, long long w) {
     it.ntiles = hi / 64 - it.jlo + 1;
   }
   return it;
+}
+
+// Whether sample b keeps its linear branch (post-training branch dropping:
+// the branch is skipped when the gate value is below the threshold).
+__device__ __forceinline__ bool lin_on(const Params& P, int b) {
+  const float g = P.s != nullptr ? __ldg(P.s + b) : P.gate_override;
+  return !(g < P.drop);
 }
 
 __device__ __forceinline__ void tile_of(const Item& it, int t, int mode, int& j, int& mask) {
@@ -345,6 +353,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
                  ks > 0 ? 1u : 0u);
         mma_commit(s_full(b));
       };
+      uint32_t lc = 0;   // items with a linear term so far
       for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++ic) {
         const Item it = make_item(P, w);
         const int npair = (it.ntiles + 1) / 2;
@@ -378,10 +387,11 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         }
         if (!ok) break;
         pc += npair;
-        if constexpr (HYB) {
+        if (HYB && lin_on(P, it.b)) {
           // Linear term into S_0 (free once the last PV has run): L = phi(Q) G,
           // B = the item's G image in its own buffer.
-          if (!mbar_wait(g_full, ic & 1, wait_ns, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(g_full, lc & 1, wait_ns, abort_flag)) { ok = false; break; }
+          ++lc;
           tc_fence_after();
           const uint32_t gaddr = smem_u32(gbuf);
 #pragma unroll
@@ -407,15 +417,22 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
     bool ok = true;
     // One thread streams each item's G image into its buffer: the first now,
     // each next one as soon as the linear term of the current item is done.
+    // Items whose sample dropped its linear branch are skipped.
     const bool g_loader = HYB && warp == 2 && lane == 0;
     long long g_issued = 0;
-    auto load_g = [&](long long w) {
-      const Item nx = make_item(P, w);
-      mbar_arrive_expect_tx(g_full, C::kGImg);
-      bulk_load(smem_u32(gbuf), P.Gimg + static_cast<long long>(nx.bh) * D * D, C::kGImg, g_full);
-      ++g_issued;
+    uint32_t lc = 0;   // items with a linear term so far
+    auto load_g = [&](long long from) {
+      for (long long w = from; w < total; w += gridDim.x) {
+        const Item nx = make_item(P, w);
+        if (!lin_on(P, nx.b)) continue;
+        mbar_arrive_expect_tx(g_full, C::kGImg);
+        bulk_load(smem_u32(gbuf), P.Gimg + static_cast<long long>(nx.bh) * D * D, C::kGImg,
+                  g_full);
+        ++g_issued;
+        return;
+      }
     };
-    if (g_loader && blockIdx.x < total) load_g(blockIdx.x);
+    if (g_loader) load_g(blockIdx.x);
     // Exchange of a per-row value with the other half's warp of this quarter.
     auto exchange = [&](float mine) -> float {
       float* slot = xrow + (xc & 1) * 256;
@@ -435,6 +452,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
       const int row_pos = it.p * 128 + r;        // position in the head's (possibly regrouped) order
       const bool row_valid = row_pos < P.N;
       const int npair = (it.ntiles + 1) / 2;
+      const bool lin = HYB && lin_on(P, it.b);   // this item adds the linear term
       float den_row = 0.f;   // phi(q) . Z + eps of the row
       if (hf == 1) {
         // This warp's previous epilogue is complete: O, S and the linear
@@ -448,7 +466,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
           ok = false;
           break;
         }
-        if constexpr (HYB) den_row = xden[r];
+        if (lin) den_row = xden[r];
       } else {
         // ---- Q and phi(Q) into TMEM (A operands); den = phi(q) . Z + eps
         const __nv_bfloat16* qsrc =
@@ -467,7 +485,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
             pk[4 * u + 0] = v.x; pk[4 * u + 1] = v.y; pk[4 * u + 2] = v.z; pk[4 * u + 3] = v.w;
           }
           tmem_st16(lane_base + C::kQ + c0, pk);
-          if constexpr (HYB) {
+          if (lin) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               pk[e] = relu_bf16x2(pk[e]);
@@ -607,16 +625,17 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
       if (!ok) break;
       const float inv_l = 1.0f / L;
       float lin_scale = 0.f;
-      if constexpr (HYB) {
+      if (lin) {
         const float gate = P.s != nullptr ? __ldg(P.s + it.b) : P.gate_override;
         const float den = den_row;
         lin_scale = den > 0.f ? gate / den : 0.f;
-        if (!__all_sync(0xffffffffu, mbar_wait(lin_done, ic & 1, wait_ns, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(lin_done, lc & 1, wait_ns, abort_flag))) {
           ok = false;
           break;
         }
+        ++lc;
         // The linear term has read G: the next item's image may replace it.
-        if (g_loader && w + gridDim.x < total) load_g(w + gridDim.x);
+        if (g_loader) load_g(w + gridDim.x);
       }
       tc_fence_after();
       // ---- epilogue: this warp writes columns [hf*D/2, (hf+1)*D/2) of the row
@@ -635,7 +654,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         float v[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o32[e]) * inv_l;
-        if constexpr (HYB) {
+        if (lin) {
           uint32_t l32[32];
           tmem_ld32(lane_base + C::kL + c0, l32);
 #pragma unroll
@@ -732,6 +751,7 @@ cudaError_t launch_attention(const Ctx& c, const AttnArgs& a) {
   P.Z = a.Z;
   P.s = a.s;
   P.gate_override = a.gate_override;
+  P.drop = a.drop;
   P.eps = a.eps;
   P.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(a.d));
   P.o = static_cast<__nv_bfloat16*>(a.o);

@@ -40,9 +40,18 @@ size_t linear_state_ws_bytes(int B, int H, int N, int d);
 // Hst = phi(K)^T V and Z = phi(K)^T 1 per (b, h).  With w_lin given, also
 // G[b,h] = Hst[b,h] W_lin[h], written as bf16 MMA B-operand images
 // [B*H][d*d] (K-major over the row index of G, 128-byte swizzle) into Gimg.
+// Post-training branch dropping on the device: sample b's linear branch is
+// skipped when its gate value (s[b], or gate_override when s is null) is
+// below thr.  thr = 0 or NaN never drops (gate values are >= 0).
+struct BranchDrop {
+  const float* s = nullptr;
+  float gate_override = 0.0f;
+  float thr = 0.0f;
+};
 cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int B, int H, int N,
                                 int d, float* Hst, float* Z, void* ws,
-                                const void* w_lin = nullptr, void* Gimg = nullptr);
+                                const void* w_lin = nullptr, void* Gimg = nullptr,
+                                BranchDrop drop = BranchDrop());
 cudaError_t launch_linear_apply(const Ctx& c, const void* q, const float* Hst, const float* Z,
                                 float eps, int B, int H, int N, int d, void* o);
 
@@ -81,6 +90,7 @@ struct AttnArgs {
   const float* Z;             // [B,H,d]
   const float* s;             // [B] gate values (device)
   float gate_override;        // used when s is null
+  float drop = 0.0f;          // the linear term of sample b is skipped when s_b < drop
   float eps;
   void* o;                    // bf16 [B,H,N,d]
 };

@@ -36,12 +36,20 @@ struct LS {
   static constexpr int kSmem = 1024 /*align slack*/ + kStages * kStage + kZero + kRed + kBars;
 };
 
+__device__ __forceinline__ bool branch_dropped(const BranchDrop& d, int b) {
+  const float g = d.s != nullptr ? __ldg(d.s + b) : d.gate_override;
+  return g < d.thr;
+}
+
 template <int D>
 __global__ void __launch_bounds__(192, 1) linear_state_kernel(
     const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv, int nblk,
     int blocks_per_cta, int ctas_per_head, float* __restrict__ partH, float* __restrict__ partZ,
-    unsigned* err, unsigned long long wait_ns) {
+    unsigned* err, unsigned long long wait_ns, BranchDrop drop, int H) {
   using C = LS<D>;
+  // A sample whose linear branch is dropped needs no state: the whole CTA
+  // leaves before touching shared memory, barriers or TMEM.
+  if (branch_dropped(drop, static_cast<int>(blockIdx.x / ctas_per_head) / H)) return;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -259,7 +267,8 @@ constexpr int kFoldRows = 4;
 __global__ void __launch_bounds__(256) linear_reduce_fold_kernel(
     const float* __restrict__ partH, const float* __restrict__ partZ, int H, int D, int cph,
     const __nv_bfloat16* __restrict__ W, float* __restrict__ Hst, float* __restrict__ Z,
-    __nv_bfloat16* __restrict__ Gimg) {
+    __nv_bfloat16* __restrict__ Gimg, BranchDrop drop) {
+  if (branch_dropped(drop, static_cast<int>(blockIdx.y) / H)) return;
   extern __shared__ __align__(16) float fold_sm[];
   float* hrows = fold_sm;                                                       // [4][D]
   __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(fold_sm + kFoldRows * D);  // [D][D]
@@ -444,7 +453,7 @@ size_t linear_state_ws_bytes(int B, int H, int N, int d) {
 
 cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int B, int H, int N,
                                 int d, float* Hst, float* Z, void* ws, const void* w_lin,
-                                void* Gimg) {
+                                void* Gimg, BranchDrop drop) {
   const LSPlan p = ls_plan(B, H, N, c.num_sms < 256 ? c.num_sms : 256);
   const int BH = B * H;
   const size_t parts = static_cast<size_t>(BH) * p.ctas_per_head;
@@ -461,13 +470,15 @@ cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int 
                              LS<128>::kSmem);
     if (e != cudaSuccess) return e;
     linear_state_kernel<128><<<grid, 192, LS<128>::kSmem, c.stream>>>(
-        mk, mv, p.nblk, p.blocks_per_cta, p.ctas_per_head, partH, partZ, c.err, c.wait_ns);
+        mk, mv, p.nblk, p.blocks_per_cta, p.ctas_per_head, partH, partZ, c.err, c.wait_ns, drop,
+        H);
   } else {
     e = cudaFuncSetAttribute(linear_state_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              LS<64>::kSmem);
     if (e != cudaSuccess) return e;
     linear_state_kernel<64><<<grid, 192, LS<64>::kSmem, c.stream>>>(
-        mk, mv, p.nblk, p.blocks_per_cta, p.ctas_per_head, partH, partZ, c.err, c.wait_ns);
+        mk, mv, p.nblk, p.blocks_per_cta, p.ctas_per_head, partH, partZ, c.err, c.wait_ns, drop,
+        H);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -482,7 +493,7 @@ cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int 
   if (e != cudaSuccess) return e;
   linear_reduce_fold_kernel<<<dim3(d / kFoldRows, BH), 256, smem, c.stream>>>(
       partH, partZ, H, d, p.ctas_per_head, static_cast<const __nv_bfloat16*>(w_lin), Hst, Z,
-      static_cast<__nv_bfloat16*>(Gimg));
+      static_cast<__nv_bfloat16*>(Gimg), drop);
   return cudaGetLastError();
 }
 

@@ -8,6 +8,8 @@ oracle's only at near ties (k-th and (k+1)-th scores within 1e-5 relative);
 the output is then compared under the GPU's selection.
 Bar: max |err| <= 2e-2, relative L2 <= 5e-3.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -87,6 +89,43 @@ def test_forward_gate_zero_and_zero_projection_give_sparse_branch(salad):
     o0 = _plan(salad, w, dev0).run()
     assert torch.equal(o0, o_sparse)
     salad.check_error()
+
+
+# Two samples, d = 128, ragged N: the batch case of post-training branch
+# dropping (the gate value, and so the decision, is per sample).
+RAGGED128_B2 = dataclasses.replace(RAGGED128, name="ragged128_b2", B=2, seeds=(3, 7))
+
+
+def test_forward_branch_dropping(salad):
+    w = RAGGED128_B2
+    inp = generate(w)
+    # Shift sample 1's hidden state so the two gate values are well apart.
+    inp["x"][1] = (inp["x"][1].float() + 0.5).to(torch.bfloat16)
+    dev = device_inputs(inp)
+    full = _plan(salad, w, dev)
+    o_full = full.run().clone()
+    s = full.s_out.cpu()
+    lo, hi = (0, 1) if s[0] < s[1] else (1, 0)
+    assert s[hi] - s[lo] > 1e-3
+    # Threshold 0 never drops; above both gate values drops both, which is
+    # the sparse branch alone, exactly as a zero gate gives it.
+    o_none = _plan(salad, w, dev, drop_threshold=0.0).run().clone()
+    assert torch.equal(o_none, o_full)
+    o_g0 = _plan(salad, w, dev, gate_override=0.0).run().clone()
+    o_all = _plan(salad, w, dev, drop_threshold=1.0).run().clone()
+    assert torch.equal(o_all, o_g0)
+    # Between the two: only the lower sample loses its linear branch.
+    thr = float(s[lo] + s[hi]) / 2
+    mid = _plan(salad, w, dev, drop_threshold=thr)
+    o_mid = mid.run().clone()
+    torch.cuda.synchronize()
+    salad.check_error()
+    assert torch.equal(o_mid[lo], o_g0[lo])
+    assert torch.equal(o_mid[hi], o_full[hi])
+    ref = oracle.forward(inp, mode="topk", block=w.block, topk=w.topk, eps=w.eps,
+                         idx_override=_selection_used(w, inp, mid.idx_out), drop_threshold=thr)
+    assert list(ref["dropped"]) == [b == lo for b in range(2)]
+    assert_close(o_mid, ref["o"], "forward with branch dropping")
 
 
 def test_forward_is_deterministic(salad):

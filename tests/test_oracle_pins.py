@@ -242,11 +242,11 @@ def test_linear_state_token_shuffle_invariant():
 
 
 # ----------------------------------------------------- combine / forward ---
-def _tiny_inputs(N=192, H=2, d=16, D=32, seed=90):
+def _tiny_inputs(N=192, H=2, d=16, D=32, seed=90, B=1):
     rng = np.random.default_rng(seed)
     return {
-        "q": rng.standard_normal((1, H, N, d)), "k": rng.standard_normal((1, H, N, d)),
-        "v": rng.standard_normal((1, H, N, d)), "x": rng.standard_normal((1, N, D)),
+        "q": rng.standard_normal((B, H, N, d)), "k": rng.standard_normal((B, H, N, d)),
+        "v": rng.standard_normal((B, H, N, d)), "x": rng.standard_normal((B, N, D)),
         "w_gate": rng.normal(0, 0.5, D), "bias": 0.1,
         "w_lin": rng.normal(0, 0.2, (H, d, d)),
     }
@@ -259,6 +259,33 @@ def test_forward_gate_zero_is_sparse_branch_exactly():
     inp["w_lin"] = np.zeros_like(inp["w_lin"])
     r = oracle.forward(inp, mode="topk", block=64, topk=2)
     np.testing.assert_array_equal(r["o"], r["o_sparse"])
+
+
+def test_forward_branch_dropping_per_sample_threshold():
+    # Step 8 of the method: a sample whose gate value is below the threshold
+    # keeps only its sparse branch; the others are untouched.
+    inp = _tiny_inputs(B=2, seed=93)
+    inp["x"][1] += 0.5          # separates the two samples' gate values
+    full = oracle.forward(inp, mode="topk", block=64, topk=2)
+    s = full["s"]
+    assert s[0] != s[1]
+    lo, hi = sorted(range(2), key=lambda b: s[b])
+    none = oracle.forward(inp, mode="topk", block=64, topk=2, drop_threshold=0.0)
+    np.testing.assert_array_equal(none["o"], full["o"])
+    assert not none["dropped"].any()
+    both = oracle.forward(inp, mode="topk", block=64, topk=2, drop_threshold=1.0)
+    np.testing.assert_array_equal(both["o"], full["o_sparse"])
+    np.testing.assert_array_equal(both["o"],
+                                  oracle.forward(inp, mode="topk", block=64, topk=2,
+                                                 gate_override=0.0)["o"])
+    mid = oracle.forward(inp, mode="topk", block=64, topk=2,
+                         drop_threshold=float(s[lo] + s[hi]) / 2)
+    assert mid["dropped"][lo] and not mid["dropped"][hi]
+    np.testing.assert_array_equal(mid["o"][lo], full["o_sparse"][lo])
+    np.testing.assert_array_equal(mid["o"][hi], full["o"][hi])
+    # The comparison is strict: a gate value equal to the threshold is kept.
+    at = oracle.forward(inp, mode="topk", block=64, topk=2, drop_threshold=float(s[lo]))
+    assert not at["dropped"][lo]
 
 
 def test_forward_linear_in_gate_and_projection():

@@ -24,8 +24,11 @@ Readings where the pages are silent (each is listed in the design notes):
   block means over valid rows only; no forced blocks; ties broken towards the
   lower block index; eps = 1e-6 added to the linear-attention denominator;
   gate s = sigmoid(w . mean_tokens(X) + b) with X already time-modulated;
-  W_lin per head, d x d, right-multiplying row vectors; no 3-D RoPE in the
-  linear branch; space-major order r = (y * Wh + x) * F + f; window
+  W_lin per head, d x d, right-multiplying row vectors; the 3-D rotary
+  encoding of the linear branch (optional) rotates adjacent channel pairs of
+  phi(q) and phi(k) in the numerator only, channel groups (frame, row,
+  column) of d - 4*floor(d/6), 2*floor(d/6), 2*floor(d/6) channels, base
+  10000; space-major order r = (y * Wh + x) * F + f; window
   |r - c| <= W clipped at the sequence ends.
 
 Parity pins: every function here is checked by ``tests/test_oracle_pins.py``
@@ -42,6 +45,7 @@ __all__ = [
     "as64", "gate", "block_means", "block_scores", "select_topk",
     "topk_attention_rows", "topk_attention", "space_major_order",
     "swa_attention_rows", "swa_attention", "dense_attention",
+    "rope3d_split", "rope3d_angles", "rope3d_rotate",
     "linear_state", "linear_apply", "combine", "forward",
     "near_tie_equivalent",
 ]
@@ -225,22 +229,67 @@ def dense_attention(q, k, v) -> np.ndarray:
 
 
 # ------------------------------------------------------ linear branch -----
-def linear_state(k, v):
+def rope3d_split(d: int):
+    """Channel groups (frame, row, column) of the 3-D rotary encoding.
+
+    The pages give no split (reading): 2*floor(d/6) channels each for the row
+    and column positions, the remaining channels for the frame position, in
+    that order: d = 128 -> (44, 42, 42).
+    """
+    dy = 2 * (d // 6)
+    return d - 2 * dy, dy, dy
+
+
+def rope3d_angles(N: int, d: int, F: int, Hh: int, Wh: int, base: float = 10000.0) -> np.ndarray:
+    """Rotation angle of each channel pair of each token: [N, d // 2].
+
+    Token t (frame-major) sits at frame f = t // (Hh*Wh), row y = (t // Wh) %
+    Hh, column x = t % Wh.  Pair i of a group with g channels turns by
+    position * base^(-2i/g) (the rotary encoding, applied per axis).
+    """
+    assert F * Hh * Wh == N
+    t = np.arange(N)
+    pos = (t // (Hh * Wh), (t // Wh) % Hh, t % Wh)
+    cols = []
+    for g, p in zip(rope3d_split(d), pos):
+        theta = base ** (-2.0 * np.arange(g // 2) / g)
+        cols.append(np.outer(p, theta))
+    return np.concatenate(cols, axis=1)
+
+
+def rope3d_rotate(x, angles) -> np.ndarray:
+    """Turns each adjacent channel pair (2i, 2i+1) of each row by its angle."""
+    x = as64(x)
+    a, b = x[:, 0::2], x[:, 1::2]
+    c, s = np.cos(angles), np.sin(angles)
+    out = np.empty_like(x)
+    out[:, 0::2] = a * c - b * s
+    out[:, 1::2] = a * s + b * c
+    return out
+
+
+def linear_state(k, v, angles=None):
     """H = phi(K)^T V and Z = phi(K)^T 1 with phi = ReLU, for one head.
 
     "SALAD ... (paper.rainbus.top)" 前置知识 Linear Attention.  k, v: [N, d]
-    -> H [d, d], Z [d].
+    -> H [d, d], Z [d].  With ``angles`` (the 3-D rotary encoding the linear
+    branch integrates, 方法步骤详情 step 3), H sums the rotated features
+    R_j phi(k_j) v_j^T; Z stays unrotated (reading: the rotation enters the
+    numerator only, which keeps the denominator positive).
     """
     k, v = as64(k), as64(v)
     pk = np.maximum(k, 0.0)
-    return pk.T @ v, pk.sum(axis=0)
+    rk = pk if angles is None else rope3d_rotate(pk, angles)
+    return rk.T @ v, pk.sum(axis=0)
 
 
-def linear_apply(q, Hst, Z, eps: float) -> np.ndarray:
-    """O_l = phi(Q) H / (phi(Q) Z + eps) for one head: [N, d]."""
+def linear_apply(q, Hst, Z, eps: float, angles=None) -> np.ndarray:
+    """O_l = phi(Q) H / (phi(Q) Z + eps) for one head: [N, d].  With
+    ``angles`` the numerator uses the rotated R_i phi(q_i)."""
     q = as64(q)
     pq = np.maximum(q, 0.0)
-    return (pq @ Hst) / ((pq @ Z) + eps)[:, None]
+    rq = pq if angles is None else rope3d_rotate(pq, angles)
+    return (rq @ Hst) / ((pq @ Z) + eps)[:, None]
 
 
 # ------------------------------------------------------------ combine -----
@@ -254,7 +303,8 @@ def forward(inp: Dict, *, mode: str, block: int = 64, topk: int = 0, window: int
             space_major_heads: Sequence[int] = (), F: int = 0, Hh: int = 0, Wh: int = 0,
             eps: float = 1e-6, gate_override: Optional[float] = None,
             idx_override: Optional[np.ndarray] = None,
-            drop_threshold: float = 0.0) -> Dict[str, np.ndarray]:
+            drop_threshold: float = 0.0, rope3d: bool = False,
+            rope_base: float = 10000.0) -> Dict[str, np.ndarray]:
     """The whole hybrid layer, in the step order of the method.
 
     inp: q, k, v [B, H, N, d]; x [B, N, D]; w_gate [D]; bias; w_lin [H, d, d].
@@ -265,7 +315,9 @@ def forward(inp: Dict, *, mode: str, block: int = 64, topk: int = 0, window: int
     3.1-3.2): a sample whose gate value s_b is below the threshold keeps only
     its sparse branch, O = O_sparse (0 never drops, since s_b > 0).
     Returns s [B], idx [B, H, nb, topk] (topk mode), scores, o_sparse, o_lin,
-    o and dropped [B].
+    o and dropped [B].  ``rope3d``: the linear branch integrates the 3-D
+    rotary encoding over the (F, Hh, Wh) grid of the tokens (see
+    ``linear_state``).
     """
     q, k, v = as64(inp["q"]), as64(inp["k"]), as64(inp["v"])
     B, H, N, d = q.shape
@@ -276,6 +328,7 @@ def forward(inp: Dict, *, mode: str, block: int = 64, topk: int = 0, window: int
     o_sparse = np.empty_like(q)
     o_lin = np.empty_like(q)
     o = np.empty_like(q)
+    angles = rope3d_angles(N, d, F, Hh, Wh, rope_base) if rope3d else None
     idx = np.zeros((B, H, nb, max(topk, 1)), np.int64) if mode == "topk" else None
     scores = np.zeros((B, H, nb, nb)) if mode == "topk" else None
     for b in range(B):
@@ -292,8 +345,8 @@ def forward(inp: Dict, *, mode: str, block: int = 64, topk: int = 0, window: int
                 o_sparse[b, h] = dense_attention(q[b, h], k[b, h], v[b, h])
             else:
                 raise ValueError(mode)
-            Hst, Z = linear_state(k[b, h], v[b, h])
-            o_lin[b, h] = linear_apply(q[b, h], Hst, Z, eps)
+            Hst, Z = linear_state(k[b, h], v[b, h], angles)
+            o_lin[b, h] = linear_apply(q[b, h], Hst, Z, eps, angles)
             if s[b] < drop_threshold:
                 o[b, h] = o_sparse[b, h]
             else:

@@ -241,6 +241,82 @@ def test_linear_state_token_shuffle_invariant():
     assert np.all(Z1 >= 0)
 
 
+# ------------------------------------------------------- 3-D rotary code ---
+def test_rope3d_angles_per_axis_closed_form():
+    F, Hh, Wh, d = 3, 4, 5, 64
+    N = F * Hh * Wh
+    gt, gy, gx = oracle.rope3d_split(d)
+    assert (gt, gy, gx) == (24, 20, 20) and oracle.rope3d_split(128) == (44, 42, 42)
+    A = oracle.rope3d_angles(N, d, F, Hh, Wh, base=100.0)
+    assert A.shape == (N, d // 2)
+    f, y, x = 2, 3, 1
+    t = (f * Hh + y) * Wh + x
+    for i in range(gt // 2):
+        assert math.isclose(A[t, i], f * 100.0 ** (-2 * i / gt), rel_tol=1e-13)
+    for i in range(gy // 2):
+        assert math.isclose(A[t, gt // 2 + i], y * 100.0 ** (-2 * i / gy), rel_tol=1e-13)
+    for i in range(gx // 2):
+        assert math.isclose(A[t, (gt + gy) // 2 + i], x * 100.0 ** (-2 * i / gx), rel_tol=1e-13)
+    np.testing.assert_array_equal(A[0], 0.0)
+
+
+def test_rope3d_rotation_is_complex_multiplication_and_relative():
+    rng = np.random.default_rng(95)
+    F, Hh, Wh, d = 2, 3, 4, 16
+    N = F * Hh * Wh
+    A = oracle.rope3d_angles(N, d, F, Hh, Wh)
+    x = rng.standard_normal((N, d))
+    r = oracle.rope3d_rotate(x, A)
+    z = (x[:, 0::2] + 1j * x[:, 1::2]) * np.exp(1j * A)
+    np.testing.assert_allclose(r[:, 0::2], z.real, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(r[:, 1::2], z.imag, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(np.linalg.norm(r, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+    # (R_s a) . (R_t b) depends on the positions only through their difference:
+    # the same vectors at two token pairs with equal (df, dy, dx) give one value.
+    a, b = rng.standard_normal(d), rng.standard_normal(d)
+    tok = lambda f, yy, xx: (f * Hh + yy) * Wh + xx
+    def dot(s_, t_):
+        return float(oracle.rope3d_rotate(a[None], A[[s_]])[0] @ oracle.rope3d_rotate(b[None], A[[t_]])[0])
+    assert math.isclose(dot(tok(0, 0, 1), tok(1, 1, 3)), dot(tok(0, 1, 0), tok(1, 2, 2)),
+                        rel_tol=1e-12, abs_tol=1e-12)
+
+
+def test_linear_branch_with_rope_vs_quadratic_form():
+    # The rotation enters the numerator only: num_i = sum_j (R_i phi(q_i)) .
+    # (R_j phi(k_j)) v_j, den_i = sum_j phi(q_i) . phi(k_j) + eps, written out
+    # token pair by token pair.
+    rng = np.random.default_rng(96)
+    F, Hh, Wh, d = 2, 3, 5, 8
+    N = F * Hh * Wh
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    A = oracle.rope3d_angles(N, d, F, Hh, Wh)
+    Hst, Z = oracle.linear_state(k, v, A)
+    got = oracle.linear_apply(q, Hst, Z, 1e-6, A)
+    pq, pk = np.maximum(q, 0), np.maximum(k, 0)
+    want = np.zeros((N, d))
+    for i in range(N):
+        num, den = np.zeros(d), 1e-6
+        for j in range(N):
+            qi = pq[i].copy(); kj = pk[j].copy()
+            w_ = 0.0
+            for m in range(d // 2):
+                ai, aj = A[i, m], A[j, m]
+                qa = (qi[2 * m] * math.cos(ai) - qi[2 * m + 1] * math.sin(ai),
+                      qi[2 * m] * math.sin(ai) + qi[2 * m + 1] * math.cos(ai))
+                ka = (kj[2 * m] * math.cos(aj) - kj[2 * m + 1] * math.sin(aj),
+                      kj[2 * m] * math.sin(aj) + kj[2 * m + 1] * math.cos(aj))
+                w_ += qa[0] * ka[0] + qa[1] * ka[1]
+            num += w_ * v[j]
+            den += float(qi @ kj)
+        want[i] = num / den
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-12)
+    # Z ignores the rotation; at a single token (every position 0) nothing turns.
+    np.testing.assert_allclose(Z, pk.sum(axis=0), rtol=1e-13)
+    H0, Z0 = oracle.linear_state(k[:1], v[:1], oracle.rope3d_angles(1, d, 1, 1, 1))
+    H1, Z1 = oracle.linear_state(k[:1], v[:1])
+    np.testing.assert_array_equal(H0, H1)
+
+
 # ----------------------------------------------------- combine / forward ---
 def _tiny_inputs(N=192, H=2, d=16, D=32, seed=90, B=1):
     rng = np.random.default_rng(seed)

@@ -199,6 +199,17 @@ typedef struct salad_forward_args {
      * threshold is calibrated offline (a percentile of gate values).  0 or
      * NaN: never drop.  +-inf is rejected. */
     float drop_threshold;
+    /* 3-D rotary position encoding in the linear branch ("SALAD ...
+     * (paper.rainbus.top)" 方法步骤详情 step 3): 1 = on, 0 = off.  Adjacent
+     * channel pairs of phi(q) and phi(k) turn by the token's frame, row and
+     * column positions on the F x Hh x Wh grid (F*Hh*Wh == N required; the
+     * tokens are frame-major) over three channel groups of d - 4*floor(d/6),
+     * 2*floor(d/6), 2*floor(d/6) channels, pair i of a g-channel group at
+     * rate rope_base^(-2i/g).  The rotation enters the numerator only:
+     * O_l = (R phi(q)) H_R / (phi(q) Z + eps) with H_R = sum_j R_j phi(k_j) v_j^T
+     * and Z = sum_j phi(k_j). */
+    int rope3d;
+    float rope_base;            /* > 1, usually 10000 */
     float* s_out;               /* optional device float32 [B] (out), may be NULL */
     int32_t* idx_out;           /* optional device int32 [B,H,nb,topk] (out), may be NULL */
     void* workspace;            /* device scratch, >= salad_forward_workspace_bytes() */

@@ -62,6 +62,7 @@ class ForwardArgs(ctypes.Structure):
         ("F", ctypes.c_int), ("Hh", ctypes.c_int), ("Wh", ctypes.c_int),
         ("eps", ctypes.c_float), ("gate_override", ctypes.c_float),
         ("drop_threshold", ctypes.c_float),
+        ("rope3d", ctypes.c_int), ("rope_base", ctypes.c_float),
         ("s_out", ctypes.c_void_p), ("idx_out", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("phase_events", ctypes.c_void_p),
@@ -291,7 +292,8 @@ class ForwardPlan:
     def __init__(self, q, k, v, x, w_gate, w_lin, *, mode: str = "topk", topk: int = 0,
                  window: int = 0, space_major_heads: Optional[Sequence[int]] = None,
                  F: int = 0, Hh: int = 0, Wh: int = 0, bias: float = 0.0, eps: float = 1e-6,
-                 gate_override: Optional[float] = None, drop_threshold: float = 0.0, o=None,
+                 gate_override: Optional[float] = None, drop_threshold: float = 0.0,
+                 rope3d: bool = False, rope_base: float = 10000.0, o=None,
                  s_out=None, idx_out=None, block: int = 64):
         for n, t in (("q", q), ("k", k), ("v", v), ("x", x), ("w_gate", w_gate),
                      ("w_lin", w_lin)):
@@ -314,6 +316,9 @@ class ForwardPlan:
         # Post-training branch dropping: sample b's linear branch is skipped
         # (on the device) when s_b < drop_threshold; 0 never drops.
         a.drop_threshold = float(drop_threshold)
+        # 3-D rotary encoding of the linear branch over the F x Hh x Wh grid.
+        a.rope3d = 1 if rope3d else 0
+        a.rope_base = float(rope_base)
         a.s_out = _ptr(s_out)
         a.idx_out = _ptr(idx_out)
         need = lib.salad_forward_workspace_bytes(ctypes.byref(a))

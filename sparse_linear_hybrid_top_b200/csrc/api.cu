@@ -134,7 +134,7 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, int S, int N, int d) 
 
 // ------------------------------------------------------- forward layout --
 struct FwdLayout {
-  size_t gate, s, sel, idx, lists, counts, lin, hst, z, g, qp, kp, vp, total;
+  size_t gate, s, sel, idx, lists, counts, lin, hst, z, g, rope, qp, kp, vp, total;
   int Hs;
   int slot[kMaxHeads];
 };
@@ -163,6 +163,8 @@ static FwdLayout forward_layout(const salad_forward_args* a) {
   L.hst = take(B * H * d * d * sizeof(float));
   L.z = take(B * H * d * sizeof(float));
   L.g = take(B * H * d * d * 2);
+  if (a->rope3d)
+    L.rope = take(rope_table_entries(a->d, a->F, a->Hh, a->Wh) * sizeof(float2));
   L.Hs = 0;
   for (int h = 0; h < kMaxHeads; ++h) L.slot[h] = -1;
   if (a->mode == SALAD_MODE_SWA && a->H <= kMaxHeads)
@@ -195,7 +197,7 @@ const char* salad_status_string(salad_status s) {
   }
 }
 
-int salad_version(void) { return 200; }
+int salad_version(void) { return 300; }
 
 // ------------------------------------------------------------------ gate --
 size_t salad_gate_workspace_bytes(int B, int N, int D) {
@@ -401,6 +403,11 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   const bool override_gate = !std::isnan(a->gate_override);
   if (override_gate && !std::isfinite(a->gate_override)) return SALAD_ERR_INVALID_ARG;
   if (std::isinf(a->drop_threshold)) return SALAD_ERR_INVALID_ARG;
+  if (a->rope3d != 0 && a->rope3d != 1) return SALAD_ERR_INVALID_ARG;
+  if (a->rope3d && (a->F < 1 || a->Hh < 1 || a->Wh < 1 ||
+                    static_cast<long long>(a->F) * a->Hh * a->Wh != a->N ||
+                    !(a->rope_base > 1.0f) || !std::isfinite(a->rope_base)))
+    return SALAD_ERR_INVALID_ARG;
   if (a->mode == SALAD_MODE_TOPK && (a->topk < 1 || a->topk > nblocks(a->N)))
     return SALAD_ERR_INVALID_ARG;
   if (a->mode == SALAD_MODE_SWA && a->window < 0) return SALAD_ERR_INVALID_ARG;
@@ -479,7 +486,15 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   BranchDrop drop;
   drop.s = s;
   drop.thr = at.drop;
-  e = launch_linear_state(c, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, a->w_lin, G, drop);
+  Rope3D rope;
+  if (a->rope3d) {
+    e = launch_rope_table(c, d, a->F, a->Hh, a->Wh, a->rope_base,
+                          reinterpret_cast<float2*>(ws + L.rope), &rope);
+    if (e != cudaSuccess) return SALAD_ERR_CUDA;
+  }
+  at.rope = rope;
+  e = launch_linear_state(c, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, a->w_lin, G, drop,
+                          rope);
   if (e != cudaSuccess || !mark(3)) return SALAD_ERR_CUDA;
   at.Gimg = G;
   at.Z = Z;

@@ -104,6 +104,7 @@ struct Params {
   const float* s;
   float gate_override;
   float drop;                 // the linear term of sample b is skipped when s_b < drop
+  Rope3D rope;                // 3-D rotary encoding of phi(Q) in the linear term
   float eps;
   float scale_log2;
   __nv_bfloat16* o;
@@ -476,6 +477,21 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
             qsrc + static_cast<long long>(row_valid ? row_pos : 0) * D);
         const float* zrow = HYB ? P.Z + static_cast<long long>(it.bh) * D : nullptr;
         float den = 0.f;
+        // Grid position of the row's token (its frame-major index) for the
+        // rotary encoding of the linear term.
+        const bool rope_on = lin && P.rope.tab != nullptr && row_valid;
+        int rf = 0, ry = 0, rx = 0;
+        if (rope_on) {
+          int tok = row_pos;
+          if (it.slot >= 0) {
+            const int fr = row_pos % P.F, pos = row_pos / P.F;
+            tok = fr * (P.Hh * P.Wh) + pos;
+          }
+          const int plane = P.rope.Hh * P.rope.Wh;
+          rf = tok / plane;
+          ry = (tok / P.rope.Wh) % P.rope.Hh;
+          rx = tok % P.rope.Wh;
+        }
 #pragma unroll
         for (int c0 = 0; c0 < D / 2; c0 += 16) {
           uint32_t pk[16];
@@ -492,6 +508,16 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
               const float2 f = unpack_bf16x2(pk[e]);
               den = fmaf(f.x, __ldg(zrow + 2 * (c0 + e)), den);
               den = fmaf(f.y, __ldg(zrow + 2 * (c0 + e) + 1), den);
+            }
+            if (rope_on) {
+              // The numerator's phi(q) is rotated (word c0 + e is pair c0 + e);
+              // the denominator above is not.
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const float2 cs = rope_cs(P.rope, rf, ry, rx, c0 + e);
+                const float2 a = unpack_bf16x2(pk[e]);
+                pk[e] = pack_bf16x2(a.x * cs.x - a.y * cs.y, a.x * cs.y + a.y * cs.x);
+              }
             }
             tmem_st16(lane_base + C::kPQ + c0, pk);
           }
@@ -752,6 +778,7 @@ cudaError_t launch_attention(const Ctx& c, const AttnArgs& a) {
   P.s = a.s;
   P.gate_override = a.gate_override;
   P.drop = a.drop;
+  P.rope = a.rope;
   P.eps = a.eps;
   P.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(a.d));
   P.o = static_cast<__nv_bfloat16*>(a.o);

@@ -40,6 +40,31 @@ size_t linear_state_ws_bytes(int B, int H, int N, int d);
 // Hst = phi(K)^T V and Z = phi(K)^T 1 per (b, h).  With w_lin given, also
 // G[b,h] = Hst[b,h] W_lin[h], written as bf16 MMA B-operand images
 // [B*H][d*d] (K-major over the row index of G, 128-byte swizzle) into Gimg.
+// 3-D rotary encoding of the linear branch: adjacent channel pairs (2m,
+// 2m+1) of phi(q) and phi(k) turn by the token's (frame, row, column)
+// position over three channel groups of 2*gt2, 2*gy2, 2*gx2 channels.  tab
+// holds (cos, sin) per axis and position: [F][gt2], then [Hh][gy2], then
+// [Wh][gx2].  tab == null: no encoding.
+struct Rope3D {
+  const float2* tab = nullptr;
+  int F = 0, Hh = 0, Wh = 0;
+  int gt2 = 0, gy2 = 0, gx2 = 0;
+};
+size_t rope_table_entries(int d, int F, int Hh, int Wh);
+cudaError_t launch_rope_table(const Ctx& c, int d, int F, int Hh, int Wh, float base,
+                              float2* tab, Rope3D* out);
+
+#ifdef __CUDACC__
+// (cos, sin) of pair m of a token at frame f, row y, column x.
+__device__ __forceinline__ float2 rope_cs(const Rope3D& r, int f, int y, int x, int m) {
+  if (m < r.gt2) return __ldg(r.tab + f * r.gt2 + m);
+  m -= r.gt2;
+  if (m < r.gy2) return __ldg(r.tab + r.F * r.gt2 + y * r.gy2 + m);
+  m -= r.gy2;
+  return __ldg(r.tab + r.F * r.gt2 + r.Hh * r.gy2 + x * r.gx2 + m);
+}
+#endif
+
 // Post-training branch dropping on the device: sample b's linear branch is
 // skipped when its gate value (s[b], or gate_override when s is null) is
 // below thr.  thr = 0 or NaN never drops (gate values are >= 0).
@@ -51,7 +76,7 @@ struct BranchDrop {
 cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int B, int H, int N,
                                 int d, float* Hst, float* Z, void* ws,
                                 const void* w_lin = nullptr, void* Gimg = nullptr,
-                                BranchDrop drop = BranchDrop());
+                                BranchDrop drop = BranchDrop(), Rope3D rope = Rope3D());
 cudaError_t launch_linear_apply(const Ctx& c, const void* q, const float* Hst, const float* Z,
                                 float eps, int B, int H, int N, int d, void* o);
 
@@ -91,6 +116,7 @@ struct AttnArgs {
   const float* s;             // [B] gate values (device)
   float gate_override;        // used when s is null
   float drop = 0.0f;          // the linear term of sample b is skipped when s_b < drop
+  Rope3D rope;                // 3-D rotary encoding of phi(Q) in the linear term
   float eps;
   void* o;                    // bf16 [B,H,N,d]
 };

@@ -45,7 +45,7 @@ template <int D>
 __global__ void __launch_bounds__(192, 1) linear_state_kernel(
     const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv, int nblk,
     int blocks_per_cta, int ctas_per_head, float* __restrict__ partH, float* __restrict__ partZ,
-    unsigned* err, unsigned long long wait_ns, BranchDrop drop, int H) {
+    unsigned* err, unsigned long long wait_ns, BranchDrop drop, int H, Rope3D rope, int N) {
   using C = LS<D>;
   // A sample whose linear branch is dropped needs no state: the whole CTA
   // leaves before touching shared memory, barriers or TMEM.
@@ -179,18 +179,36 @@ __global__ void __launch_bounds__(192, 1) linear_state_kernel(
         const int q = tid + 128 * (i % 4);
         uint4* p = reinterpret_cast<uint4*>(ktile + half * kSlab + q * 16);
         uint4 v = *p;
-        v.x = relu_bf16x2(v.x);
-        v.y = relu_bf16x2(v.y);
-        v.z = relu_bf16x2(v.z);
-        v.w = relu_bf16x2(v.w);
-        *p = v;
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        uint32_t w4[4] = {relu_bf16x2(v.x), relu_bf16x2(v.y), relu_bf16x2(v.z), relu_bf16x2(v.w)};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = unpack_bf16x2(w4[e]);
           zacc[half * 8 + 2 * e] += f.x;
           zacc[half * 8 + 2 * e + 1] += f.y;
         }
+        if (rope.tab != nullptr) {
+          // The numerator's features are rotated; Z above is not.  Chunk q
+          // of the swizzled slab holds channels half*64 + 8L .. +7 of tile
+          // row q/8, with L = (q%8) ^ (row%8): pairs half*32 + 4L + e.
+          const int row = q / 8;
+          const int tok = (b0 + t) * 64 + row;
+          if (tok < N) {
+            const int L = (q % 8) ^ (row % 8);
+            const int plane = rope.Hh * rope.Wh;
+            const int f = tok / plane, y = (tok / rope.Wh) % rope.Hh, x = tok % rope.Wh;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 cs = rope_cs(rope, f, y, x, half * 32 + 4 * L + e);
+              const float2 a = unpack_bf16x2(w4[e]);
+              w4[e] = pack_bf16x2(a.x * cs.x - a.y * cs.y, a.x * cs.y + a.y * cs.x);
+            }
+          }
+        }
+        v.x = w4[0];
+        v.y = w4[1];
+        v.z = w4[2];
+        v.w = w4[3];
+        *p = v;
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -453,7 +471,7 @@ size_t linear_state_ws_bytes(int B, int H, int N, int d) {
 
 cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int B, int H, int N,
                                 int d, float* Hst, float* Z, void* ws, const void* w_lin,
-                                void* Gimg, BranchDrop drop) {
+                                void* Gimg, BranchDrop drop, Rope3D rope) {
   const LSPlan p = ls_plan(B, H, N, c.num_sms < 256 ? c.num_sms : 256);
   const int BH = B * H;
   const size_t parts = static_cast<size_t>(BH) * p.ctas_per_head;
@@ -471,14 +489,14 @@ cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int 
     if (e != cudaSuccess) return e;
     linear_state_kernel<128><<<grid, 192, LS<128>::kSmem, c.stream>>>(
         mk, mv, p.nblk, p.blocks_per_cta, p.ctas_per_head, partH, partZ, c.err, c.wait_ns, drop,
-        H);
+        H, rope, N);
   } else {
     e = cudaFuncSetAttribute(linear_state_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              LS<64>::kSmem);
     if (e != cudaSuccess) return e;
     linear_state_kernel<64><<<grid, 192, LS<64>::kSmem, c.stream>>>(
         mk, mv, p.nblk, p.blocks_per_cta, p.ctas_per_head, partH, partZ, c.err, c.wait_ns, drop,
-        H);
+        H, rope, N);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -494,6 +512,57 @@ cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int 
   linear_reduce_fold_kernel<<<dim3(d / kFoldRows, BH), 256, smem, c.stream>>>(
       partH, partZ, H, d, p.ctas_per_head, static_cast<const __nv_bfloat16*>(w_lin), Hst, Z,
       static_cast<__nv_bfloat16*>(Gimg), drop);
+  return cudaGetLastError();
+}
+
+// (cos, sin) table of the 3-D rotary encoding: entry (axis, position p,
+// pair i) = angle p * base^(-2i/g) for a channel group of g = 2 * pairs
+// channels, computed in float64.
+__global__ void rope_table_kernel(float2* tab, int F, int Hh, int Wh, int gt2, int gy2, int gx2,
+                                  double base) {
+  const int n0 = F * gt2, n1 = n0 + Hh * gy2, n2 = n1 + Wh * gx2;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n2; e += gridDim.x * blockDim.x) {
+    int pos, i, g2;
+    if (e < n0) {
+      pos = e / gt2; i = e % gt2; g2 = gt2;
+    } else if (e < n1) {
+      pos = (e - n0) / gy2; i = (e - n0) % gy2; g2 = gy2;
+    } else {
+      pos = (e - n1) / gx2; i = (e - n1) % gx2; g2 = gx2;
+    }
+    const double angle = pos * pow(base, -static_cast<double>(i) / g2);
+    double sn, cs;
+    sincos(angle, &sn, &cs);
+    tab[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+  }
+}
+
+static void rope_groups(int d, int* gt2, int* gy2, int* gx2) {
+  const int gy = 2 * (d / 6);
+  *gy2 = gy / 2;
+  *gx2 = gy / 2;
+  *gt2 = (d - 2 * gy) / 2;
+}
+
+size_t rope_table_entries(int d, int F, int Hh, int Wh) {
+  int gt2, gy2, gx2;
+  rope_groups(d, &gt2, &gy2, &gx2);
+  return static_cast<size_t>(F) * gt2 + static_cast<size_t>(Hh) * gy2 +
+         static_cast<size_t>(Wh) * gx2;
+}
+
+cudaError_t launch_rope_table(const Ctx& c, int d, int F, int Hh, int Wh, float base,
+                              float2* tab, Rope3D* out) {
+  Rope3D r;
+  rope_groups(d, &r.gt2, &r.gy2, &r.gx2);
+  r.F = F;
+  r.Hh = Hh;
+  r.Wh = Wh;
+  r.tab = tab;
+  const long long n = static_cast<long long>(rope_table_entries(d, F, Hh, Wh));
+  rope_table_kernel<<<static_cast<int>((n + 255) / 256), 256, 0, c.stream>>>(
+      tab, F, Hh, Wh, r.gt2, r.gy2, r.gx2, static_cast<double>(base));
+  *out = r;
   return cudaGetLastError();
 }
 

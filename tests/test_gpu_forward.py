@@ -128,6 +128,27 @@ def test_forward_branch_dropping(salad):
     assert_close(o_mid, ref["o"], "forward with branch dropping")
 
 
+@pytest.mark.parametrize("w", CASES + [SWA_SMALL, SWA_SMALL64], ids=lambda w: w.name)
+def test_forward_rope3d(salad, w):
+    # The linear branch with the 3-D rotary encoding over the workload's grid.
+    inp = generate(w)
+    dev = device_inputs(inp)
+    grid = {} if w.mode == "swa" else dict(F=w.F, Hh=w.Hh, Wh=w.Wh)
+    plan = _plan(salad, w, dev, rope3d=True, **grid)
+    o = plan.run().clone()
+    torch.cuda.synchronize()
+    salad.check_error()
+    kw = dict(mode=w.mode, block=w.block, topk=w.topk, window=w.window,
+              space_major_heads=w.space_major_heads, F=w.F, Hh=w.Hh, Wh=w.Wh, eps=w.eps)
+    if w.mode == "topk":
+        kw["idx_override"] = _selection_used(w, inp, plan.idx_out)
+    ref = oracle.forward(inp, rope3d=True, **kw)
+    assert_close(o, ref["o"], f"forward with rope3d {w.name}")
+    if w.N == 1:
+        # A single token sits at position 0: nothing turns.
+        assert torch.equal(o, _plan(salad, w, dev).run())
+
+
 def test_forward_is_deterministic(salad):
     w = RAGGED128
     dev = device_inputs(generate(w))

@@ -68,12 +68,13 @@ def step_flops(w) -> dict:
 
 
 def launches_per_step(w) -> int:
-    # gate (2) + [pool, score, topk, pair_union | gather] + linear (3) + attention (1)
+    # gate (2) + [pool, score, topk, pair_union | gather] + linear state and
+    # reduce+fold (2) + attention (1)
     if w.mode == "topk":
-        return 2 + 4 + 3 + 1
+        return 2 + 4 + 2 + 1
     if w.mode == "swa":
-        return 2 + (1 if w.space_major_heads else 0) + 3 + 1
-    return 2 + 3 + 1
+        return 2 + (1 if w.space_major_heads else 0) + 2 + 1
+    return 2 + 2 + 1
 
 
 def load_peaks() -> tuple:
@@ -332,6 +333,32 @@ def run_ours(args, w) -> int:
     torch.cuda.synchronize(device)
     dense_ms = d0.elapsed_time(d1) / nd
 
+    # The optional parts of the layer, timed the same way (diagnostics; the
+    # headline above is the default layer): the 3-D rotary encoding in the
+    # linear branch, and post-training branch dropping with every sample
+    # below the threshold (the sparse branch alone plus the gate).
+    def time_plan(p, n):
+        for _ in range(3):
+            p.run(stream)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(n):
+            p.run(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+        salad.check_error(stream)
+        return reduce_max(t0.elapsed_time(t1) / n, device)
+    nv = max(3, min(args.steps, 100))
+    grid = {} if w.mode == "swa" else dict(F=w.F, Hh=w.Hh, Wh=w.Wh)
+    variants = {
+        "rope3d": time_plan(salad.ForwardPlan(
+            dev["q"], dev["k"], dev["v"], dev["x"], dev["w_gate"], dev["w_lin"], mode=w.mode,
+            topk=w.topk, bias=w.bias, eps=w.eps, rope3d=True, **extra, **grid), nv),
+        "branch_dropped": time_plan(salad.ForwardPlan(
+            dev["q"], dev["k"], dev["v"], dev["x"], dev["w_gate"], dev["w_lin"], mode=w.mode,
+            topk=w.topk, bias=w.bias, eps=w.eps, drop_threshold=1.0, **extra), nv),
+    }
+
     # End to end through the public API: pinned host inputs -> device ->
     # salad_forward -> result back to the host, every step.
     names = ("q", "k", "v", "x", "w_gate", "w_lin")
@@ -376,6 +403,7 @@ def run_ours(args, w) -> int:
         "ms_per_layer": round(agg["ms_per_step"], 5),
         "phases_ms": {k: round(v, 5) for k, v in phases.items()},
         "dense_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / agg["ms_per_step"], 3),
+        "variants_ms_per_layer": {k: round(v, 5) for k, v in variants.items()},
         "flops_per_step": fl["total"],
         "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,hybrid>",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",

@@ -134,7 +134,7 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, int S, int N, int d) 
 
 // ------------------------------------------------------- forward layout --
 struct FwdLayout {
-  size_t gate, s, sel, idx, lists, counts, lin, hst, z, g, rope, qp, kp, vp, total;
+  size_t gate, s, sel, idx, lists, counts, lin, hst, z, g, qp, kp, vp, total;
   int Hs;
   int slot[kMaxHeads];
 };
@@ -163,8 +163,6 @@ static FwdLayout forward_layout(const salad_forward_args* a) {
   L.hst = take(B * H * d * d * sizeof(float));
   L.z = take(B * H * d * sizeof(float));
   L.g = take(B * H * d * d * 2);
-  if (a->rope3d)
-    L.rope = take(rope_table_entries(a->d, a->F, a->Hh, a->Wh) * sizeof(float2));
   L.Hs = 0;
   for (int h = 0; h < kMaxHeads; ++h) L.slot[h] = -1;
   if (a->mode == SALAD_MODE_SWA && a->H <= kMaxHeads)
@@ -487,11 +485,7 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   drop.s = s;
   drop.thr = at.drop;
   Rope3D rope;
-  if (a->rope3d) {
-    e = launch_rope_table(c, d, a->F, a->Hh, a->Wh, a->rope_base,
-                          reinterpret_cast<float2*>(ws + L.rope), &rope);
-    if (e != cudaSuccess) return SALAD_ERR_CUDA;
-  }
+  if (a->rope3d) rope = make_rope3d(d, a->F, a->Hh, a->Wh, a->rope_base);
   at.rope = rope;
   e = launch_linear_state(c, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, a->w_lin, G, drop,
                           rope);

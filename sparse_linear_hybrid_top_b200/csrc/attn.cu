@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         float den = 0.f;
         // Grid position of the row's token (its frame-major index) for the
         // rotary encoding of the linear term.
-        const bool rope_on = lin && P.rope.tab != nullptr && row_valid;
+        const bool rope_on = lin && P.rope.on && row_valid;
         int rf = 0, ry = 0, rx = 0;
         if (rope_on) {
           int tok = row_pos;
@@ -487,7 +487,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
             const int fr = row_pos % P.F, pos = row_pos / P.F;
             tok = fr * (P.Hh * P.Wh) + pos;
           }
-          const int plane = P.rope.Hh * P.rope.Wh;
+          const int plane = P.rope.Hh * P.rope.Wh;   // token -> (frame, row, column)
           rf = tok / plane;
           ry = (tok / P.rope.Wh) % P.rope.Hh;
           rx = tok % P.rope.Wh;
@@ -514,7 +514,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
               // the denominator above is not.
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
-                const float2 cs = rope_cs(P.rope, rf, ry, rx, c0 + e);
+                const float2 cs = rope_cs(P.rope, P.rope.theta, c0 + e, rf, ry, rx);
                 const float2 a = unpack_bf16x2(pk[e]);
                 pk[e] = pack_bf16x2(a.x * cs.x - a.y * cs.y, a.x * cs.y + a.y * cs.x);
               }

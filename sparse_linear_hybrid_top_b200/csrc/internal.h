@@ -41,27 +41,33 @@ size_t linear_state_ws_bytes(int B, int H, int N, int d);
 // G[b,h] = Hst[b,h] W_lin[h], written as bf16 MMA B-operand images
 // [B*H][d*d] (K-major over the row index of G, 128-byte swizzle) into Gimg.
 // 3-D rotary encoding of the linear branch: adjacent channel pairs (2m,
-// 2m+1) of phi(q) and phi(k) turn by the token's (frame, row, column)
-// position over three channel groups of 2*gt2, 2*gy2, 2*gx2 channels.  tab
-// holds (cos, sin) per axis and position: [F][gt2], then [Hh][gy2], then
-// [Wh][gx2].  tab == null: no encoding.
+// 2m+1) of phi(q) and phi(k) turn by angle pos * theta[m], pos being the
+// token's frame, row or column on the F x Hh x Wh grid for the first gt2
+// pairs, the next gy2 pairs and the remaining pairs.  on == 0: no encoding.
 struct Rope3D {
-  const float2* tab = nullptr;
+  int on = 0;
   int F = 0, Hh = 0, Wh = 0;
-  int gt2 = 0, gy2 = 0, gx2 = 0;
+  int gt2 = 0, gy2 = 0;
+  double theta[64] = {};
 };
-size_t rope_table_entries(int d, int F, int Hh, int Wh);
-cudaError_t launch_rope_table(const Ctx& c, int d, int F, int Hh, int Wh, float base,
-                              float2* tab, Rope3D* out);
+// theta[m] = base^(-2i/g) for pair i of a group of g channels.
+Rope3D make_rope3d(int d, int F, int Hh, int Wh, float base);
 
 #ifdef __CUDACC__
-// (cos, sin) of pair m of a token at frame f, row y, column x.
-__device__ __forceinline__ float2 rope_cs(const Rope3D& r, int f, int y, int x, int m) {
-  if (m < r.gt2) return __ldg(r.tab + f * r.gt2 + m);
-  m -= r.gt2;
-  if (m < r.gy2) return __ldg(r.tab + r.F * r.gt2 + y * r.gy2 + m);
-  m -= r.gy2;
-  return __ldg(r.tab + r.F * r.gt2 + r.Hh * r.gy2 + x * r.gx2 + m);
+// (cos, sin) of the angle of pair m for a token at frame f, row y, column x.
+// The angle pos * theta[m] is formed and reduced modulo 2 pi in float64 (its
+// error stays near 1e-11 rad for every position the library accepts); the
+// reduced angle in [-pi, pi] is turned by the CUDA intrinsic __sincosf,
+// accurate to about 2^-21 absolute there.
+__device__ __forceinline__ float2 rope_cs(const Rope3D& r, const double* theta, int m, int f,
+                                          int y, int x) {
+  const int pos = m < r.gt2 ? f : (m < r.gt2 + r.gy2 ? y : x);
+  const double a = static_cast<double>(pos) * theta[m];
+  const double k = rint(a * 0.15915494309189535);     // a / (2 pi), rounded
+  const float red = static_cast<float>(fma(-k, 6.283185307179586, a));
+  float sn, cs;
+  __sincosf(red, &sn, &cs);
+  return make_float2(cs, sn);
 }
 #endif
 

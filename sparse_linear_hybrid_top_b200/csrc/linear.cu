@@ -16,6 +16,8 @@
 // into bf16 hi + lo parts (H ~= hi + lo to ~16 mantissa bits) in a K-major
 // swizzled shared-memory image, two MMAs into one TMEM accumulator; the
 // denominator phi(q) . Z + eps is a per-thread float32 dot product.
+#include <cmath>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -33,7 +35,8 @@ struct LS {
   static constexpr int kZero = (D == 64) ? kSlab : 0;    // zero slab pads M to 128
   static constexpr int kRed = 128 * 16 * 4;              // Z partials
   static constexpr int kBars = 256;
-  static constexpr int kSmem = 1024 /*align slack*/ + kStages * kStage + kZero + kRed + kBars;
+  static constexpr int kTheta = 64 * 8;                  // rotary rates, one per channel pair
+  static constexpr int kSmem = 1024 /*align slack*/ + kStages * kStage + kZero + kRed + kBars + kTheta;
 };
 
 __device__ __forceinline__ bool branch_dropped(const BranchDrop& d, int b) {
@@ -60,6 +63,7 @@ __global__ void __launch_bounds__(192, 1) linear_state_kernel(
   // bars: full[0..S), relu[S..2S), empty[2S..3S), acc, drain; then tmem holder, abort
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * C::kStages + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  double* theta = reinterpret_cast<double*>(reinterpret_cast<unsigned char*>(bars) + C::kBars);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.x / ctas_per_head;
@@ -161,6 +165,10 @@ __global__ void __launch_bounds__(192, 1) linear_state_kernel(
   } else {
     // ---------------- ReLU + Z workers (warps 2..5) and the epilogue
     const int tid = threadIdx.x - 64;
+    if (rope.on) {
+      if (tid < D / 2) theta[tid] = rope.theta[tid];
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
     float zacc[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) zacc[e] = 0.f;
@@ -186,7 +194,7 @@ __global__ void __launch_bounds__(192, 1) linear_state_kernel(
           zacc[half * 8 + 2 * e] += f.x;
           zacc[half * 8 + 2 * e + 1] += f.y;
         }
-        if (rope.tab != nullptr) {
+        if (rope.on) {
           // The numerator's features are rotated; Z above is not.  Chunk q
           // of the swizzled slab holds channels half*64 + 8L .. +7 of tile
           // row q/8, with L = (q%8) ^ (row%8): pairs half*32 + 4L + e.
@@ -198,7 +206,7 @@ __global__ void __launch_bounds__(192, 1) linear_state_kernel(
             const int f = tok / plane, y = (tok / rope.Wh) % rope.Hh, x = tok % rope.Wh;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 cs = rope_cs(rope, f, y, x, half * 32 + 4 * L + e);
+              const float2 cs = rope_cs(rope, theta, half * 32 + 4 * L + e, f, y, x);
               const float2 a = unpack_bf16x2(w4[e]);
               w4[e] = pack_bf16x2(a.x * cs.x - a.y * cs.y, a.x * cs.y + a.y * cs.x);
             }
@@ -515,55 +523,27 @@ cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int 
   return cudaGetLastError();
 }
 
-// (cos, sin) table of the 3-D rotary encoding: entry (axis, position p,
-// pair i) = angle p * base^(-2i/g) for a channel group of g = 2 * pairs
-// channels, computed in float64.
-__global__ void rope_table_kernel(float2* tab, int F, int Hh, int Wh, int gt2, int gy2, int gx2,
-                                  double base) {
-  const int n0 = F * gt2, n1 = n0 + Hh * gy2, n2 = n1 + Wh * gx2;
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n2; e += gridDim.x * blockDim.x) {
-    int pos, i, g2;
-    if (e < n0) {
-      pos = e / gt2; i = e % gt2; g2 = gt2;
-    } else if (e < n1) {
-      pos = (e - n0) / gy2; i = (e - n0) % gy2; g2 = gy2;
-    } else {
-      pos = (e - n1) / gx2; i = (e - n1) % gx2; g2 = gx2;
-    }
-    const double angle = pos * pow(base, -static_cast<double>(i) / g2);
-    double sn, cs;
-    sincos(angle, &sn, &cs);
-    tab[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
-  }
-}
-
-static void rope_groups(int d, int* gt2, int* gy2, int* gx2) {
-  const int gy = 2 * (d / 6);
-  *gy2 = gy / 2;
-  *gx2 = gy / 2;
-  *gt2 = (d - 2 * gy) / 2;
-}
-
-size_t rope_table_entries(int d, int F, int Hh, int Wh) {
-  int gt2, gy2, gx2;
-  rope_groups(d, &gt2, &gy2, &gx2);
-  return static_cast<size_t>(F) * gt2 + static_cast<size_t>(Hh) * gy2 +
-         static_cast<size_t>(Wh) * gx2;
-}
-
-cudaError_t launch_rope_table(const Ctx& c, int d, int F, int Hh, int Wh, float base,
-                              float2* tab, Rope3D* out) {
+Rope3D make_rope3d(int d, int F, int Hh, int Wh, float base) {
   Rope3D r;
-  rope_groups(d, &r.gt2, &r.gy2, &r.gx2);
+  r.on = 1;
   r.F = F;
   r.Hh = Hh;
   r.Wh = Wh;
-  r.tab = tab;
-  const long long n = static_cast<long long>(rope_table_entries(d, F, Hh, Wh));
-  rope_table_kernel<<<static_cast<int>((n + 255) / 256), 256, 0, c.stream>>>(
-      tab, F, Hh, Wh, r.gt2, r.gy2, r.gx2, static_cast<double>(base));
-  *out = r;
-  return cudaGetLastError();
+  const int gy = 2 * (d / 6), gt = d - 2 * gy;
+  r.gt2 = gt / 2;
+  r.gy2 = gy / 2;
+  for (int m = 0; m < d / 2; ++m) {
+    int i, g;
+    if (m < r.gt2) {
+      i = m; g = gt;
+    } else if (m < r.gt2 + r.gy2) {
+      i = m - r.gt2; g = gy;
+    } else {
+      i = m - r.gt2 - r.gy2; g = gy;
+    }
+    r.theta[m] = std::pow(static_cast<double>(base), -2.0 * i / g);
+  }
+  return r;
 }
 
 cudaError_t launch_linear_apply(const Ctx& c, const void* q, const float* Hst, const float* Z,

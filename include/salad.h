@@ -20,9 +20,12 @@
  *     size must be 64.  N must be in [1, 262144].
  *   - All tensor pointers are DEVICE pointers, 16-byte aligned, owned by the
  *     caller.  Pointers documented as HOST are read during the call only.
- *   - The library never allocates, frees or synchronises.  Scratch memory is
- *     a caller-provided device workspace whose size is returned by the
- *     matching *_workspace_bytes query; 256-byte alignment is required.
+ *   - The library never allocates or frees device memory and never
+ *     synchronises.  Scratch memory is a caller-provided device workspace
+ *     whose size is returned by the matching *_workspace_bytes query;
+ *     256-byte alignment is required.  salad_forward alone creates, on its
+ *     first call on a device, two streams and three events of its own (kept
+ *     until the process exits) to run independent steps side by side.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) in call order.  All argument checks run on the host before any
  *     launch: an invalid call returns an error and enqueues nothing.
@@ -170,9 +173,15 @@ salad_status salad_dense_attn(const void* q, const void* k, const void* v,
                               int B, int H, int N, int d, void* o, salad_stream stream);
 
 /*
- * The whole hybrid layer (paper.rainbus.top 方法步骤详情 steps 2-6):
+ * The whole hybrid layer (paper.rainbus.top 方法步骤详情 steps 2-6, 8):
  * gate, sparse branch, linear branch, per-head projection W_lin (d x d,
  * right-multiplying row vectors: O_l' = O_l W_lin[h]), gated residual sum.
+ * The sparse pattern runs on `stream`; the gate and the linear branch run on
+ * two streams of the library forked from `stream` by an event and joined
+ * back to it before the attention kernel, so all work is ordered after the
+ * caller's earlier work on `stream` and before its later work.  Calls on one
+ * device are serialised on the host while they enqueue (the fork and join
+ * events are shared).
  */
 typedef struct salad_forward_args {
     const void* q;              /* bf16 [B,H,N,d] device */
@@ -214,10 +223,13 @@ typedef struct salad_forward_args {
     int32_t* idx_out;           /* optional device int32 [B,H,nb,topk] (out), may be NULL */
     void* workspace;            /* device scratch, >= salad_forward_workspace_bytes() */
     size_t workspace_bytes;
-    /* Optional profiling hook: NULL, or a HOST array of 5 cudaEvent_t that
-     * are recorded on `stream` at the start, after the gate, after the
-     * sparse-pattern step (selection or regrouping), after the linear
-     * state, and after the attention kernel. */
+    /* Optional profiling hook: NULL, or a HOST array of 5 cudaEvent_t,
+     * recorded at the start (on `stream`), when the gate ends, when the
+     * sparse-pattern step (selection or regrouping) ends, when the attention
+     * kernel starts (every input ready), and when it ends.  The gate and the
+     * linear branch run on two library-owned streams forked from `stream`
+     * and joined back before the attention, so only the last two events
+     * bound one kernel. */
     void* const* phase_events;
 } salad_forward_args;
 

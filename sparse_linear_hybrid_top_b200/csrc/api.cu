@@ -27,9 +27,33 @@ struct DevInfo {
   bool supported = false;
   int num_sms = 0;
   unsigned* err = nullptr;
+  // salad_forward's side streams and fork/join events (created on first use).
+  bool side_ready = false;
+  cudaStream_t side[2] = {nullptr, nullptr};
+  cudaEvent_t fork = nullptr, join_gate = nullptr, join_lin = nullptr;
+  std::mutex enqueue_mu;      // one forward at a time records and waits on the events
 };
 DevInfo g_dev[kMaxDevices];
 std::mutex g_mu;
+
+// The side streams and events of the current device, created once.
+DevInfo* side_resources() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.side_ready) {
+    for (int i = 0; i < 2; ++i)
+      if (cudaStreamCreateWithFlags(&d.side[i], cudaStreamNonBlocking) != cudaSuccess)
+        return nullptr;
+    if (cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&d.join_gate, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&d.join_lin, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+    d.side_ready = true;
+  }
+  return &d;
+}
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -417,23 +441,40 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   Ctx c;
   if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
 
+  DevInfo* dv = side_resources();
+  if (dv == nullptr) return SALAD_ERR_CUDA;
+  // Fork/join on per-device events: enqueues of concurrent calls must not
+  // interleave.
+  std::lock_guard<std::mutex> enqueue_lock(dv->enqueue_mu);
+
   char* ws = static_cast<char*>(a->workspace);
   const int B = a->B, H = a->H, N = a->N, d = a->d;
   const int nb = nblocks(N);
-  cudaError_t e;
-  auto mark = [&](int i) -> bool {
+  // Three chains run side by side: the sparse pattern on the caller's
+  // stream, the gate and the linear branch on two side streams forked from
+  // it; the attention waits for both.  The side chains are joined back even
+  // when a launch fails, so the caller's stream never runs ahead of them.
+  Ctx cg = c, cl = c;
+  cg.stream = dv->side[0];
+  cl.stream = dv->side[1];
+  auto mark = [&](int i, cudaStream_t st) -> bool {
     if (a->phase_events == nullptr || a->phase_events[i] == nullptr) return true;
-    return cudaEventRecord(static_cast<cudaEvent_t>(a->phase_events[i]), c.stream) == cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(a->phase_events[i]), st) == cudaSuccess;
   };
-  if (!mark(0)) return SALAD_ERR_CUDA;
-  // 1. gate (paper.rainbus.top 方法步骤详情 step 5)
+  if (!mark(0, c.stream)) return SALAD_ERR_CUDA;
+  if (cudaEventRecord(dv->fork, c.stream) != cudaSuccess ||
+      cudaStreamWaitEvent(cg.stream, dv->fork, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(cl.stream, dv->fork, 0) != cudaSuccess)
+    return SALAD_ERR_CUDA;
+  bool ok = true;
+  auto check = [&](cudaError_t e) { ok = ok && e == cudaSuccess; };
+
+  // 1. gate (paper.rainbus.top 方法步骤详情 step 5), side stream 0
   float* s = a->s_out != nullptr ? a->s_out : reinterpret_cast<float*>(ws + L.s);
-  if (override_gate) {
-    e = launch_fill_f32(c, s, a->gate_override, B);
-  } else {
-    e = launch_gate(c, a->x, a->w_gate, a->gate_bias, B, N, a->D, s, ws + L.gate);
-  }
-  if (e != cudaSuccess || !mark(1)) return SALAD_ERR_CUDA;
+  if (override_gate) check(launch_fill_f32(cg, s, a->gate_override, B));
+  else check(launch_gate(cg, a->x, a->w_gate, a->gate_bias, B, N, a->D, s, ws + L.gate));
+  ok = ok && mark(1, cg.stream);
+  check(cudaEventRecord(dv->join_gate, cg.stream));
 
   AttnArgs at;
   std::memset(&at, 0, sizeof(at));
@@ -445,15 +486,37 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   at.s = s;
   // NaN compares false: never drop.
   at.drop = std::isnan(a->drop_threshold) ? 0.0f : a->drop_threshold;
-  // 2. sparse-branch pattern (ijyty.com 1.1 / 1.2)
+
+  // 3. linear branch state and the folded projection G = H W_lin (steps 3-4),
+  // side stream 1.  Branch dropping reads the gate's output: only then does
+  // this chain wait for the gate.
+  float* Hst = reinterpret_cast<float*>(ws + L.hst);
+  float* Z = reinterpret_cast<float*>(ws + L.z);
+  void* G = ws + L.g;
+  BranchDrop drop;   // default: never drop, reads nothing
+  if (at.drop > 0.0f) {
+    // Only here does this chain read s: it waits for the gate first.
+    check(cudaStreamWaitEvent(cl.stream, dv->join_gate, 0));
+    drop.s = s;
+    drop.thr = at.drop;
+  }
+  Rope3D rope;
+  if (a->rope3d) rope = make_rope3d(d, a->F, a->Hh, a->Wh, a->rope_base);
+  at.rope = rope;
+  if (ok)
+    check(launch_linear_state(cl, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, a->w_lin, G, drop,
+                              rope));
+  check(cudaEventRecord(dv->join_lin, cl.stream));
+  at.Gimg = G;
+  at.Z = Z;
+
+  // 2. sparse-branch pattern (ijyty.com 1.1 / 1.2), the caller's stream
   if (a->mode == SALAD_MODE_TOPK) {
     int32_t* idx = a->idx_out != nullptr ? a->idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
-    e = launch_select(c, a->q, a->k, B, H, N, d, a->topk, idx, ws + L.sel);
-    if (e != cudaSuccess) return SALAD_ERR_CUDA;
     int32_t* lists = reinterpret_cast<int32_t*>(ws + L.lists);
     int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
-    e = launch_pair_union(c, idx, B * H, nb, a->topk, lists, counts);
-    if (e != cudaSuccess) return SALAD_ERR_CUDA;
+    if (ok) check(launch_select(c, a->q, a->k, B, H, N, d, a->topk, idx, ws + L.sel));
+    if (ok) check(launch_pair_union(c, idx, B * H, nb, a->topk, lists, counts));
     at.mode = kModeTopk;
     at.lists = lists;
     at.counts = counts;
@@ -464,9 +527,10 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
       int sel[kMaxHeads];
       for (int h = 0; h < H; ++h)
         if (L.slot[h] >= 0) sel[L.slot[h]] = h;
-      e = launch_gather_heads_space_major(c, a->q, a->k, a->v, ws + L.qp, ws + L.kp, ws + L.vp, B,
-                                          H, N, d, a->F, a->Hh, a->Wh, sel, L.Hs);
-      if (e != cudaSuccess) return SALAD_ERR_CUDA;
+      if (ok)
+        check(launch_gather_heads_space_major(c, a->q, a->k, a->v, ws + L.qp, ws + L.kp,
+                                              ws + L.vp, B, H, N, d, a->F, a->Hh, a->Wh, sel,
+                                              L.Hs));
       at.qp = ws + L.qp;
       at.kp = ws + L.kp;
       at.vp = ws + L.vp;
@@ -476,25 +540,14 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   } else {
     at.mode = kModeDense;
   }
-  if (!mark(2)) return SALAD_ERR_CUDA;
-  // 3. linear branch state and the folded projection G = H W_lin (steps 3-4)
-  float* Hst = reinterpret_cast<float*>(ws + L.hst);
-  float* Z = reinterpret_cast<float*>(ws + L.z);
-  void* G = ws + L.g;
-  BranchDrop drop;
-  drop.s = s;
-  drop.thr = at.drop;
-  Rope3D rope;
-  if (a->rope3d) rope = make_rope3d(d, a->F, a->Hh, a->Wh, a->rope_base);
-  at.rope = rope;
-  e = launch_linear_state(c, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, a->w_lin, G, drop,
-                          rope);
-  if (e != cudaSuccess || !mark(3)) return SALAD_ERR_CUDA;
-  at.Gimg = G;
-  at.Z = Z;
-  // 4. sparse attention with the gated residual epilogue (steps 2, 6)
-  e = launch_attention(c, at);
-  if (e != cudaSuccess || !mark(4)) return SALAD_ERR_CUDA;
+  ok = ok && mark(2, c.stream);
+
+  // Join the side chains, then 4. sparse attention with the gated residual
+  // epilogue (steps 2, 6).
+  const bool joined = cudaStreamWaitEvent(c.stream, dv->join_gate, 0) == cudaSuccess &&
+                      cudaStreamWaitEvent(c.stream, dv->join_lin, 0) == cudaSuccess;
+  if (!ok || !joined || !mark(3, c.stream)) return SALAD_ERR_CUDA;
+  if (launch_attention(c, at) != cudaSuccess || !mark(4, c.stream)) return SALAD_ERR_CUDA;
   return SALAD_OK;
 }
 

@@ -149,6 +149,25 @@ def test_forward_rope3d(salad, w):
         assert torch.equal(o, _plan(salad, w, dev).run())
 
 
+@pytest.mark.parametrize("fill", [-1.0, float("nan")])
+def test_forward_never_reads_the_gate_buffer_early(salad, fill):
+    # The gate and the linear branch run side by side; without dropping, the
+    # linear branch must not read the gate's output buffer at all, so stale
+    # contents there (negative, NaN) change nothing.
+    w = RAGGED128
+    inp = generate(w)
+    dev = device_inputs(inp)
+    plan = _plan(salad, w, dev)
+    for _ in range(3):
+        plan.s_out.fill_(fill)
+        o = plan.run().clone()
+        torch.cuda.synchronize()
+        salad.check_error()
+        ref = oracle.forward(inp, mode="topk", block=w.block, topk=w.topk, eps=w.eps,
+                             idx_override=_selection_used(w, inp, plan.idx_out))
+        assert_close(o, ref["o"], f"forward after s_out filled with {fill}")
+
+
 def test_forward_is_deterministic(salad):
     w = RAGGED128
     dev = device_inputs(generate(w))

@@ -9,85 +9,81 @@
 // algebraic regrouping of (phi(Q) H / den) W_lin).
 //
 // Tiling for sm_100a.  One work item is a pair of 64-row query blocks
-// (M = 128 rows, the full tcgen05 datapath).  Its key tiles are the merged,
+// (M = 128 rows, the full tcgen05 datapath).  Its key blocks are the merged,
 // ascending list of the blocks either query block keeps (Top-K), the band of
-// blocks its rows' windows touch (ST-SWA) or all blocks (dense).  For each
-// 64-key tile:  S = Q K^T  (A = Q from TMEM, B = K tile from smem, N = 64),
-// P = exp2(S*c - m) written back over S in TMEM as bf16, O += P V
-// (A = P from TMEM, B = V tile from smem, MN-major).  Rows whose query block
-// did not keep a tile get P = 0 for it.
+// blocks its rows' windows touch (ST-SWA) or all blocks (dense), taken two
+// at a time: a tile holds 128 keys, so the QK MMA has N = 128 (an M = 128
+// tcgen05.mma occupies the tensor pipe for ~64 cycles at any N <= 128).
+// A query block that did not keep one of a tile's blocks gets P = 0 there.
 //
-// S tiles hold 128 keys (two 64-key blocks of the list), so the QK MMA has
-// N = 128: a tcgen05.mma with M = 128 occupies the tensor pipe for at least
-// ~64 cycles whatever its N, which leaves an N = 64 MMA at half rate.  The K
-// ring keeps consecutive 64-key stages contiguous inside each 128-byte-
-// swizzled d-half slab, so a block pair is one B operand.
+// Split-K ping-pong.  The item's tiles alternate between two slots, A (even
+// tiles) and B (odd tiles), each with its own S and O accumulators in TMEM
+// and its own running max and sum; the two partial results are merged once,
+// at the end of the item.  The single MMA thread interleaves the slots: while
+// the tensor pipe runs slot A's PV(t) and QK(t+2), slot B's softmax runs, and
+// the reverse.  Each slot's softmax has four warps, one per TMEM lane
+// quarter, one query row per thread: a pass over the tile's two 64-key halves
+// finds the row max, a second pass exponentiates (exp2, running max raised
+// lazily: O is rescaled only when it grows by more than 2^8) and writes P
+// back over S as bf16.  S = Q K^T is an SS MMA (Q from shared memory, TMA-
+// loaded, double-buffered across items); O += P V a TS MMA (P from TMEM).
+// QK(t+2) is issued right behind PV(t) into the buffer PV(t) reads (tcgen05
+// MMAs of one thread execute in issue order).
 //
-// Eight softmax warps: four row quarters (the TMEM lane groups) times two
-// column halves.  The two warps holding a row exchange their partial row max
-// every tile (through a bounded mbarrier), so both apply the same running max
-// and O stays a single accumulator; each warp exponentiates 64 of the 128
-// columns, rescales its half of O when the max grows by more than 2^8, and
-// writes its half of the output.  S is double-buffered so the QK of the next
-// tile runs during the softmax of this one.  The linear term
-// s_b * phi(Q) G / (phi(Q) Z + eps) is one more MMA (A = phi(Q) from TMEM,
-// B = the bf16 image of G streamed into the V slots of a ring stage) into the
-// S_0 columns, which are free once the last PV has run.
+// K tiles, V tiles and the item's G image stream through one ring of stages
+// in the order the MMA thread consumes them: K0, K1, then V(t), K(t+2) for
+// each tile t, then G.  The linear term s_b * phi(Q) G / (phi(Q) Z + eps) is
+// one more SS MMA (A = phi(Q), written over the item's Q buffer by the
+// softmax threads once every QK has run; B = the G image) into slot A's S
+// columns.  The epilogue merges the slots, adds the linear term and writes
+// the rows; each slot writes half of the columns.
 //
 // Warp roles (320 threads, one CTA per SM, persistent over work items):
-//   warp 0      TMA producer: K and V blocks (64 x d, 128B swizzle), two per
-//               ring stage, and the G image.
+//   warp 0      TMA producer: Q (two 64-row boxes per d-slab), K and V
+//               tiles (64 x 64 boxes, 128B swizzle), the G image.
 //   warp 1      TMEM allocator and the single MMA-issuing thread.
-//   warps 2..5  softmax, column half 0; also load Q and phi(Q).
-//   warps 6..9  softmax, column half 1.
-// TMEM columns (d = 128): O [0,128) S_0 [128,256) S_1 [256,384) Q [384,448)
-// phi(Q) [448,512); the linear term lands in S_0.
+//   warps 2..5  slot A softmax; warp w holds TMEM lane quarter w % 4.
+//   warps 6..9  slot B softmax.
+// TMEM columns (d = 128): O_A [0,128) O_B [128,256) S_A [256,384)
+// S_B [384,512); the linear term lands in S_A.
 //
 // Barrier discipline: an mbarrier parity wait is only sound when the waiter is
 // at most one phase behind.  Every barrier is observed by each of its waiters
-// at every phase: in particular each softmax warp waits for its previous PV
-// once per tile (after computing and storing P, so the wait overlaps its own
-// work), rescales its O only then, and only then releases the tile.  Every
-// wait is bounded; a wait that runs out raises the device error word and the
-// CTA leaves through the common teardown (loads drained, MMAs committed, TMEM
-// freed).
+// at every phase: in particular each softmax warp waits for its slot's
+// previous PV once per tile, rescales its O only then, and only then releases
+// the tile.  Every wait is bounded; a wait that runs out raises the device
+// error word and the CTA leaves through the common teardown (loads drained,
+// MMAs committed, TMEM accesses completed, TMEM freed).
 #include "common.cuh"
 #include "internal.h"
 
 namespace salad {
 namespace {
 
-constexpr int kSlab = 64 * 128;
+constexpr int kSlab = 64 * 128;   // one 64-row x 128-byte swizzled slab
 
 template <int D, bool HYB>
 struct AT {
-  static constexpr int kKS = 6;                          // 64-key stages (even: pairs never wrap)
-  static constexpr int kPairs = kKS / 2;                 // ring stages of two blocks
   static constexpr int kHalves = D / 64;                 // 128-byte d-slabs per row
-  static constexpr int kTile = kHalves * kSlab;          // one 64-key K (or V) block
-  static constexpr int kKRingHalf = kKS * kSlab;         // one d-slab of the K ring
-  static constexpr int kKRing = kHalves * kKRingHalf;
-  static constexpr int kVRing = kKS * kTile;
-  static constexpr int kGImg = D * D * 2;                // bf16 G image bytes (own buffer)
-  static constexpr int kXchg = (2 * 2 * 128 + 128) * 4;  // row max/sum per parity, den
-  static constexpr int kBarBytes = 256;
-  // The dynamic shared memory is declared 1024-byte aligned (the 128-byte
-  // swizzle atoms need it), so no slack is reserved for aligning it.
-  static constexpr int kSmemUsed = kKRing + kVRing + kGImg + kXchg + kBarBytes;
+  static constexpr int kRowSlab = 128 * 128;             // 128 rows of one d-slab
+  static constexpr int kQBuf = kHalves * kRowSlab;       // 128 rows of Q (or phi(Q))
+  static constexpr int kStage = kHalves * kRowSlab;      // 128 keys of K or V, or a G image
+  static constexpr int kStages = D == 128 ? 4 : 8;
+  static constexpr int kGImg = D * D * 2;
+  static_assert(kGImg <= kStage, "the G image fills one ring stage");
+  static constexpr int kXchg = 2 * 128 * 16;             // per slot and row: m, l, den part
+  static constexpr int kBarBytes = 512;
+  static constexpr int kSmemUsed = 2 * kQBuf + kStages * kStage + kXchg + kBarBytes;
   static_assert(kSmemUsed <= 227 * 1024, "shared memory budget");
   // At least ~half of the SM's shared memory, so one CTA (and its 512 TMEM
   // columns) occupies each SM.
   static constexpr int kSmem = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
   // TMEM columns.
-  static constexpr uint32_t kO = 0;            // D columns
-  static constexpr uint32_t kS0 = D;           // 128 columns (P aliases the first 64)
-  static constexpr uint32_t kS1 = D + 128;     // 128 columns
-  static constexpr uint32_t kL = D;            // linear term, D columns over S_0
-  static constexpr uint32_t kQ = D + 256;      // D/2 columns (A operand)
-  static constexpr uint32_t kPQ = kQ + D / 2;  // D/2 columns (A operand)
+  __host__ __device__ static constexpr uint32_t o_col(int slot) { return slot ? D : 0; }
+  __host__ __device__ static constexpr uint32_t s_col(int slot) { return 2 * D + (slot ? 128 : 0); }
+  static constexpr uint32_t kL = 2 * D;        // linear term, D columns over S_A
   static constexpr uint32_t kCols = 512;
-  static_assert(kPQ + D / 2 <= kCols, "TMEM budget");
-  static_assert(D <= 128, "the linear term must fit S_0");
+  static_assert(2 * D + 256 <= kCols, "TMEM budget");
 };
 
 struct Params {
@@ -152,15 +148,13 @@ __device__ __forceinline__ bool lin_on(const Params& P, int b) {
   return !(g < P.drop);
 }
 
-__device__ __forceinline__ void tile_of(const Item& it, int t, int mode, int& j, int& mask) {
-  if (mode == kModeTopk) {
-    const int e = __ldg(it.list + t);
-    j = e & 0xFFFF;
-    mask = e >> 16;
-  } else {
-    j = it.jlo + t;
-    mask = 3;
-  }
+// Entry t of the item's key-block list: j | mask << 16 (mask bit 0: the
+// first query block of the pair keeps block j, bit 1: the second); 0 past
+// the end.  Band and dense items keep every block of their range for both.
+__device__ __forceinline__ int list_entry(const Item& it, int t, int mode) {
+  if (t >= it.ntiles) return 0;
+  if (mode == kModeTopk) return __ldg(it.list + t);
+  return (it.jlo + t) | (3 << 16);
 }
 
 // Maximum of 64 values by a tree of three-input maxima (64 -> 22 -> 8 -> 3 -> 1).
@@ -198,73 +192,76 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 }
 
 template <int D, bool HYB>
-__global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CUtensorMap mk,
+__global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CUtensorMap mq,
+                                                      const __grid_constant__ CUtensorMap mk,
                                                       const __grid_constant__ CUtensorMap mv,
+                                                      const __grid_constant__ CUtensorMap mqp,
                                                       const __grid_constant__ CUtensorMap mkp,
                                                       const __grid_constant__ CUtensorMap mvp,
                                                       const __grid_constant__ Params P) {
   using C = AT<D, HYB>;
-  constexpr int NP = C::kPairs;
+  constexpr int NS = C::kStages;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // The layout below assumes the declared alignment; refuse to run without it.
   if (reinterpret_cast<uintptr_t>(smem_raw) & 1023u) {
     if (threadIdx.x == 0) atomicOr(P.err, kErrLayout);
     return;
   }
-  unsigned char* sm = smem_raw;
-  unsigned char* kring = sm;                         // [d-slab][kKS x 64 rows x 128 B]
-  unsigned char* vring = sm + C::kKRing;             // [kKS][d-slab][64 rows x 128 B]
-  unsigned char* gbuf = vring + C::kVRing;           // G image of the current item's head
-  float* xrow = reinterpret_cast<float*>(gbuf + C::kGImg);    // [parity][half][128] row max / sum
-  float* xden = xrow + 2 * 2 * 128;                            // [128] phi(q) . Z + eps
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(xrow) + C::kXchg);
-  // bars: full[NP] empty[NP] s_full[2] p_full[2] o_done q_ready lin_done drain x_row[4] g_full
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NP + 13);
-  static_assert((2 * NP + 13) * 8 + 8 <= C::kBarBytes, "barrier region");
+  unsigned char* qbuf = smem_raw;                          // [2][d-slab][128 rows x 128 B]
+  unsigned char* ring = qbuf + 2 * C::kQBuf;               // [NS] stages
+  float4* xchg = reinterpret_cast<float4*>(ring + NS * C::kStage);  // [slot][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(xchg) + C::kXchg);
+  // bars: full[NS] empty[NS] q_full[2] q_empty[2] s_full[2] p_full[2] o_done[2] q_free
+  //       phiq_ready lin_done x_bar epi_done drain
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NS + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  static_assert((2 * NS + 16) * 8 + 8 <= C::kBarBytes, "barrier region");
 
-  auto full = [&](int p) { return smem_u32(bars + p); };
-  auto empty = [&](int p) { return smem_u32(bars + NP + p); };
-  auto s_full = [&](int b) { return smem_u32(bars + 2 * NP + b); };
-  auto p_full = [&](int b) { return smem_u32(bars + 2 * NP + 2 + b); };
-  const uint32_t o_done = smem_u32(bars + 2 * NP + 4);
-  const uint32_t q_ready = smem_u32(bars + 2 * NP + 5);
-  const uint32_t lin_done = smem_u32(bars + 2 * NP + 6);
-  const uint32_t drain = smem_u32(bars + 2 * NP + 7);
-  auto x_row = [&](int q) { return smem_u32(bars + 2 * NP + 8 + q); };
-  const uint32_t g_full = smem_u32(bars + 2 * NP + 12);
-  // Shared-memory addresses of the blocks of ring stage (pair) p.
-  auto k_addr = [&](int p, int half) {   // rows of block 2p (then 2p+1) of one d-slab
-    return smem_u32(kring + half * C::kKRingHalf + 2 * p * kSlab);
-  };
-  auto v_addr = [&](int p, int which) {  // V block 2p + which
-    return smem_u32(vring + (2 * p + which) * C::kTile);
-  };
+  auto full = [&](int i) { return smem_u32(bars + i); };
+  auto empty = [&](int i) { return smem_u32(bars + NS + i); };
+  auto q_full = [&](int i) { return smem_u32(bars + 2 * NS + i); };
+  auto q_empty = [&](int i) { return smem_u32(bars + 2 * NS + 2 + i); };
+  auto s_full = [&](int i) { return smem_u32(bars + 2 * NS + 4 + i); };
+  auto p_full = [&](int i) { return smem_u32(bars + 2 * NS + 6 + i); };
+  auto o_done = [&](int i) { return smem_u32(bars + 2 * NS + 8 + i); };
+  const uint32_t q_free = smem_u32(bars + 2 * NS + 10);
+  const uint32_t phiq_ready = smem_u32(bars + 2 * NS + 11);
+  const uint32_t lin_done = smem_u32(bars + 2 * NS + 12);
+  const uint32_t x_bar = smem_u32(bars + 2 * NS + 13);
+  const uint32_t epi_done = smem_u32(bars + 2 * NS + 14);
+  const uint32_t drain = smem_u32(bars + 2 * NS + 15);
+  auto q_addr = [&](int b) { return smem_u32(qbuf + b * C::kQBuf); };
+  auto st_addr = [&](long long c) { return smem_u32(ring + static_cast<int>(c % NS) * C::kStage); };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const long long total = static_cast<long long>(P.B) * P.H * P.npairs;
   const unsigned long long wait_ns = P.wait_ns;
 
   if (threadIdx.x == 0) {
-    for (int p = 0; p < NP; ++p) {
-      mbar_init(full(p), 1);
-      mbar_init(empty(p), 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(full(i), 1);
+      mbar_init(empty(i), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full(b), 1);
-      mbar_init(p_full(b), 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full(i), 1);
+      mbar_init(q_empty(i), 1);
+      mbar_init(s_full(i), 1);
+      mbar_init(p_full(i), 4);   // the slot's four softmax warps
+      mbar_init(o_done(i), 1);
     }
-    mbar_init(o_done, 1);
-    mbar_init(q_ready, 8);   // half 0 after writing Q, half 1 after its previous epilogue
+    mbar_init(q_free, 1);
+    mbar_init(phiq_ready, 8);    // every softmax warp has written its part of phi(Q)
     mbar_init(lin_done, 1);
+    mbar_init(x_bar, 8);         // every softmax warp has posted its row's m, l and den part
+    mbar_init(epi_done, 8);      // every softmax warp has finished the item's epilogue
     mbar_init(drain, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(x_row(q), 2);   // the two warps of a row quarter
-    mbar_init(g_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    tma_prefetch_map(&mq);
     tma_prefetch_map(&mk);
     tma_prefetch_map(&mv);
     if (P.Hs > 0) {
+      tma_prefetch_map(&mqp);
       tma_prefetch_map(&mkp);
       tma_prefetch_map(&mvp);
     }
@@ -281,53 +278,74 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
   if (warp == 0) {
     if (lane == 0) {
       // ================================================= TMA producer
-      long long pc = 0;   // ring stages filled so far
+      long long sc = 0;   // ring stages filled so far
+      uint32_t qc = 0;    // items started (Q buffer qc & 1)
+      uint32_t q_issued = 0;   // Q loads issued (drained at the end)
       bool ok = true;
-      for (long long w = blockIdx.x; w < total && ok; w += gridDim.x) {
+      for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++qc) {
         const Item it = make_item(P, w);
+        const CUtensorMap* qm = it.slot >= 0 ? &mqp : &mq;
         const CUtensorMap* km = it.slot >= 0 ? &mkp : &mk;
         const CUtensorMap* vm = it.slot >= 0 ? &mvp : &mv;
         const int z = it.slot >= 0 ? it.b * P.Hs + it.slot : it.bh;
-        const int npair = (it.ntiles + 1) / 2;
-        if (w + gridDim.x < total) {
-          // The next item's rows of Q into L2 (one contiguous run), an item
-          // ahead of the softmax warps that load them.
-          const Item nx = make_item(P, w + gridDim.x);
-          const __nv_bfloat16* qsrc =
-              nx.slot >= 0 ? P.qp + (static_cast<long long>(nx.b) * P.Hs + nx.slot) * P.N * D
-                           : P.q + static_cast<long long>(nx.bh) * P.N * D;
-          const int rows = min(128, P.N - nx.p * 128);
-          prefetch_l2(qsrc + static_cast<long long>(nx.p) * 128 * D,
-                      static_cast<uint32_t>(rows) * D * 2);
+        const int T = (it.ntiles + 1) / 2;
+        const bool lin = HYB && lin_on(P, it.b);
+        // Q rows of the item (two 64-row boxes per d-slab; rows past N read 0).
+        const int qb = static_cast<int>(qc & 1);
+        if (qc >= 2 && !mbar_wait(q_empty(qb), ((qc - 2) / 2) & 1, wait_ns, abort_flag)) {
+          ok = false;
+          break;
         }
-        for (int u = 0; u < npair; ++u, ++pc) {
-          const int p = static_cast<int>(pc % NP);
-          const long long n = pc / NP;
-          if (n > 0 && !mbar_wait(empty(p), static_cast<uint32_t>((n - 1) & 1), wait_ns, abort_flag)) {
-            raise_timeout(P.err, abort_flag);
-            ok = false;
-            break;
-          }
-          if (u < npair) {
-            const int nblk = (2 * u + 1 < it.ntiles) ? 2 : 1;
-            mbar_arrive_expect_tx(full(p), nblk * 2 * C::kTile);
-            for (int x = 0; x < nblk; ++x) {
-              int j, mask;
-              tile_of(it, 2 * u + x, P.mode, j, mask);
+        mbar_arrive_expect_tx(q_full(qb), C::kQBuf);
 #pragma unroll
-              for (int hh = 0; hh < D / 64; ++hh) {
-                tma_load_3d(k_addr(p, hh) + x * kSlab, km, full(p), hh * 64, j * 64, z);
-                tma_load_3d(v_addr(p, x) + hh * kSlab, vm, full(p), hh * 64, j * 64, z);
-              }
+        for (int hh = 0; hh < D / 64; ++hh)
+#pragma unroll
+          for (int rb = 0; rb < 2; ++rb)
+            tma_load_3d(q_addr(qb) + hh * C::kRowSlab + rb * kSlab, qm, q_full(qb), hh * 64,
+                        it.p * 128 + rb * 64, z);
+        q_issued = qc + 1;
+        // The item's loads in the MMA thread's order: K0, K1, then V(t) and
+        // K(t+2) for each tile t, then the G image.
+        auto push = [&](int kind, int t) -> bool {
+          const int si = static_cast<int>(sc % NS);
+          const long long n = sc / NS;
+          if (n > 0 && !mbar_wait(empty(si), static_cast<uint32_t>((n - 1) & 1), wait_ns, abort_flag))
+            return false;
+          const uint32_t dst = st_addr(sc);
+          ++sc;
+          if (kind == 2) {
+            mbar_arrive_expect_tx(full(si), C::kGImg);
+            bulk_load(dst, P.Gimg + static_cast<long long>(it.bh) * D * D, C::kGImg, full(si));
+            return true;
+          }
+          const int nblk = (2 * t + 1 < it.ntiles) ? 2 : 1;
+          mbar_arrive_expect_tx(full(si), nblk * (D / 64) * kSlab);
+          for (int x = 0; x < nblk; ++x) {
+            const int j = list_entry(it, 2 * t + x, P.mode) & 0xFFFF;
+#pragma unroll
+            for (int hh = 0; hh < D / 64; ++hh) {
+              if (kind == 0)   // K: [d-slab][128 rows]; block x from row 64x
+                tma_load_3d(dst + hh * C::kRowSlab + x * kSlab, km, full(si), hh * 64, j * 64, z);
+              else             // V: [block][d-slab][64 rows]
+                tma_load_3d(dst + x * (D / 64) * kSlab + hh * kSlab, vm, full(si), hh * 64, j * 64, z);
             }
           }
-        }
+          return true;
+        };
+        ok = push(0, 0) && (T < 2 || push(0, 1));
+        for (int t = 0; t < T && ok; ++t) ok = push(1, t) && (t + 2 >= T || push(0, t + 2));
+        if (ok && lin) ok = push(2, 0);
       }
+      if (!ok) raise_timeout(P.err, abort_flag);
       // Drain every issued load before leaving.
-      for (int p = 0; p < NP && p < pc; ++p) {
-        const long long last = p + ((pc - 1 - p) / NP) * NP;
-        if (!mbar_wait(full(p), static_cast<uint32_t>((last / NP) & 1), wait_ns, nullptr))
+      for (int i = 0; i < NS && i < sc; ++i) {
+        const long long last = i + ((sc - 1 - i) / NS) * NS;
+        if (!mbar_wait(full(i), static_cast<uint32_t>((last / NS) & 1), wait_ns, nullptr))
           atomicOr(P.err, kErrTimeout);
+      }
+      for (uint32_t b = 0; b < 2 && b < q_issued; ++b) {
+        const uint32_t uses = (q_issued - b + 1) / 2;   // Q loads into buffer b
+        if (!mbar_wait(q_full(b), (uses - 1) & 1, wait_ns, nullptr)) atomicOr(P.err, kErrTimeout);
       }
     }
   } else if (warp == 1) {
@@ -336,72 +354,83 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
       constexpr uint32_t idesc_lin = idesc_bf16(128, D, false, false);
-      long long pc = 0;
-      uint32_t ic = 0;
-      uint32_t pf[2] = {0, 0};
+      long long sc = 0;   // ring stages consumed so far
+      uint32_t ic = 0, lc = 0, pf[2] = {0, 0};
       bool ok = true;
-      auto wait_full = [&](long long c) -> bool {
-        return mbar_wait(full(static_cast<int>(c % NP)), static_cast<uint32_t>((c / NP) & 1),
+      auto wait_stage = [&]() -> bool {
+        return mbar_wait(full(static_cast<int>(sc % NS)), static_cast<uint32_t>((sc / NS) & 1),
                          wait_ns, abort_flag);
       };
-      auto issue_qk = [&](long long c, int b) {
-        const int p = static_cast<int>(c % NP);
-        const uint32_t sbuf = b ? C::kS1 : C::kS0;
+      // S_slot = Q K(t)^T from the K tile in the current stage.
+      auto issue_qk = [&](int qb, int slot) {
+        const uint32_t ka = st_addr(sc), qa = q_addr(qb);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          mma_ts(tmem + sbuf, tmem + C::kQ + ks * 8,
-                 sdesc_sw128(k_addr(p, ks / 4) + (ks % 4) * 32, 16, 1024), idesc_qk,
+          mma_ss(tmem + C::s_col(slot),
+                 sdesc_sw128(qa + (ks / 4) * C::kRowSlab + (ks % 4) * 32, 16, 1024),
+                 sdesc_sw128(ka + (ks / 4) * C::kRowSlab + (ks % 4) * 32, 16, 1024), idesc_qk,
                  ks > 0 ? 1u : 0u);
-        mma_commit(s_full(b));
+        mma_commit(empty(static_cast<int>(sc % NS)));
+        mma_commit(s_full(slot));
+        ++sc;
       };
-      uint32_t lc = 0;   // items with a linear term so far
       for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++ic) {
         const Item it = make_item(P, w);
-        const int npair = (it.ntiles + 1) / 2;
-        if (!mbar_wait(q_ready, ic & 1, wait_ns, abort_flag)) { ok = false; break; }
+        const int T = (it.ntiles + 1) / 2;
+        const bool lin = HYB && lin_on(P, it.b);
+        const int qb = static_cast<int>(ic & 1);
+        // The previous item's epilogue has read O, S and the linear term.
+        if (ic > 0 && !mbar_wait(epi_done, (ic - 1) & 1, wait_ns, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(q_full(qb), (ic / 2) & 1, wait_ns, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        for (int u = 0; u < 2 && u < npair; ++u) {
-          if (!wait_full(pc + u)) { ok = false; break; }
+        for (int t = 0; t < 2 && t < T; ++t) {
+          if (!wait_stage()) { ok = false; break; }
           tc_fence_after();
-          issue_qk(pc + u, u);
+          issue_qk(qb, t);
         }
         if (!ok) break;
-        for (int u = 0; u < npair; ++u) {
-          const int b = u & 1;
-          if (!mbar_wait(p_full(b), pf[b] & 1, wait_ns, abort_flag)) { ok = false; break; }
-          ++pf[b];
+        if (T <= 2) mma_commit(q_free);   // every QK of the item is issued
+        for (int t = 0; t < T; ++t) {
+          const int slot = t & 1;
+          if (!mbar_wait(p_full(slot), pf[slot] & 1, wait_ns, abort_flag)) { ok = false; break; }
+          ++pf[slot];
+          if (!wait_stage()) { ok = false; break; }
           tc_fence_after();
-          const int p = static_cast<int>((pc + u) % NP);
-          const uint32_t pbuf = b ? C::kS1 : C::kS0;
-          const int nks = (2 * u + 1 < it.ntiles) ? 8 : 4;   // K-steps: 16 keys each
+          const uint32_t va = st_addr(sc);
+          const int nks = (2 * t + 1 < it.ntiles) ? 8 : 4;   // K-steps: 16 keys each
           for (int ks = 0; ks < nks; ++ks)
-            mma_ts(tmem + C::kO, tmem + pbuf + ks * 8,
-                   sdesc_sw128(v_addr(p, ks / 4) + (ks % 4) * 2048, kSlab, 1024), idesc_pv,
-                   (u > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(empty(p));
-          mma_commit(o_done);
-          if (u + 2 < npair) {
-            if (!wait_full(pc + u + 2)) { ok = false; break; }
+            mma_ts(tmem + C::o_col(slot), tmem + C::s_col(slot) + ks * 8,
+                   sdesc_sw128(va + (ks / 4) * (D / 64) * kSlab + (ks % 4) * 2048, kSlab, 1024),
+                   idesc_pv, (t >= 2 || ks > 0) ? 1u : 0u);
+          mma_commit(empty(static_cast<int>(sc % NS)));
+          mma_commit(o_done(slot));
+          ++sc;
+          if (t + 2 < T) {
+            if (!wait_stage()) { ok = false; break; }
             tc_fence_after();
-            issue_qk(pc + u + 2, b);   // same S buffer: runs after this PV in issue order
+            issue_qk(qb, slot);   // same S buffer: runs after this PV in issue order
+            if (t + 3 == T) mma_commit(q_free);   // that was the item's last QK
           }
         }
         if (!ok) break;
-        pc += npair;
-        if (HYB && lin_on(P, it.b)) {
-          // Linear term into S_0 (free once the last PV has run): L = phi(Q) G,
-          // B = the item's G image in its own buffer.
-          if (!mbar_wait(g_full, lc & 1, wait_ns, abort_flag)) { ok = false; break; }
-          ++lc;
+        if (lin) {
+          // Linear term into S_A (every S of the item has been read):
+          // L = phi(Q) G, A = phi(Q) over the Q buffer, B = the G image.
+          if (!mbar_wait(phiq_ready, lc & 1, wait_ns, abort_flag)) { ok = false; break; }
+          if (!wait_stage()) { ok = false; break; }
           tc_fence_after();
-          const uint32_t gaddr = smem_u32(gbuf);
+          const uint32_t ga = st_addr(sc), qa = q_addr(qb);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
-            mma_ts(tmem + C::kL, tmem + C::kPQ + ks * 8,
-                   sdesc_sw128(gaddr + (ks / 4) * (D * 128) + (ks % 4) * 32, 16, 1024), idesc_lin,
+            mma_ss(tmem + C::kL, sdesc_sw128(qa + (ks / 4) * C::kRowSlab + (ks % 4) * 32, 16, 1024),
+                   sdesc_sw128(ga + (ks / 4) * (D * 128) + (ks % 4) * 32, 16, 1024), idesc_lin,
                    ks > 0 ? 1u : 0u);
+          mma_commit(empty(static_cast<int>(sc % NS)));
           mma_commit(lin_done);
+          ++sc;
+          ++lc;
         }
+        mma_commit(q_empty(qb));   // the item's Q buffer is free once these MMAs ran
       }
       if (!ok) raise_timeout(P.err, abort_flag);
       mma_commit(drain);
@@ -409,262 +438,258 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
     }
   } else {
     // ================================================= softmax + epilogue
-    const int hf = (warp - 2) / 4;              // column half of S, P, O and the output
+    // Slot A = warps 2..5 (even tiles), slot B = warps 6..9 (odd tiles); one
+    // query row per thread, warp w on TMEM lane quarter w % 4.
+    const int slot = (warp - 2) / 4;
     const int quarter = warp % 4;
-    const int r = quarter * 32 + lane;          // row within the pair (TMEM lane)
+    const int r = quarter * 32 + lane;            // row within the pair (TMEM lane)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    uint32_t ic = 0, sf[2] = {0, 0}, xc = 0;
-    long long pv_base = 0;                      // PVs completed before this item
+    const int half_bit = r >= 64 ? 2 : 1;         // the row's query block inside the pair
+    const float c2 = P.scale_log2;
+    constexpr int HC = D / 16;                    // 16-byte chunks in half a row of Q
+    uint32_t ic = 0, lc = 0, sf = 0;
+    long long pv_base = 0;                        // this slot's PVs completed before this item
     bool ok = true;
-    // One thread streams each item's G image into its buffer: the first now,
-    // each next one as soon as the linear term of the current item is done.
-    // Items whose sample dropped its linear branch are skipped.
-    const bool g_loader = HYB && warp == 2 && lane == 0;
-    long long g_issued = 0;
-    uint32_t lc = 0;   // items with a linear term so far
-    auto load_g = [&](long long from) {
-      for (long long w = from; w < total; w += gridDim.x) {
-        const Item nx = make_item(P, w);
-        if (!lin_on(P, nx.b)) continue;
-        mbar_arrive_expect_tx(g_full, C::kGImg);
-        bulk_load(smem_u32(gbuf), P.Gimg + static_cast<long long>(nx.bh) * D * D, C::kGImg,
-                  g_full);
-        ++g_issued;
-        return;
-      }
-    };
-    if (g_loader) load_g(blockIdx.x);
-    // Exchange of a per-row value with the other half's warp of this quarter.
-    auto exchange = [&](float mine) -> float {
-      float* slot = xrow + (xc & 1) * 256;
-      slot[hf * 128 + r] = mine;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(x_row(quarter));
-      const bool got = __all_sync(0xffffffffu, mbar_wait(x_row(quarter), xc & 1, wait_ns, abort_flag));
-      ++xc;
-      if (!got) {
-        ok = false;
-        return mine;
-      }
-      return slot[(1 - hf) * 128 + r];
-    };
     for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++ic) {
       const Item it = make_item(P, w);
       const int row_pos = it.p * 128 + r;        // position in the head's (possibly regrouped) order
       const bool row_valid = row_pos < P.N;
-      const int npair = (it.ntiles + 1) / 2;
+      const int T = (it.ntiles + 1) / 2;
+      const int nt = (T - slot + 1) / 2;          // this slot's tiles: t = slot, slot + 2, ...
       const bool lin = HYB && lin_on(P, it.b);   // this item adds the linear term
-      float den_row = 0.f;   // phi(q) . Z + eps of the row
-      if (hf == 1) {
-        // This warp's previous epilogue is complete: O, S and the linear
-        // term may be overwritten by this item's MMAs.
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_ready);
-        // Half 0 has written den for this item once q_ready completes; it
-        // writes the next one only after this item's last PV, which needs
-        // this warp's P, so the single slot is safe to read here.
-        if (!__all_sync(0xffffffffu, mbar_wait(q_ready, ic & 1, wait_ns, abort_flag))) {
+      const int qb = static_cast<int>(ic & 1);
+      // The item's Q rows have landed (observed every item, in order).
+      if (!__all_sync(0xffffffffu, mbar_wait(q_full(qb), (ic / 2) & 1, wait_ns, abort_flag))) {
+        ok = false;
+        break;
+      }
+      // Chunk c (8 columns) of this thread's row of the item's Q buffer.
+      unsigned char* qrow = qbuf + qb * C::kQBuf + r * 128;
+      auto q_chunk = [&](int c) -> uint4* {
+        return reinterpret_cast<uint4*>(qrow + (c / 8) * C::kRowSlab + ((c % 8) ^ (r % 8)) * 16);
+      };
+      // This slot's half of phi(q) . Z.
+      float den_part = 0.f;
+      if (lin) {
+        const float* zrow = P.Z + static_cast<long long>(it.bh) * D;
+#pragma unroll
+        for (int cc = 0; cc < HC; ++cc) {
+          const int c = slot * HC + cc;
+          const uint4 v = *q_chunk(c);
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 fz = unpack_bf16x2(relu_bf16x2(wv[e]));
+            den_part = fmaf(fz.x, __ldg(zrow + 8 * c + 2 * e), den_part);
+            den_part = fmaf(fz.y, __ldg(zrow + 8 * c + 2 * e + 1), den_part);
+          }
+        }
+      }
+
+      // ---- softmax over this slot's tiles (128 keys each)
+      float m = -INFINITY;   // running max of the row in the exp2 domain
+      float l = 0.f;         // row sum of exp2(S*c - m) over this slot's keys
+      int e0 = list_entry(it, 2 * slot, P.mode), e1 = list_entry(it, 2 * slot + 1, P.mode);
+      const uint32_t sbuf = lane_base + C::s_col(slot);
+      for (int k = 0; k < nt; ++k) {
+        const int t = slot + 2 * k;
+        // The next tile's list entries travel while this one is processed.
+        const int e0n = list_entry(it, 2 * t + 4, P.mode), e1n = list_entry(it, 2 * t + 5, P.mode);
+        // Waits and TMEM accesses are warp-collective: every decision that
+        // guards one is made uniform across the warp first.
+        if (!__all_sync(0xffffffffu, mbar_wait(s_full(slot), sf & 1, wait_ns, abort_flag))) {
           ok = false;
           break;
         }
-        if (lin) den_row = xden[r];
-      } else {
-        // ---- Q and phi(Q) into TMEM (A operands); den = phi(q) . Z + eps
-        const __nv_bfloat16* qsrc =
-            it.slot >= 0 ? P.qp + (static_cast<long long>(it.b) * P.Hs + it.slot) * P.N * D
-                         : P.q + static_cast<long long>(it.bh) * P.N * D;
-        const uint4* qrow = reinterpret_cast<const uint4*>(
-            qsrc + static_cast<long long>(row_valid ? row_pos : 0) * D);
-        const float* zrow = HYB ? P.Z + static_cast<long long>(it.bh) * D : nullptr;
-        float den = 0.f;
-        // Grid position of the row's token (its frame-major index) for the
-        // rotary encoding of the linear term.
-        const bool rope_on = lin && P.rope.on && row_valid;
+        ++sf;
+        tc_fence_after();
+        // The tile's two key blocks; inside each, the row's valid keys form
+        // one contiguous range [lo, hi] of the block's 64 columns.
+        const int jb[2] = {e0 & 0xFFFF, e1 & 0xFFFF};
+        const int mk[2] = {e0 >> 16, e1 >> 16};
+        int lo[2], hi[2];
+        bool live[2], any[2], part[2];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          lo[x] = 0;
+          hi[x] = min(63, P.N - 1 - jb[x] * 64);
+          if (P.mode == kModeBand) {
+            lo[x] = max(lo[x], row_pos - P.window - jb[x] * 64);
+            hi[x] = min(hi[x], row_pos + P.window - jb[x] * 64);
+          }
+          live[x] = row_valid && (mk[x] & half_bit) && lo[x] <= hi[x];
+          any[x] = __any_sync(0xffffffffu, live[x]);
+          part[x] = any[x] && __any_sync(0xffffffffu, !(live[x] && lo[x] == 0 && hi[x] == 63));
+        }
+        // Pass 1: the row max over both halves (keys outside the row's range
+        // count as -inf; only halves with a partial or dead row pay for it).
+        float pm = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (!any[x]) continue;
+          uint32_t s64[64];
+          tmem_ld64(sbuf + 64 * x, s64);
+          float sv[64];
+#pragma unroll
+          for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(s64[c]);
+          if (part[x]) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              sv[c] = (live[x] && c >= lo[x] && c <= hi[x]) ? sv[c] : -INFINITY;
+          }
+          pm = fmaxf(pm, max64(sv));
+        }
+        pm *= c2;                    // c2 > 0: max of scaled = scaled max
+        float f = 1.0f;              // factor O must be rescaled by before this PV
+        if (pm > m + 8.0f) {
+          f = (m == -INFINITY) ? 1.0f : ex2(m - pm);
+          l *= f;
+          m = pm;
+        }
+        // A row with no valid key so far keeps m = -inf: use 0 as the offset
+        // so its -inf scores give exp2(-inf) = 0, never NaN.
+        const float nm = (m == -INFINITY) ? 0.0f : -m;
+        // Pass 2: exponentiate each half; P (bf16 pairs) goes over the first
+        // 64 columns of S (half x -> columns 32x .. 32x+31, already read).
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          uint32_t pk[32];
+          if (any[x]) {
+            uint32_t s64[64];
+            tmem_ld64(sbuf + 64 * x, s64);
+            float sv[64];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(s64[c]);
+            if (part[x]) {
+#pragma unroll
+              for (int c = 0; c < 64; ++c)
+                sv[c] = (live[x] && c >= lo[x] && c <= hi[x]) ? sv[c] : -INFINITY;
+            }
+            float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+#pragma unroll
+            for (int c = 0; c < 64; c += 4) {
+              const float p0 = ex2(fmaf(sv[c], c2, nm)), p1 = ex2(fmaf(sv[c + 1], c2, nm));
+              const float p2 = ex2(fmaf(sv[c + 2], c2, nm)), p3 = ex2(fmaf(sv[c + 3], c2, nm));
+              pk[c / 2] = pack_bf16x2(p0, p1);
+              pk[c / 2 + 1] = pack_bf16x2(p2, p3);
+              ls0 += p0;
+              ls1 += p1;
+              ls2 += p2;
+              ls3 += p3;
+            }
+            l += (ls0 + ls1) + (ls2 + ls3);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pk[e] = 0u;
+          }
+          tmem_st32(sbuf + 32 * x, pk);
+        }
+        // Observe this slot's previous PV: every warp observes every PV of
+        // its slot in order, so each parity wait is at most one phase behind.
+        if (k >= 1) {
+          const long long g = pv_base + k - 1;
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait(o_done(slot), static_cast<uint32_t>(g & 1), wait_ns, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        if (__any_sync(0xffffffffu, f != 1.0f)) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o32[32];
+            tmem_ld32(lane_base + C::o_col(slot) + c0, o32);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o32[e] = __float_as_uint(__uint_as_float(o32[e]) * f);
+            tmem_st32(lane_base + C::o_col(slot) + c0, o32);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(slot));
+        e0 = e0n;
+        e1 = e1n;
+      }
+      if (!ok) break;
+      if (nt > 0) {
+        // This slot's last PV has landed.
+        const long long g = pv_base + nt - 1;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(o_done(slot), static_cast<uint32_t>(g & 1), wait_ns, abort_flag))) {
+          ok = false;
+          break;
+        }
+        pv_base += nt;
+      }
+      // ---- every QK of the item has run: phi(Q) (rotated with the 3-D
+      // rotary encoding when on) over the Q buffer, this slot's half.
+      if (!__all_sync(0xffffffffu, mbar_wait(q_free, ic & 1, wait_ns, abort_flag))) {
+        ok = false;
+        break;
+      }
+      if (lin) {
+        const bool rope_on = P.rope.on && row_valid;
         int rf = 0, ry = 0, rx = 0;
         if (rope_on) {
-          int tok = row_pos;
-          if (it.slot >= 0) {
-            const int fr = row_pos % P.F, pos = row_pos / P.F;
-            tok = fr * (P.Hh * P.Wh) + pos;
-          }
-          const int plane = P.rope.Hh * P.rope.Wh;   // token -> (frame, row, column)
+          int tok = row_pos;   // frame-major index of the row's token
+          if (it.slot >= 0) tok = (row_pos % P.F) * (P.Hh * P.Wh) + row_pos / P.F;
+          const int plane = P.rope.Hh * P.rope.Wh;
           rf = tok / plane;
           ry = (tok / P.rope.Wh) % P.rope.Hh;
           rx = tok % P.rope.Wh;
         }
 #pragma unroll
-        for (int c0 = 0; c0 < D / 2; c0 += 16) {
-          uint32_t pk[16];
+        for (int cc = 0; cc < HC; ++cc) {
+          const int c = slot * HC + cc;
+          uint4* pq = q_chunk(c);
+          const uint4 v = *pq;
+          uint32_t wv[4] = {relu_bf16x2(v.x), relu_bf16x2(v.y), relu_bf16x2(v.z), relu_bf16x2(v.w)};
+          if (rope_on) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 v = row_valid ? __ldg(qrow + c0 / 4 + u) : make_uint4(0, 0, 0, 0);
-            pk[4 * u + 0] = v.x; pk[4 * u + 1] = v.y; pk[4 * u + 2] = v.z; pk[4 * u + 3] = v.w;
-          }
-          tmem_st16(lane_base + C::kQ + c0, pk);
-          if (lin) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              pk[e] = relu_bf16x2(pk[e]);
-              const float2 f = unpack_bf16x2(pk[e]);
-              den = fmaf(f.x, __ldg(zrow + 2 * (c0 + e)), den);
-              den = fmaf(f.y, __ldg(zrow + 2 * (c0 + e) + 1), den);
+            for (int e = 0; e < 4; ++e) {
+              const float2 cs = rope_cs(P.rope, P.rope.theta, 4 * c + e, rf, ry, rx);
+              const float2 a = unpack_bf16x2(wv[e]);
+              wv[e] = pack_bf16x2(a.x * cs.x - a.y * cs.y, a.x * cs.y + a.y * cs.x);
             }
-            if (rope_on) {
-              // The numerator's phi(q) is rotated (word c0 + e is pair c0 + e);
-              // the denominator above is not.
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const float2 cs = rope_cs(P.rope, P.rope.theta, c0 + e, rf, ry, rx);
-                const float2 a = unpack_bf16x2(pk[e]);
-                pk[e] = pack_bf16x2(a.x * cs.x - a.y * cs.y, a.x * cs.y + a.y * cs.x);
-              }
-            }
-            tmem_st16(lane_base + C::kPQ + c0, pk);
           }
+          *pq = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
-        den_row = den + P.eps;
-        xden[r] = den_row;
-        tmem_st_wait();
-        tc_fence_before();
+        fence_proxy_async_smem();   // generic-proxy writes -> the MMA's operand reads
         __syncwarp();
-        if (lane == 0) mbar_arrive(q_ready);
+        if (lane == 0) mbar_arrive(phiq_ready);
       }
-
-      // ---- softmax over the item's S tiles (128 keys each)
-      const float c2 = P.scale_log2;
-      float m = -INFINITY;   // running max of the row in the exp2 domain (same in both halves)
-      float l = 0.f;         // this half's share of the row sum
-      const int half_bit = r >= 64 ? 2 : 1;
-      for (int u = 0; u < npair; ++u) {
-        const int b = u & 1;
-        const uint32_t sbuf = b ? C::kS1 : C::kS0;
-        // Waits and TMEM accesses are warp-collective: every decision that
-        // guards one is made uniform across the warp first.
-        if (!__all_sync(0xffffffffu, mbar_wait(s_full(b), sf[b] & 1, wait_ns, abort_flag))) {
-          ok = false;
-          break;
-        }
-        ++sf[b];
-        tc_fence_after();
-        const int t = 2 * u + hf;                  // this half's key block
-        int j = 0, mask = 0;
-        if (t < it.ntiles) tile_of(it, t, P.mode, j, mask);
-        // Valid key columns of the block form one contiguous range [lo, hi].
-        int lo = 0, hi = min(63, P.N - 1 - j * 64);
-        if (P.mode == kModeBand) {
-          lo = max(lo, row_pos - P.window - j * 64);
-          hi = min(hi, row_pos + P.window - j * 64);
-        }
-        const bool live = row_valid && (mask & half_bit) && lo <= hi;
-        const bool whole = live && lo == 0 && hi == 63;
-        const bool any_live = __any_sync(0xffffffffu, live);
-        float sv[64];
-        float pm = -INFINITY;
-        if (any_live) {
-          {
-            uint32_t s64[64];
-            tmem_ld64(lane_base + sbuf + hf * 64, s64);
-#pragma unroll
-            for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(s64[c]);
-          }
-          // Columns outside [lo, hi] (and every column of a dead row) become
-          // -inf; only blocks with a partial row in this warp pay for it.
-          if (__any_sync(0xffffffffu, !whole)) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) sv[c] = (live && c >= lo && c <= hi) ? sv[c] : -INFINITY;
-          }
-          // Row max by a tree of three-input maxima (64 -> 22 -> 8 -> 3 -> 1).
-          pm = max64(sv) * c2;   // c2 > 0: max of scaled = scaled max
-        }
-        // Both halves have loaded their S columns once the exchange completes,
-        // so P may now be written over S.
-        const float mx = fmaxf(pm, exchange(pm));
-        if (!ok) break;
-        float f = 1.0f;            // factor O must be rescaled by before this PV
-        if (mx > m + 8.0f) {
-          // Raise the running max.  O (earlier PVs) is rescaled below, once
-          // the previous PV has landed; l is rescaled here.
-          f = (m == -INFINITY) ? 1.0f : ex2(m - mx);
-          l *= f;
-          m = mx;
-        }
-        uint32_t pk[32];
-        if (any_live) {
-          // A row with no valid key so far keeps m = -inf: use 0 as the
-          // offset so its -inf scores give exp2(-inf) = 0, never NaN.
-          const float nm = (m == -INFINITY) ? 0.0f : -m;
-          float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float a0 = ex2(fmaf(sv[c], c2, nm));
-            const float a1 = ex2(fmaf(sv[c + 1], c2, nm));
-            const float b0 = ex2(fmaf(sv[c + 32], c2, nm));
-            const float b1 = ex2(fmaf(sv[c + 33], c2, nm));
-            pk[c / 2] = pack_bf16x2(a0, a1);
-            pk[16 + c / 2] = pack_bf16x2(b0, b1);
-            ls0 += a0 + a1;
-            ls1 += b0 + b1;
-          }
-          l += ls0 + ls1;
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = 0u;
-        }
-        tmem_st32(lane_base + sbuf + hf * 32, pk);
-        // Observe PV(u-1): every warp observes every PV completion in order,
-        // so each parity wait is at most one phase behind the barrier.
-        if (u >= 1) {
-          const long long g = pv_base + u - 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(o_done, static_cast<uint32_t>(g & 1), wait_ns, abort_flag))) {
-            ok = false;
-            break;
-          }
-        }
-        if (__any_sync(0xffffffffu, f != 1.0f)) {
-          tc_fence_after();
-#pragma unroll
-          for (int c0 = hf * (D / 2); c0 < (hf + 1) * (D / 2); c0 += 32) {
-            uint32_t o32[32];
-            tmem_ld32(lane_base + C::kO + c0, o32);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o32[e] = __float_as_uint(__uint_as_float(o32[e]) * f);
-            tmem_st32(lane_base + C::kO + c0, o32);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full(b));
+      // ---- merge the two slots' partial results for this row
+      xchg[slot * 128 + r] = make_float4(m, l, den_part, 0.f);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(x_bar);
+      if (!__all_sync(0xffffffffu, mbar_wait(x_bar, ic & 1, wait_ns, abort_flag))) {
+        ok = false;
+        break;
       }
-      if (!ok) break;
-      {
-        // The item's last PV has landed.
-        const long long g = pv_base + npair - 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(o_done, static_cast<uint32_t>(g & 1), wait_ns, abort_flag))) {
-          ok = false;
-          break;
-        }
-        pv_base += npair;
-      }
-      // ---- row sum over both halves
-      const float L = l + exchange(l);
-      if (!ok) break;
-      const float inv_l = 1.0f / L;
+      const float4 ot = xchg[(1 - slot) * 128 + r];
+      const float mA = slot ? ot.x : m, mB = slot ? m : ot.x;
+      const float lA = slot ? ot.y : l, lB = slot ? l : ot.y;
+      const float dA = slot ? ot.z : den_part, dB = slot ? den_part : ot.z;
+      const float M = fmaxf(mA, mB);
+      const float fA = (mA == -INFINITY) ? 0.0f : ex2(mA - M);
+      const float fB = (mB == -INFINITY) ? 0.0f : ex2(mB - M);
+      const float Lsum = lA * fA + lB * fB;
+      const float inv_l = Lsum > 0.f ? 1.0f / Lsum : 0.0f;
       float lin_scale = 0.f;
       if (lin) {
         const float gate = P.s != nullptr ? __ldg(P.s + it.b) : P.gate_override;
-        const float den = den_row;
-        lin_scale = den > 0.f ? gate / den : 0.f;
+        const float dd = (dA + dB) + P.eps;
+        lin_scale = dd > 0.f ? gate / dd : 0.f;
         if (!__all_sync(0xffffffffu, mbar_wait(lin_done, lc & 1, wait_ns, abort_flag))) {
           ok = false;
           break;
         }
         ++lc;
-        // The linear term has read G: the next item's image may replace it.
-        if (g_loader) load_g(w + gridDim.x);
       }
       tc_fence_after();
-      // ---- epilogue: this warp writes columns [hf*D/2, (hf+1)*D/2) of the row
+      // ---- epilogue: this slot writes columns [slot*D/2, (slot+1)*D/2) of the row
       long long out_row = row_pos;
       if (it.slot >= 0 && row_valid) {
         const int fr = row_pos % P.F, pos = row_pos / P.F;
@@ -672,40 +697,49 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         out_row = (static_cast<long long>(fr) * P.Hh + y) * P.Wh + x;
       }
       uint4* orow = reinterpret_cast<uint4*>(
-          P.o + (static_cast<long long>(it.bh) * P.N + (row_valid ? out_row : 0)) * D);
+          P.o + (static_cast<long long>(it.bh) * P.N + (row_valid ? out_row : 0)) * D + slot * (D / 2));
+      const bool has_b = T > 1;                 // slot B ran at least one tile
 #pragma unroll
-      for (int c0 = hf * (D / 2); c0 < (hf + 1) * (D / 2); c0 += 32) {
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {
+        const uint32_t col = slot * (D / 2) + c0;
         uint32_t o32[32];
-        tmem_ld32(lane_base + C::kO + c0, o32);
         float v[32];
+        tmem_ld32(lane_base + C::o_col(0) + col, o32);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o32[e]) * inv_l;
+        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o32[e]) * fA;
+        if (has_b) {
+          tmem_ld32(lane_base + C::o_col(1) + col, o32);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = fmaf(__uint_as_float(o32[e]), fB, v[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] *= inv_l;
         if (lin) {
-          uint32_t l32[32];
-          tmem_ld32(lane_base + C::kL + c0, l32);
+          tmem_ld32(lane_base + C::kL + col, o32);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = fmaf(__uint_as_float(l32[e]), lin_scale, v[e]);
+          for (int e = 0; e < 32; ++e) v[e] = fmaf(__uint_as_float(o32[e]), lin_scale, v[e]);
         }
         if (row_valid) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u4 = 0; u4 < 4; ++u4) {
             uint4 wv;
-            wv.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
-            wv.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
-            wv.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
-            wv.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
-            orow[c0 / 8 + u] = wv;
+            wv.x = pack_bf16x2(v[8 * u4 + 0], v[8 * u4 + 1]);
+            wv.y = pack_bf16x2(v[8 * u4 + 2], v[8 * u4 + 3]);
+            wv.z = pack_bf16x2(v[8 * u4 + 4], v[8 * u4 + 5]);
+            wv.w = pack_bf16x2(v[8 * u4 + 6], v[8 * u4 + 7]);
+            orow[c0 / 8 + u4] = wv;
           }
         }
       }
+      // This warp is done with O, S and the linear term of the item.
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_done);
     }
     if (!ok) raise_timeout(P.err, abort_flag);
-    // Drain the last G load before the CTA leaves (it has landed already
-    // unless a wait above ran out).
-    if (g_loader && g_issued > 0 &&
-        !mbar_wait(g_full, static_cast<uint32_t>((g_issued - 1) & 1), wait_ns, nullptr))
-      atomicOr(P.err, kErrTimeout);
+    // No TMEM access of this warp may be in flight at the teardown.
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    tmem_st_wait();
   }
   tc_fence_before();
   __syncthreads();
@@ -728,15 +762,18 @@ __global__ void debug_wait_kernel(unsigned* err, unsigned long long wait_ns) {
 template <int D, bool HYB>
 cudaError_t launch_attn_t(const Ctx& c, const AttnArgs& a, const Params& P) {
   using C = AT<D, HYB>;
-  CUtensorMap mk, mv, mkp, mvp;
+  CUtensorMap mq, mk, mv, mqp, mkp, mvp;
   const int BH = a.B * a.H;
-  if (!make_tmap_bf16_3d(&mk, a.k, BH, a.N, D) || !make_tmap_bf16_3d(&mv, a.v, BH, a.N, D))
+  if (!make_tmap_bf16_3d(&mq, a.q, BH, a.N, D) || !make_tmap_bf16_3d(&mk, a.k, BH, a.N, D) ||
+      !make_tmap_bf16_3d(&mv, a.v, BH, a.N, D))
     return cudaErrorInvalidValue;
   if (a.Hs > 0) {
-    if (!make_tmap_bf16_3d(&mkp, a.kp, a.B * a.Hs, a.N, D) ||
+    if (!make_tmap_bf16_3d(&mqp, a.qp, a.B * a.Hs, a.N, D) ||
+        !make_tmap_bf16_3d(&mkp, a.kp, a.B * a.Hs, a.N, D) ||
         !make_tmap_bf16_3d(&mvp, a.vp, a.B * a.Hs, a.N, D))
       return cudaErrorInvalidValue;
   } else {
+    mqp = mq;
     mkp = mk;
     mvp = mv;
   }
@@ -746,7 +783,8 @@ cudaError_t launch_attn_t(const Ctx& c, const AttnArgs& a, const Params& P) {
   const long long items = static_cast<long long>(BH) * P.npairs;
   long long grid = items < c.num_sms ? items : c.num_sms;
   if (grid < 1) grid = 1;
-  attn_kernel<D, HYB><<<static_cast<int>(grid), 320, C::kSmem, c.stream>>>(mk, mv, mkp, mvp, P);
+  attn_kernel<D, HYB><<<static_cast<int>(grid), 320, C::kSmem, c.stream>>>(mq, mk, mv, mqp, mkp,
+                                                                             mvp, P);
   return cudaGetLastError();
 }
 

@@ -87,7 +87,7 @@ def load_peaks() -> tuple:
 
 def attn_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("attn.cu", "common.cuh"):
+    for f in ("attn.cu", "common.cuh", "internal.h"):
         with open(os.path.join(ROOT, "sparse_linear_hybrid_top_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

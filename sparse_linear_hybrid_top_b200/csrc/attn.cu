@@ -351,34 +351,45 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
   } else if (warp == 1) {
     if (lane == 0) {
       // ================================================= MMA issuer
+      // Descriptors are built once per operand and advanced by constant
+      // offsets per K-step (shared addresses stay below 2^18, so the 14-bit
+      // address field never carries); the ring position is kept as a stage
+      // index and a phase bit.  This thread shares its sub-partition with two
+      // softmax warps, so every instruction it saves is issue time the tensor
+      // pipe does not wait for.
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
       constexpr uint32_t idesc_lin = idesc_bf16(128, D, false, false);
-      long long sc = 0;   // ring stages consumed so far
+      const uint32_t ring_base = smem_u32(ring);
+      int stage = 0;
+      uint32_t sphase = 0;
       uint32_t ic = 0, lc = 0, pf[2] = {0, 0};
       bool ok = true;
-      auto wait_stage = [&]() -> bool {
-        return mbar_wait(full(static_cast<int>(sc % NS)), static_cast<uint32_t>((sc / NS) & 1),
-                         wait_ns, abort_flag);
+      auto wait_stage = [&]() -> bool { return mbar_wait(full(stage), sphase, wait_ns, abort_flag); };
+      auto next_stage = [&]() {
+        if (++stage == NS) {
+          stage = 0;
+          sphase ^= 1u;
+        }
       };
       // S_slot = Q K(t)^T from the K tile in the current stage.
-      auto issue_qk = [&](int qb, int slot) {
-        const uint32_t ka = st_addr(sc), qa = q_addr(qb);
+      auto issue_qk = [&](uint64_t qdesc, int slot) {
+        const uint64_t kdesc = sdesc_sw128(ring_base + stage * C::kStage, 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          mma_ss(tmem + C::s_col(slot),
-                 sdesc_sw128(qa + (ks / 4) * C::kRowSlab + (ks % 4) * 32, 16, 1024),
-                 sdesc_sw128(ka + (ks / 4) * C::kRowSlab + (ks % 4) * 32, 16, 1024), idesc_qk,
-                 ks > 0 ? 1u : 0u);
-        mma_commit(empty(static_cast<int>(sc % NS)));
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t off = static_cast<uint64_t>(((ks / 4) * C::kRowSlab + (ks % 4) * 32) >> 4);
+          mma_ss(tmem + C::s_col(slot), qdesc + off, kdesc + off, idesc_qk, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(empty(stage));
         mma_commit(s_full(slot));
-        ++sc;
+        next_stage();
       };
       for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++ic) {
         const Item it = make_item(P, w);
         const int T = (it.ntiles + 1) / 2;
         const bool lin = HYB && lin_on(P, it.b);
         const int qb = static_cast<int>(ic & 1);
+        const uint64_t qdesc = sdesc_sw128(q_addr(qb), 16, 1024);
         // The previous item's epilogue has read O, S and the linear term.
         if (ic > 0 && !mbar_wait(epi_done, (ic - 1) & 1, wait_ns, abort_flag)) { ok = false; break; }
         if (!mbar_wait(q_full(qb), (ic / 2) & 1, wait_ns, abort_flag)) { ok = false; break; }
@@ -386,7 +397,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         for (int t = 0; t < 2 && t < T; ++t) {
           if (!wait_stage()) { ok = false; break; }
           tc_fence_after();
-          issue_qk(qb, t);
+          issue_qk(qdesc, t);
         }
         if (!ok) break;
         if (T <= 2) mma_commit(q_free);   // every QK of the item is issued
@@ -396,19 +407,29 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
           ++pf[slot];
           if (!wait_stage()) { ok = false; break; }
           tc_fence_after();
-          const uint32_t va = st_addr(sc);
-          const int nks = (2 * t + 1 < it.ntiles) ? 8 : 4;   // K-steps: 16 keys each
-          for (int ks = 0; ks < nks; ++ks)
-            mma_ts(tmem + C::o_col(slot), tmem + C::s_col(slot) + ks * 8,
-                   sdesc_sw128(va + (ks / 4) * (D / 64) * kSlab + (ks % 4) * 2048, kSlab, 1024),
-                   idesc_pv, (t >= 2 || ks > 0) ? 1u : 0u);
-          mma_commit(empty(static_cast<int>(sc % NS)));
+          const uint64_t vdesc = sdesc_sw128(ring_base + stage * C::kStage, kSlab, 1024);
+          const uint32_t sa = tmem + C::s_col(slot), oa = tmem + C::o_col(slot);
+          const uint32_t acc0 = t >= 2 ? 1u : 0u;
+          if (2 * t + 1 < it.ntiles) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {   // K-steps: 16 keys each
+              const uint64_t off = static_cast<uint64_t>(((ks / 4) * (D / 64) * kSlab + (ks % 4) * 2048) >> 4);
+              mma_ts(oa, sa + ks * 8, vdesc + off, idesc_pv, ks > 0 ? 1u : acc0);
+            }
+          } else {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {   // a single 64-key block
+              const uint64_t off = static_cast<uint64_t>(((ks % 4) * 2048) >> 4);
+              mma_ts(oa, sa + ks * 8, vdesc + off, idesc_pv, ks > 0 ? 1u : acc0);
+            }
+          }
+          mma_commit(empty(stage));
           mma_commit(o_done(slot));
-          ++sc;
+          next_stage();
           if (t + 2 < T) {
             if (!wait_stage()) { ok = false; break; }
             tc_fence_after();
-            issue_qk(qb, slot);   // same S buffer: runs after this PV in issue order
+            issue_qk(qdesc, slot);   // same S buffer: runs after this PV in issue order
             if (t + 3 == T) mma_commit(q_free);   // that was the item's last QK
           }
         }
@@ -419,15 +440,16 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
           if (!mbar_wait(phiq_ready, lc & 1, wait_ns, abort_flag)) { ok = false; break; }
           if (!wait_stage()) { ok = false; break; }
           tc_fence_after();
-          const uint32_t ga = st_addr(sc), qa = q_addr(qb);
+          const uint64_t gdesc = sdesc_sw128(ring_base + stage * C::kStage, 16, 1024);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_ss(tmem + C::kL, sdesc_sw128(qa + (ks / 4) * C::kRowSlab + (ks % 4) * 32, 16, 1024),
-                   sdesc_sw128(ga + (ks / 4) * (D * 128) + (ks % 4) * 32, 16, 1024), idesc_lin,
-                   ks > 0 ? 1u : 0u);
-          mma_commit(empty(static_cast<int>(sc % NS)));
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t qoff = static_cast<uint64_t>(((ks / 4) * C::kRowSlab + (ks % 4) * 32) >> 4);
+            const uint64_t goff = static_cast<uint64_t>(((ks / 4) * (D * 128) + (ks % 4) * 32) >> 4);
+            mma_ss(tmem + C::kL, qdesc + qoff, gdesc + goff, idesc_lin, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(empty(stage));
           mma_commit(lin_done);
-          ++sc;
+          next_stage();
           ++lc;
         }
         mma_commit(q_empty(qb));   // the item's Q buffer is free once these MMAs ran

@@ -46,7 +46,8 @@ __all__ = [
     "topk_attention_rows", "topk_attention", "space_major_order",
     "swa_attention_rows", "swa_attention", "dense_attention",
     "rope3d_split", "rope3d_angles", "rope3d_rotate",
-    "linear_state", "linear_apply", "combine", "forward",
+    "linear_state", "linear_apply", "combine", "combine_full", "output_projection",
+    "forward",
     "near_tie_equivalent",
 ]
 
@@ -298,13 +299,40 @@ def combine(o_sparse, o_lin, w_lin_h, s: float) -> np.ndarray:
     return as64(o_sparse) + float(s) * (as64(o_lin) @ as64(w_lin_h))
 
 
+def combine_full(o_sparse, o_lin, w_full, s: float) -> np.ndarray:
+    """O = O_s + s * (O_l W_full) with the projection over all heads.
+
+    Reading of the zero-init projection as one full-width linear layer (its
+    share of the parameters in "SALAD ... (paper.rainbus.top)" suggests a
+    full-width layer; 方法步骤详情 step 4): the heads' linear outputs of a token
+    are concatenated (head-major: column h*d + c), multiplied by w_full
+    [H*d, H*d] as a row vector, and split back into heads.  o_sparse, o_lin:
+    [H, N, d] of one sample.
+    """
+    o_sparse, o_lin, w_full = as64(o_sparse), as64(o_lin), as64(w_full)
+    H, N, d = o_lin.shape
+    cat = o_lin.transpose(1, 0, 2).reshape(N, H * d)
+    mixed = (cat @ w_full).reshape(N, H, d).transpose(1, 0, 2)
+    return o_sparse + float(s) * mixed
+
+
+def output_projection(o, w_out) -> np.ndarray:
+    """The final projection of 方法步骤详情 step 7: the heads of a token
+    concatenated (column h*d + c) times w_out [H*d, D_out].  o: [H, N, d] of
+    one sample -> [N, D_out]."""
+    o = as64(o)
+    H, N, d = o.shape
+    return o.transpose(1, 0, 2).reshape(N, H * d) @ as64(w_out)
+
+
 # ------------------------------------------------------------ forward -----
 def forward(inp: Dict, *, mode: str, block: int = 64, topk: int = 0, window: int = 0,
             space_major_heads: Sequence[int] = (), F: int = 0, Hh: int = 0, Wh: int = 0,
             eps: float = 1e-6, gate_override: Optional[float] = None,
             idx_override: Optional[np.ndarray] = None,
             drop_threshold: float = 0.0, rope3d: bool = False,
-            rope_base: float = 10000.0) -> Dict[str, np.ndarray]:
+            rope_base: float = 10000.0, w_lin_full=None,
+            w_out=None) -> Dict[str, np.ndarray]:
     """The whole hybrid layer, in the step order of the method.
 
     inp: q, k, v [B, H, N, d]; x [B, N, D]; w_gate [D]; bias; w_lin [H, d, d].
@@ -317,7 +345,10 @@ def forward(inp: Dict, *, mode: str, block: int = 64, topk: int = 0, window: int
     Returns s [B], idx [B, H, nb, topk] (topk mode), scores, o_sparse, o_lin,
     o and dropped [B].  ``rope3d``: the linear branch integrates the 3-D
     rotary encoding over the (F, Hh, Wh) grid of the tokens (see
-    ``linear_state``).
+    ``linear_state``).  ``w_lin_full`` [H*d, H*d]: the projection of the
+    linear branch mixes the heads (``combine_full``) instead of the per-head
+    ``w_lin``.  ``w_out`` [H*d, D_out]: also return ``out`` [B, N, D_out],
+    the output projection of the combined heads (step 7).
     """
     q, k, v = as64(inp["q"]), as64(inp["k"]), as64(inp["v"])
     B, H, N, d = q.shape
@@ -349,10 +380,15 @@ def forward(inp: Dict, *, mode: str, block: int = 64, topk: int = 0, window: int
             o_lin[b, h] = linear_apply(q[b, h], Hst, Z, eps, angles)
             if s[b] < drop_threshold:
                 o[b, h] = o_sparse[b, h]
-            else:
+            elif w_lin_full is None:
                 o[b, h] = combine(o_sparse[b, h], o_lin[b, h], w_lin[h], s[b])
+        if w_lin_full is not None and not s[b] < drop_threshold:
+            o[b] = combine_full(o_sparse[b], o_lin[b], w_lin_full, s[b])
+    out = None
+    if w_out is not None:
+        out = np.stack([output_projection(o[b], w_out) for b in range(B)])
     return {"s": s, "idx": idx, "scores": scores, "o_sparse": o_sparse,
-            "o_lin": o_lin, "o": o, "dropped": s < drop_threshold}
+            "o_lin": o_lin, "o": o, "dropped": s < drop_threshold, "out": out}
 
 
 # ------------------------------------------------- selection comparison ---

@@ -364,6 +364,41 @@ def test_forward_branch_dropping_per_sample_threshold():
     assert not at["dropped"][lo]
 
 
+def test_full_width_projection_reduces_and_orients():
+    inp = _tiny_inputs(seed=97)
+    H, d = 2, 16
+    per_head = oracle.forward(inp, mode="topk", block=64, topk=2)
+    # A block-diagonal full-width matrix is the per-head projection.
+    W = np.zeros((H * d, H * d))
+    for h in range(H):
+        W[h * d:(h + 1) * d, h * d:(h + 1) * d] = inp["w_lin"][h]
+    full = oracle.forward(inp, mode="topk", block=64, topk=2, w_lin_full=W)
+    np.testing.assert_allclose(full["o"], per_head["o"], rtol=1e-12, atol=1e-13)
+    # Identity: O_s + s * O_l.
+    ident = oracle.forward(inp, mode="topk", block=64, topk=2, w_lin_full=np.eye(H * d))
+    np.testing.assert_allclose(ident["o"], ident["o_sparse"] + ident["s"][0] * ident["o_lin"],
+                               rtol=1e-12, atol=1e-13)
+    # One entry W[h1*d + c1, h2*d + c2] = 1 moves column c1 of head h1's O_l
+    # into column c2 of head h2, and nothing else.
+    W = np.zeros((H * d, H * d)); W[0 * d + 3, 1 * d + 5] = 1.0
+    one = oracle.forward(inp, mode="topk", block=64, topk=2, w_lin_full=W)
+    diff = one["o"] - one["o_sparse"]
+    np.testing.assert_allclose(diff[0, 1, :, 5], one["s"][0] * one["o_lin"][0, 0, :, 3], rtol=1e-12)
+    diff[0, 1, :, 5] = 0.0
+    np.testing.assert_array_equal(diff, 0.0)
+
+
+def test_output_projection_orients():
+    inp = _tiny_inputs(seed=98)
+    H, d, N = 2, 16, 192
+    r = oracle.forward(inp, mode="topk", block=64, topk=2, w_out=np.eye(H * d))
+    np.testing.assert_array_equal(r["out"][0], r["o"][0].transpose(1, 0, 2).reshape(N, H * d))
+    Wo = np.zeros((H * d, 7)); Wo[1 * d + 2, 4] = 1.0
+    r = oracle.forward(inp, mode="topk", block=64, topk=2, w_out=Wo)
+    np.testing.assert_array_equal(r["out"][0][:, 4], r["o"][0, 1, :, 2])
+    assert not np.any(np.delete(r["out"][0], 4, axis=1))
+
+
 def test_forward_linear_in_gate_and_projection():
     inp = _tiny_inputs(seed=91)
     r1 = oracle.forward(inp, mode="topk", block=64, topk=2, gate_override=0.25)

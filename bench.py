@@ -271,7 +271,7 @@ def run_ours(args, w) -> int:
     device = torch.device("cuda", local)
     init_dist("nccl", world)
     import sparse_linear_hybrid_top_b200 as salad
-    from synth import generate
+    from synth import generate, generate_projections
 
     host = generate(w)
     dev = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
@@ -360,6 +360,32 @@ def run_ours(args, w) -> int:
             dev["q"], dev["k"], dev["v"], dev["x"], dev["w_gate"], dev["w_lin"], mode=w.mode,
             topk=w.topk, bias=w.bias, eps=w.eps, drop_threshold=1.0, **extra), nv),
     }
+    # Full-width projections: the linear branch's W_lin over all heads
+    # (H*d x H*d) and the output projection W_out (H*d x H*d), two tcgen05
+    # GEMMs after the attention.  The GEMM alone is timed too, against the
+    # burst bf16 peak (it runs by itself here).
+    proj = {n: t.to(device) for n, t in generate_projections(w).items()}
+    variants["full_width_proj"] = time_plan(salad.ForwardPlan(
+        dev["q"], dev["k"], dev["v"], dev["x"], dev["w_gate"], None, mode=w.mode,
+        topk=w.topk, bias=w.bias, eps=w.eps, w_lin_full=proj["w_lin_full"],
+        w_out=proj["w_out"], **extra), nv)
+    K = w.H * w.d
+    g_out = torch.empty_like(dev["q"])
+    g_s = torch.full((w.B,), 0.5, dtype=torch.float32, device=device)
+    for _ in range(3):
+        salad.project(dev["q"], proj["w_lin_full"], out_per_head=True, resid=dev["v"], s=g_s,
+                      out=g_out, stream=stream)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(nv):
+        salad.project(dev["q"], proj["w_lin_full"], out_per_head=True, resid=dev["v"], s=g_s,
+                      out=g_out, stream=stream)
+    g1.record(stream)
+    torch.cuda.synchronize(device)
+    salad.check_error(stream)
+    gemm_ms = g0.elapsed_time(g1) / nv
+    gemm_flops = 2.0 * w.B * w.N * K * K
+    del g_out
 
     # End to end through the public API: pinned host inputs -> device ->
     # salad_forward -> result back to the host, every step.
@@ -406,6 +432,11 @@ def run_ours(args, w) -> int:
         "phases_ms": {k: round(v, 5) for k, v in phases.items()},
         "dense_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / agg["ms_per_step"], 3),
         "variants_ms_per_layer": {k: round(v, 5) for k, v in variants.items()},
+        "proj_gemm": {"kernel": "proj_kernel<256>", "shape": [w.B * w.N, K, K],
+                      "ms": round(gemm_ms, 5),
+                      "tflops": round(gemm_flops / (gemm_ms * 1e-3) / 1e12, 2),
+                      "frac": round(gemm_flops / (gemm_ms * 1e-3) / 1e12 / float(peaks["bf16_tflops"]), 4),
+                      "peak_source": f"bf16 burst, {peaks_src}"},
         "flops_per_step": fl["total"],
         "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,hybrid>",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",

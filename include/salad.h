@@ -173,6 +173,28 @@ salad_status salad_dense_attn(const void* q, const void* k, const void* v,
                               int B, int H, int N, int d, void* o, salad_stream stream);
 
 /*
+ * Full-width projection of concatenated heads with a gated residual
+ * (paper.rainbus.top 方法步骤详情 step 4, the linear branch's projection read
+ * as one layer over all heads, and step 7, the output projection):
+ *   out[b,n,:] = resid[b,n,:] + s_b * (A_cat[b,n,:] W)
+ * A: bf16 [B,H,N,d] device; A_cat[b,n, h*d + c] = A[b,h,n,c] (the heads of a
+ * token concatenated, head-major; no copy is made).  W: bf16 row-major
+ * [H*d, n_out] device, n_out a positive multiple of 64.
+ * out_per_head = 1: out (and resid) are bf16 [B,H,N,d] (n_out must equal
+ *   H*d; column h*d + c of a token is out[b,h,n,c]).
+ * out_per_head = 0: out (and resid) are bf16 [B,N,n_out], token-major.
+ * resid: device, same layout as out, or NULL (no residual).  It may be the
+ *   same pointer as out (in place); otherwise it must not overlap out.
+ * s: device float32 [B] or NULL (s_b = 1).  Samples with s_b < drop_threshold
+ *   are skipped: their out is not written (0 or NaN never skips).
+ * out must not overlap A or W.  Needs no workspace.  tcgen05 GEMM with fp32
+ * accumulation; the result is rounded once to bf16.
+ */
+salad_status salad_project(const void* a, int B, int H, int N, int d, const void* w, int n_out,
+                           void* out, int out_per_head, const void* resid, const float* s,
+                           float drop_threshold, salad_stream stream);
+
+/*
  * The whole hybrid layer (paper.rainbus.top 方法步骤详情 steps 2-6, 8):
  * gate, sparse branch, linear branch, per-head projection W_lin (d x d,
  * right-multiplying row vectors: O_l' = O_l W_lin[h]), gated residual sum.
@@ -219,6 +241,19 @@ typedef struct salad_forward_args {
      * and Z = sum_j phi(k_j). */
     int rope3d;
     float rope_base;            /* > 1, usually 10000 */
+    /* Full-width projection of the linear branch (paper.rainbus.top 方法步骤详情
+     * step 4 read as one layer over all heads): bf16 [H*d, H*d] device, or
+     * NULL for the per-head w_lin.  When set, w_lin is not read and
+     *   O[b,:,n,:] = O_sparse + s_b * split_heads(cat_heads(O_l[b,:,n,:]) w_lin_full)
+     * with cat_heads putting column h*d + c = O_l[b,h,n,c] (see
+     * salad_project).  Not combined with rope3d (SALAD_ERR_UNSUPPORTED). */
+    const void* w_lin_full;
+    /* Output projection (step 7): bf16 [H*d, d_out] device, or NULL.  When
+     * set, out[b,n,:] = cat_heads(O[b,:,n,:]) w_out is written too; o still
+     * receives O. */
+    const void* w_out;
+    int d_out;                  /* multiple of 64 when w_out is set */
+    void* out;                  /* bf16 [B,N,d_out] device (out) when w_out is set */
     float* s_out;               /* optional device float32 [B] (out), may be NULL */
     int32_t* idx_out;           /* optional device int32 [B,H,nb,topk] (out), may be NULL */
     void* workspace;            /* device scratch, >= salad_forward_workspace_bytes() */
@@ -226,7 +261,8 @@ typedef struct salad_forward_args {
     /* Optional profiling hook: NULL, or a HOST array of 5 cudaEvent_t,
      * recorded at the start (on `stream`), when the gate ends, when the
      * sparse-pattern step (selection or regrouping) ends, when the attention
-     * kernel starts (every input ready), and when it ends.  The gate and the
+     * kernel starts (every input ready), and when it ends (the full-width
+     * projections, if any, follow that last event).  The gate and the
      * linear branch run on two library-owned streams forked from `stream`
      * and joined back before the attention, so only the last two events
      * bound one kernel. */

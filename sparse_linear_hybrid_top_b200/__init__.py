@@ -17,6 +17,7 @@ import torch
 __all__ = [
     "SaladError", "lib", "status_string", "version",
     "gate", "gate_noalloc", "select_blocks", "linear_state", "linear_apply", "permute_tokens",
+    "project",
     "sparse_attn", "dense_attn", "forward", "ForwardPlan", "forward_workspace_bytes",
     "check_error", "debug_wait_timeout",
     "MODE_TOPK", "MODE_SWA", "MODE_DENSE", "EXPORTED_SYMBOLS",
@@ -38,7 +39,7 @@ EXPORTED_SYMBOLS = (
     "salad_sparse_attn_workspace_bytes", "salad_sparse_attn", "salad_dense_attn",
     "salad_forward_workspace_bytes", "salad_forward",
     "salad_check_error", "salad_debug_wait_timeout",
-    "salad_gate_noalloc",
+    "salad_gate_noalloc", "salad_project",
 )
 
 
@@ -63,6 +64,8 @@ class ForwardArgs(ctypes.Structure):
         ("eps", ctypes.c_float), ("gate_override", ctypes.c_float),
         ("drop_threshold", ctypes.c_float),
         ("rope3d", ctypes.c_int), ("rope_base", ctypes.c_float),
+        ("w_lin_full", ctypes.c_void_p), ("w_out", ctypes.c_void_p), ("d_out", ctypes.c_int),
+        ("out", ctypes.c_void_p),
         ("s_out", ctypes.c_void_p), ("idx_out", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("phase_events", ctypes.c_void_p),
@@ -90,6 +93,7 @@ def _load() -> ctypes.CDLL:
         "salad_sparse_attn": (i, [vp, vp, vp, i, i, i, i, i, i, i, vp, i, vp, i, i, i, vp, vp,
                                   sz, vp]),
         "salad_dense_attn": (i, [vp, vp, vp, i, i, i, i, vp, vp]),
+        "salad_project": (i, [vp, i, i, i, i, vp, i, vp, i, vp, vp, f, vp]),
         "salad_forward_workspace_bytes": (sz, [ctypes.POINTER(ForwardArgs)]),
         "salad_forward": (i, [ctypes.POINTER(ForwardArgs), vp]),
         "salad_check_error": (i, [vp]),
@@ -240,6 +244,32 @@ def linear_apply(q: torch.Tensor, Hst: torch.Tensor, Z: torch.Tensor, eps: float
     return o
 
 
+def project(a: torch.Tensor, w: torch.Tensor, *, out_per_head: bool = False, resid=None,
+            s=None, drop_threshold: float = 0.0, out=None, stream=None) -> torch.Tensor:
+    """resid + s_b * (cat_heads(a) @ w): a bf16 [B,H,N,d], w bf16 [H*d, n_out].
+
+    out_per_head: out is [B,H,N,d] (n_out == H*d), else [B,N,n_out].  resid
+    (same layout as out, may be ``out`` itself) and s (float32 [B]) are
+    optional; samples with s_b < drop_threshold are left unwritten.
+    """
+    _dev_tensor(a, torch.bfloat16, "a")
+    _dev_tensor(w, torch.bfloat16, "w")
+    B, H, N, d = a.shape
+    n_out = w.shape[-1]
+    if out is None:
+        out = torch.empty((B, H, N, d) if out_per_head else (B, N, n_out), dtype=torch.bfloat16,
+                          device=a.device)
+    _dev_tensor(out, torch.bfloat16, "out")
+    if resid is not None:
+        _dev_tensor(resid, torch.bfloat16, "resid")
+    if s is not None:
+        _dev_tensor(s, torch.float32, "s")
+    _check(lib.salad_project(_ptr(a), B, H, N, d, _ptr(w), n_out, _ptr(out), int(bool(out_per_head)),
+                             _ptr(resid), _ptr(s), float(drop_threshold), _stream(stream)),
+           "salad_project")
+    return out
+
+
 def permute_tokens(src: torch.Tensor, F: int, Hh: int, Wh: int, *, inverse: bool = False,
                    dst=None, stream=None) -> torch.Tensor:
     """Frame-major <-> space-major row order of [..., N, d] slabs."""
@@ -294,12 +324,20 @@ class ForwardPlan:
                  F: int = 0, Hh: int = 0, Wh: int = 0, bias: float = 0.0, eps: float = 1e-6,
                  gate_override: Optional[float] = None, drop_threshold: float = 0.0,
                  rope3d: bool = False, rope_base: float = 10000.0, o=None,
-                 s_out=None, idx_out=None, block: int = 64):
+                 s_out=None, idx_out=None, block: int = 64, w_lin_full=None, w_out=None,
+                 out=None):
         for n, t in (("q", q), ("k", k), ("v", v), ("x", x), ("w_gate", w_gate),
-                     ("w_lin", w_lin)):
-            _dev_tensor(t, torch.bfloat16, n)
+                     ("w_lin", w_lin), ("w_lin_full", w_lin_full), ("w_out", w_out)):
+            if t is not None or n in ("q", "k", "v", "x", "w_gate"):
+                _dev_tensor(t, torch.bfloat16, n)
         B, H, N, d = q.shape
-        self.tensors = dict(q=q, k=k, v=v, x=x, w_gate=w_gate, w_lin=w_lin)
+        self.tensors = dict(q=q, k=k, v=v, x=x, w_gate=w_gate, w_lin=w_lin,
+                            w_lin_full=w_lin_full, w_out=w_out)
+        # Output projection (optional): out [B,N,d_out] = cat_heads(O) w_out.
+        self.out = None
+        if w_out is not None:
+            self.out = torch.empty((B, N, w_out.shape[-1]), dtype=torch.bfloat16,
+                                   device=q.device) if out is None else out
         self.o = torch.empty_like(q) if o is None else o
         self.s_out, self.idx_out = s_out, idx_out
         self._flags, fptr = _flags(space_major_heads, H)
@@ -319,6 +357,11 @@ class ForwardPlan:
         # 3-D rotary encoding of the linear branch over the F x Hh x Wh grid.
         a.rope3d = 1 if rope3d else 0
         a.rope_base = float(rope_base)
+        # Full-width projection of the linear branch instead of the per-head w_lin.
+        a.w_lin_full = _ptr(w_lin_full)
+        a.w_out = _ptr(w_out)
+        a.d_out = 0 if w_out is None else int(w_out.shape[-1])
+        a.out = _ptr(self.out)
         a.s_out = _ptr(s_out)
         a.idx_out = _ptr(idx_out)
         need = lib.salad_forward_workspace_bytes(ctypes.byref(a))

@@ -156,9 +156,40 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, int S, int N, int d) 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [B][H][N][d] bf16 viewed as 4-D (d, N, H, B), box 64 x 128 x 1 x 1, 128-byte
+// swizzle: one box is 128 token rows of 64 channels of one head.
+bool make_tmap_bf16_heads4d(CUtensorMap* map, const void* base, int B, int H, int N, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * d * 2,
+                                 static_cast<cuuint64_t>(H) * N * d * 2};
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row-major [rows][cols] bf16 viewed as 2-D (cols, rows), box 64 x 64, 128-byte
+// swizzle.
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, int rows, int cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------- forward layout --
 struct FwdLayout {
-  size_t gate, s, sel, idx, lists, counts, lin, hst, z, g, qp, kp, vp, total;
+  size_t gate, s, sel, idx, lists, counts, lin, hst, z, g, olin, qp, kp, vp, total;
   int Hs;
   int slot[kMaxHeads];
 };
@@ -186,7 +217,8 @@ static FwdLayout forward_layout(const salad_forward_args* a) {
   L.lin = take(linear_state_ws_bytes(a->B, a->H, a->N, a->d));
   L.hst = take(B * H * d * d * sizeof(float));
   L.z = take(B * H * d * sizeof(float));
-  L.g = take(B * H * d * d * 2);
+  if (a->w_lin_full != nullptr) L.olin = take(B * H * N * d * 2);   // O_l, bf16 [B,H,N,d]
+  else L.g = take(B * H * d * d * 2);                                // folded H W_lin images
   L.Hs = 0;
   for (int h = 0; h < kMaxHeads; ++h) L.slot[h] = -1;
   if (a->mode == SALAD_MODE_SWA && a->H <= kMaxHeads)
@@ -219,7 +251,7 @@ const char* salad_status_string(salad_status s) {
   }
 }
 
-int salad_version(void) { return 300; }
+int salad_version(void) { return 400; }
 
 // ------------------------------------------------------------------ gate --
 size_t salad_gate_workspace_bytes(int B, int N, int D) {
@@ -289,6 +321,47 @@ salad_status salad_linear_apply(const void* q, const float* Hst, const float* Z,
   Ctx c;
   if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
   return from_cuda(launch_linear_apply(c, q, Hst, Z, eps, B, H, N, d, o_lin));
+}
+
+// ------------------------------------------------------------- project --
+static bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const char* x = static_cast<const char*>(a);
+  const char* y = static_cast<const char*>(b);
+  return x < y + nb && y < x + na;
+}
+
+salad_status salad_project(const void* a, int B, int H, int N, int d, const void* w, int n_out,
+                           void* out, int out_per_head, const void* resid, const float* s,
+                           float drop_threshold, salad_stream stream) {
+  salad_status st = check_bhnd(B, H, N, d);
+  if (st != SALAD_OK) return st;
+  if (n_out < 64 || n_out % 64 != 0 || n_out > 65536) return SALAD_ERR_INVALID_ARG;
+  if (out_per_head != 0 && out_per_head != 1) return SALAD_ERR_INVALID_ARG;
+  if (out_per_head && n_out != H * d) return SALAD_ERR_INVALID_ARG;
+  if (!aligned(a, 16) || !aligned(w, 16) || !aligned(out, 16)) return SALAD_ERR_INVALID_ARG;
+  if (resid != nullptr && !aligned(resid, 16)) return SALAD_ERR_INVALID_ARG;
+  if (s != nullptr && !aligned(s, 4)) return SALAD_ERR_INVALID_ARG;
+  if (std::isinf(drop_threshold)) return SALAD_ERR_INVALID_ARG;
+  const size_t a_bytes = static_cast<size_t>(B) * H * N * d * 2;
+  const size_t w_bytes = static_cast<size_t>(H) * d * n_out * 2;
+  const size_t o_bytes = static_cast<size_t>(B) * N * n_out * 2;
+  if (overlaps(out, o_bytes, a, a_bytes) || overlaps(out, o_bytes, w, w_bytes))
+    return SALAD_ERR_INVALID_ARG;
+  if (resid != nullptr && resid != out && overlaps(out, o_bytes, resid, o_bytes))
+    return SALAD_ERR_INVALID_ARG;
+  Ctx c;
+  if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
+  ProjArgs p;
+  p.a = a;
+  p.B = B; p.H = H; p.N = N; p.d = d;
+  p.w = w;
+  p.n_out = n_out;
+  p.out = out;
+  p.out_per_head = out_per_head;
+  p.resid = resid;
+  p.s = s;
+  p.drop = std::isnan(drop_threshold) ? 0.0f : drop_threshold;
+  return from_cuda(launch_proj(c, p));
 }
 
 // --------------------------------------------------------------- permute --
@@ -415,9 +488,19 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   if (a->block != 64) return SALAD_ERR_UNSUPPORTED;
   if (a->mode != SALAD_MODE_TOPK && a->mode != SALAD_MODE_SWA && a->mode != SALAD_MODE_DENSE)
     return SALAD_ERR_INVALID_ARG;
+  const bool full = a->w_lin_full != nullptr;
   if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->o, 16) ||
-      !aligned(a->x, 16) || !aligned(a->w_gate, 16) || !aligned(a->w_lin, 16))
+      !aligned(a->x, 16) || !aligned(a->w_gate, 16) ||
+      !aligned(full ? a->w_lin_full : a->w_lin, 16))
     return SALAD_ERR_INVALID_ARG;
+  if (a->w_out != nullptr && (!aligned(a->w_out, 16) || !aligned(a->out, 16) ||
+                              a->d_out < 64 || a->d_out % 64 != 0 || a->d_out > 65536))
+    return SALAD_ERR_INVALID_ARG;
+  if (a->w_out != nullptr &&
+      overlaps(a->out, static_cast<size_t>(a->B) * a->N * a->d_out * 2, a->o,
+               static_cast<size_t>(a->B) * a->H * a->N * a->d * 2))
+    return SALAD_ERR_INVALID_ARG;
+  if (full && a->rope3d) return SALAD_ERR_UNSUPPORTED;
   if (a->D < 8 || a->D % 8 != 0) return SALAD_ERR_INVALID_ARG;
   if (!(a->eps >= 0.0f) || !std::isfinite(a->eps)) return SALAD_ERR_INVALID_ARG;
   if (a->s_out != nullptr && !aligned(a->s_out, 4)) return SALAD_ERR_INVALID_ARG;
@@ -503,12 +586,22 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   Rope3D rope;
   if (a->rope3d) rope = make_rope3d(d, a->F, a->Hh, a->Wh, a->rope_base);
   at.rope = rope;
-  if (ok)
-    check(launch_linear_state(cl, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, a->w_lin, G, drop,
-                              rope));
+  void* olin = ws + L.olin;
+  if (!full) {
+    if (ok)
+      check(launch_linear_state(cl, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, a->w_lin, G, drop,
+                                rope));
+    at.Gimg = G;
+    at.Z = Z;
+  } else {
+    // Full-width projection: the linear branch stops at O_l; the attention
+    // runs plain and the projection GEMM adds s_b (O_l W) afterwards.
+    if (ok)
+      check(launch_linear_state(cl, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, nullptr, nullptr,
+                                drop, rope));
+    if (ok) check(launch_linear_apply(cl, a->q, Hst, Z, a->eps, B, H, N, d, olin));
+  }
   check(cudaEventRecord(dv->join_lin, cl.stream));
-  at.Gimg = G;
-  at.Z = Z;
 
   // 2. sparse-branch pattern (ijyty.com 1.1 / 1.2), the caller's stream
   if (a->mode == SALAD_MODE_TOPK) {
@@ -548,6 +641,35 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
                       cudaStreamWaitEvent(c.stream, dv->join_lin, 0) == cudaSuccess;
   if (!ok || !joined || !mark(3, c.stream)) return SALAD_ERR_CUDA;
   if (launch_attention(c, at) != cudaSuccess || !mark(4, c.stream)) return SALAD_ERR_CUDA;
+
+  // 5. full-width projections (steps 4 and 7): O += s_b (cat(O_l) W_full) in
+  // place, then out = cat(O) W_out.
+  if (full) {
+    ProjArgs p;
+    p.a = olin;
+    p.B = B; p.H = H; p.N = N; p.d = d;
+    p.w = a->w_lin_full;
+    p.n_out = H * d;
+    p.out = a->o;
+    p.out_per_head = 1;
+    p.resid = a->o;
+    p.s = s;
+    p.drop = at.drop;
+    if (launch_proj(c, p) != cudaSuccess) return SALAD_ERR_CUDA;
+  }
+  if (a->w_out != nullptr) {
+    ProjArgs p;
+    p.a = a->o;
+    p.B = B; p.H = H; p.N = N; p.d = d;
+    p.w = a->w_out;
+    p.n_out = a->d_out;
+    p.out = a->out;
+    p.out_per_head = 0;
+    p.resid = nullptr;
+    p.s = nullptr;
+    p.drop = 0.0f;
+    if (launch_proj(c, p) != cudaSuccess) return SALAD_ERR_CUDA;
+  }
   return SALAD_OK;
 }
 

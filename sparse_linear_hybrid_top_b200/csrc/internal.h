@@ -134,5 +134,26 @@ cudaError_t launch_debug_wait(const Ctx& c);
 // Tensor map for a bf16 [S, N, d] tensor viewed as 3-D (d, N, S), box
 // (64, 64, 1), 128-byte swizzle.  Returns false on failure.
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, int S, int N, int d);
+bool make_tmap_bf16_heads4d(CUtensorMap* map, const void* base, int B, int H, int N, int d);
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, int rows, int cols);
+
+// ---- full-width projections (proj.cu)
+// out = resid + s_b * (A_cat W) per sample b, where A_cat [N][H*d] is A
+// [B][H][N][d] with the heads of a token concatenated (column h*d + c) and W
+// is row-major [H*d][n_out].  out (and resid, if given) is per-head [B][H][N][d]
+// when n_out == H*d and out_per_head, else token-major [B][N][n_out].  s null:
+// scale 1.  Samples with s_b < drop are skipped (out must equal resid then).
+struct ProjArgs {
+  const void* a;
+  int B, H, N, d;
+  const void* w;
+  int n_out;
+  void* out;
+  int out_per_head;
+  const void* resid;
+  const float* s;
+  float drop;
+};
+cudaError_t launch_proj(const Ctx& c, const ProjArgs& a);
 
 }  // namespace salad

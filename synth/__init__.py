@@ -20,6 +20,9 @@ Recipe (per batch sample b, per head h):
   * Tokens are flattened frame-major: t = (f * Hh + y) * Wh + x.
   * Gate input X ~ N(0, 1) [B, N, D]; gate weight w ~ N(0, 0.02) [D]; bias 0.
   * Per-head linear-branch projection W_lin ~ N(0, 0.02) [H, d, d].
+  * Full-width variants (``generate_projections``): W_lin_full ~ N(0, 0.02)
+    [H*d, H*d] and the output projection W_out ~ N(0, 0.02) [H*d, D_out],
+    from their own stream (seed sequence [seed_0, 0x5A1AD]).
 Random streams: numpy PCG64 seeded by ``SeedSequence(seed_b).spawn(...)``, one
 child stream per tensor.
 """
@@ -32,7 +35,7 @@ from typing import Dict, List, Optional
 import numpy as np
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "generate", "topk_for_sparsity"]
+__all__ = ["Workload", "WORKLOADS", "generate", "generate_projections", "topk_for_sparsity"]
 
 
 def topk_for_sparsity(nb: int, sparsity: float) -> int:
@@ -192,3 +195,17 @@ def generate(w: Workload, heads: Optional[List[int]] = None) -> Dict[str, torch.
         "x": torch.stack(xs), "w_gate": w_gate, "w_lin": w_lin,
         "bias": float(w.bias),
     }
+
+
+def generate_projections(w: Workload, d_out: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Full-width projection weights of one layer as CPU tensors.
+
+    w_lin_full: bf16 [H*d, H*d]; w_out: bf16 [H*d, d_out] (d_out defaults to
+    H*d, the model width of the video DiTs the workloads follow).
+    """
+    K = w.H * w.d
+    d_out = K if d_out is None else int(d_out)
+    rp = np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seeds[0], 0x5A1AD])))
+    w_full = _bf16(rp.normal(0.0, 0.02, size=(K, K)).astype(np.float32))
+    w_out = _bf16(rp.normal(0.0, 0.02, size=(K, d_out)).astype(np.float32))
+    return {"w_lin_full": w_full, "w_out": w_out}

@@ -34,7 +34,7 @@ def test_header_declarations_match_binding_and_exports():
 def test_library_is_built_for_sm100a_only():
     # The binding loads the in-tree library (no fallback path exists).
     assert os.path.dirname(salad.LIB_PATH) == os.path.join(ROOT, "sparse_linear_hybrid_top_b200")
-    assert salad.version() == 300
+    assert salad.version() == 400
 
 
 def test_status_strings():
@@ -94,6 +94,24 @@ def test_permute_argument_checks():
     assert lib.salad_permute_tokens(A, A + (1 << 20), 2, 12, 64, 2, 2, 3, 2, None) == INVALID
 
 
+def test_project_argument_checks():
+    # a [1,2,100,64] -> n_out 128 (per head) or 192 (token-major).
+    P = lib.salad_project
+    big = A + (1 << 24)
+    assert P(A, 1, 2, 100, 64, big, 100, big * 2, 0, None, None, 0.0, None) == INVALID  # n_out % 64
+    assert P(A, 1, 2, 100, 64, big, 0, big * 2, 0, None, None, 0.0, None) == INVALID
+    assert P(A, 1, 2, 100, 64, big, 192, big * 2, 1, None, None, 0.0, None) == INVALID  # != H*d
+    assert P(A, 1, 2, 100, 64, big, 128, big * 2, 2, None, None, 0.0, None) == INVALID
+    assert P(A, 1, 2, 100, 96, big, 192, big * 2, 0, None, None, 0.0, None) == UNSUP    # d
+    assert P(A + 8, 1, 2, 100, 64, big, 128, big * 2, 0, None, None, 0.0, None) == INVALID
+    assert P(A, 1, 2, 100, 64, None, 128, big * 2, 0, None, None, 0.0, None) == INVALID
+    assert P(A, 1, 2, 100, 64, big, 128, A + 64, 0, None, None, 0.0, None) == INVALID   # out over a
+    assert P(A, 1, 2, 100, 64, big, 128, big + 64, 0, None, None, 0.0, None) == INVALID  # over w
+    assert P(A, 1, 2, 100, 64, big, 128, big * 2, 0, big * 2 + 64, None, 0.0, None) == INVALID
+    assert P(A, 1, 2, 100, 64, big, 128, big * 2, 0, None, big * 3 + 2, 0.0, None) == INVALID
+    assert P(A, 1, 2, 100, 64, big, 128, big * 2, 0, None, None, float("inf"), None) == INVALID
+
+
 def _fwd_args(**kw):
     a = ForwardArgs()
     a.q = a.k = a.v = a.x = a.w_gate = a.w_lin = a.o = A
@@ -122,6 +140,22 @@ def test_forward_argument_checks_and_workspace_query():
     bad = _fwd_args(gate_override=float("inf"), workspace=A, workspace_bytes=need)
     assert lib.salad_forward(ctypes.byref(bad), None) == INVALID
     assert lib.salad_forward(None, None) == INVALID
+    # Full-width projections: d_out a multiple of 64, out given and apart
+    # from o, and not combined with the 3-D rotary encoding.
+    big = A + (1 << 24)
+    for kw in (dict(w_out=big, d_out=100, out=big * 2), dict(w_out=big, d_out=128, out=None),
+               dict(w_out=big, d_out=128, out=A + 64), dict(w_out=big + 8, d_out=128, out=big * 2),
+               dict(w_lin_full=big + 8)):
+        bad = _fwd_args(workspace=A, workspace_bytes=need, **kw)
+        assert lib.salad_forward(ctypes.byref(bad), None) == INVALID, kw
+    bad = _fwd_args(w_lin_full=big, rope3d=1, F=10, Hh=10, Wh=10, rope_base=10000.0,
+                    workspace=A, workspace_bytes=need)
+    assert lib.salad_forward(ctypes.byref(bad), None) == UNSUP
+    # The full-width path keeps O_l (bf16 [B,H,N,d]) instead of the folded images.
+    full = _fwd_args(w_lin_full=big)
+    assert (lib.salad_forward_workspace_bytes(ctypes.byref(full)) -
+            lib.salad_forward_workspace_bytes(ctypes.byref(_fwd_args()))) == \
+        2 * 1000 * 64 * 2 - 2 * 64 * 64 * 2
     # Larger problems need more workspace; SWA with regrouped heads adds copies.
     big = _fwd_args(N=31200, d=128, H=12, D=1536, topk=49)
     assert lib.salad_forward_workspace_bytes(ctypes.byref(big)) > need

@@ -432,7 +432,7 @@ def run_ours(args, w) -> int:
         "phases_ms": {k: round(v, 5) for k, v in phases.items()},
         "dense_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / agg["ms_per_step"], 3),
         "variants_ms_per_layer": {k: round(v, 5) for k, v in variants.items()},
-        "proj_gemm": {"kernel": "proj_kernel<256>", "shape": [w.B * w.N, K, K],
+        "proj_gemm": {"kernel": "proj_pair_kernel (cta_group::2, 256 x 256 pair tiles)", "shape": [w.B * w.N, K, K],
                       "ms": round(gemm_ms, 5),
                       "tflops": round(gemm_flops / (gemm_ms * 1e-3) / 1e12, 2),
                       "frac": round(gemm_flops / (gemm_ms * 1e-3) / 1e12 / float(peaks["bf16_tflops"]), 4),

@@ -36,11 +36,14 @@ def _bf16(rng, shape, scale=1.0):
         torch.bfloat16)
 
 
-# (B, H, N, d, n_out): tile widths 256 / 128 / 64, ragged and single-token N.
+# (B, H, N, d, n_out): n_out a multiple of 256 runs on CTA pairs (256-token
+# tiles), the others on single CTAs with 128- or 64-column tiles; ragged and
+# single-token N (a pair tile whose second CTA has no valid row).
 PER_HEAD = [(1, 2, 930, 128, 256), (2, 3, 198, 64, 192), (1, 1, 1, 128, 128),
-            (2, 12, 1000, 128, 1536), (1, 4, 129, 64, 256)]
+            (2, 12, 1000, 128, 1536), (1, 4, 129, 64, 256), (1, 2, 1, 128, 256),
+            (2, 2, 300, 128, 256)]
 TOKEN_MAJOR = [(1, 2, 930, 128, 64), (2, 3, 198, 64, 320), (1, 12, 700, 128, 1536),
-               (1, 1, 1, 64, 128), (2, 5, 260, 64, 384)]
+               (1, 1, 1, 64, 128), (2, 5, 260, 64, 384), (1, 2, 257, 64, 512)]
 
 
 @pytest.mark.parametrize("shape", PER_HEAD, ids=lambda s: "x".join(map(str, s)))

@@ -246,7 +246,7 @@ typedef struct salad_forward_args {
      * NULL for the per-head w_lin.  When set, w_lin is not read and
      *   O[b,:,n,:] = O_sparse + s_b * split_heads(cat_heads(O_l[b,:,n,:]) w_lin_full)
      * with cat_heads putting column h*d + c = O_l[b,h,n,c] (see
-     * salad_project).  Not combined with rope3d (SALAD_ERR_UNSUPPORTED). */
+     * salad_project).  With rope3d, O_l carries the rotation as above. */
     const void* w_lin_full;
     /* Output projection (step 7): bf16 [H*d, d_out] device, or NULL.  When
      * set, out[b,n,:] = cat_heads(O[b,:,n,:]) w_out is written too; o still

@@ -500,7 +500,6 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
       overlaps(a->out, static_cast<size_t>(a->B) * a->N * a->d_out * 2, a->o,
                static_cast<size_t>(a->B) * a->H * a->N * a->d * 2))
     return SALAD_ERR_INVALID_ARG;
-  if (full && a->rope3d) return SALAD_ERR_UNSUPPORTED;
   if (a->D < 8 || a->D % 8 != 0) return SALAD_ERR_INVALID_ARG;
   if (!(a->eps >= 0.0f) || !std::isfinite(a->eps)) return SALAD_ERR_INVALID_ARG;
   if (a->s_out != nullptr && !aligned(a->s_out, 4)) return SALAD_ERR_INVALID_ARG;
@@ -599,7 +598,7 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
     if (ok)
       check(launch_linear_state(cl, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, nullptr, nullptr,
                                 drop, rope));
-    if (ok) check(launch_linear_apply(cl, a->q, Hst, Z, a->eps, B, H, N, d, olin));
+    if (ok) check(launch_linear_apply(cl, a->q, Hst, Z, a->eps, B, H, N, d, olin, rope));
   }
   check(cudaEventRecord(dv->join_lin, cl.stream));
 

@@ -84,7 +84,8 @@ cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int 
                                 const void* w_lin = nullptr, void* Gimg = nullptr,
                                 BranchDrop drop = BranchDrop(), Rope3D rope = Rope3D());
 cudaError_t launch_linear_apply(const Ctx& c, const void* q, const float* Hst, const float* Z,
-                                float eps, int B, int H, int N, int d, void* o);
+                                float eps, int B, int H, int N, int d, void* o,
+                                Rope3D rope = Rope3D());
 
 // ---- permutation (permute.cu)
 cudaError_t launch_permute(const Ctx& c, const void* src, void* dst, int S, int N, int d, int F,

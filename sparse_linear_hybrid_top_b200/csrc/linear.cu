@@ -345,7 +345,7 @@ template <int D>
 __global__ void __launch_bounds__(128, 1) linear_apply_kernel(
     const __nv_bfloat16* __restrict__ q, const float* __restrict__ Hst,
     const float* __restrict__ Z, float eps, int N, int ntiles, __nv_bfloat16* __restrict__ o,
-    unsigned* err, unsigned long long wait_ns) {
+    unsigned* err, unsigned long long wait_ns, const __grid_constant__ Rope3D rope) {
   using C = LA<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -382,6 +382,16 @@ __global__ void __launch_bounds__(128, 1) linear_apply_kernel(
   const bool valid = row < N;
   const uint4* qrow = reinterpret_cast<const uint4*>(q + (bh * N + (valid ? row : 0)) * D);
   float den = 0.f;
+  // 3-D rotary encoding: the numerator's phi(q) turns by the token's frame,
+  // row and column positions; the denominator keeps the unrotated phi(q).
+  const bool rope_on = rope.on && valid;
+  int rf = 0, ry = 0, rx = 0;
+  if (rope_on) {
+    const int tok = static_cast<int>(row);
+    rf = tok / (rope.Hh * rope.Wh);
+    ry = (tok / rope.Wh) % rope.Hh;
+    rx = tok % rope.Wh;
+  }
 #pragma unroll
   for (int c0 = 0; c0 < D / 2; c0 += 16) {  // 16 packed columns = 32 bf16 per step
     uint32_t pk[16];
@@ -398,6 +408,10 @@ __global__ void __launch_bounds__(128, 1) linear_apply_kernel(
       const float2 f = unpack_bf16x2(pk[e]);
       den = fmaf(f.x, zs[2 * (c0 + e)], den);
       den = fmaf(f.y, zs[2 * (c0 + e) + 1], den);
+      if (rope_on) {   // pair c0 + e = channels 2(c0 + e), 2(c0 + e) + 1
+        const float2 cs = rope_cs(rope, rope.theta, c0 + e, rf, ry, rx);
+        pk[e] = pack_bf16x2(f.x * cs.x - f.y * cs.y, f.x * cs.y + f.y * cs.x);
+      }
     }
     tmem_st16(tmem_addr(tmem, warp * 32, a_col + c0), pk);
   }
@@ -547,7 +561,7 @@ Rope3D make_rope3d(int d, int F, int Hh, int Wh, float base) {
 }
 
 cudaError_t launch_linear_apply(const Ctx& c, const void* q, const float* Hst, const float* Z,
-                                float eps, int B, int H, int N, int d, void* o) {
+                                float eps, int B, int H, int N, int d, void* o, Rope3D rope) {
   const int ntiles = (N + 127) / 128;
   const int grid = B * H * ntiles;
   cudaError_t e;
@@ -557,14 +571,14 @@ cudaError_t launch_linear_apply(const Ctx& c, const void* q, const float* Hst, c
     if (e != cudaSuccess) return e;
     linear_apply_kernel<128><<<grid, 128, LA<128>::kSmem, c.stream>>>(
         static_cast<const __nv_bfloat16*>(q), Hst, Z, eps, N, ntiles,
-        static_cast<__nv_bfloat16*>(o), c.err, c.wait_ns);
+        static_cast<__nv_bfloat16*>(o), c.err, c.wait_ns, rope);
   } else {
     e = cudaFuncSetAttribute(linear_apply_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              LA<64>::kSmem);
     if (e != cudaSuccess) return e;
     linear_apply_kernel<64><<<grid, 128, LA<64>::kSmem, c.stream>>>(
         static_cast<const __nv_bfloat16*>(q), Hst, Z, eps, N, ntiles,
-        static_cast<__nv_bfloat16*>(o), c.err, c.wait_ns);
+        static_cast<__nv_bfloat16*>(o), c.err, c.wait_ns, rope);
   }
   return cudaGetLastError();
 }

@@ -141,16 +141,13 @@ def test_forward_argument_checks_and_workspace_query():
     assert lib.salad_forward(ctypes.byref(bad), None) == INVALID
     assert lib.salad_forward(None, None) == INVALID
     # Full-width projections: d_out a multiple of 64, out given and apart
-    # from o, and not combined with the 3-D rotary encoding.
+    # from o.
     big = A + (1 << 24)
     for kw in (dict(w_out=big, d_out=100, out=big * 2), dict(w_out=big, d_out=128, out=None),
                dict(w_out=big, d_out=128, out=A + 64), dict(w_out=big + 8, d_out=128, out=big * 2),
                dict(w_lin_full=big + 8)):
         bad = _fwd_args(workspace=A, workspace_bytes=need, **kw)
         assert lib.salad_forward(ctypes.byref(bad), None) == INVALID, kw
-    bad = _fwd_args(w_lin_full=big, rope3d=1, F=10, Hh=10, Wh=10, rope_base=10000.0,
-                    workspace=A, workspace_bytes=need)
-    assert lib.salad_forward(ctypes.byref(bad), None) == UNSUP
     # The full-width path keeps O_l (bf16 [B,H,N,d]) instead of the folded images.
     full = _fwd_args(w_lin_full=big)
     assert (lib.salad_forward_workspace_bytes(ctypes.byref(full)) -

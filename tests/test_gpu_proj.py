@@ -142,6 +142,25 @@ def test_forward_full_width(salad, w):
     assert_close(plan.out, ref["out"], f"forward output projection {w.name}")
 
 
+@pytest.mark.parametrize("w", CASES + [SWA_SMALL], ids=lambda w: w.name)
+def test_forward_full_width_rope3d(salad, w):
+    # The rotary encoding turns phi(q) in the linear-apply kernel that feeds
+    # the full-width projection (numerator only, as in the per-head path).
+    inp = generate(w)
+    dev = device_inputs(inp)
+    proj_cpu = generate_projections(w)
+    proj = device_inputs(proj_cpu)
+    grid = {} if w.mode == "swa" else dict(F=w.F, Hh=w.Hh, Wh=w.Wh)
+    plan = _full_plan(salad, w, dev, proj, rope3d=True, **grid)
+    o = plan.run()
+    torch.cuda.synchronize()
+    salad.check_error()
+    ref = oracle.forward(inp, w_lin_full=proj_cpu["w_lin_full"], w_out=proj_cpu["w_out"],
+                         rope3d=True, **_oracle_kw(w, inp, plan))
+    assert_close(o, ref["o"], f"forward full-width with rope3d {w.name}")
+    assert_close(plan.out, ref["out"], f"output projection with rope3d {w.name}")
+
+
 def test_forward_full_width_branch_dropping(salad):
     w = RAGGED128_B2
     inp = generate(w)

@@ -388,6 +388,16 @@ def test_full_width_projection_reduces_and_orients():
     np.testing.assert_array_equal(diff, 0.0)
 
 
+def test_full_width_golden():
+    # Hand-derived worked example (tests/golden/full_width_projection.json).
+    g = json.load(open(os.path.join(GOLD, "full_width_projection.json")))
+    o = oracle.combine_full(np.array(g["o_sparse"]), np.array(g["o_lin"]), np.array(g["w_full"]),
+                            g["s"])
+    np.testing.assert_array_equal(o, np.array(g["o"]))
+    out = oracle.output_projection(o, np.array(g["w_out"]))
+    np.testing.assert_array_equal(out, np.array(g["out"]))
+
+
 def test_output_projection_orients():
     inp = _tiny_inputs(seed=98)
     H, d, N = 2, 16, 192

@@ -148,6 +148,14 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _shape(t, shape, name: str):
+    """Exact shape check, before any device access (a wrong size would make a
+    kernel read past the tensor)."""
+    if not isinstance(t, torch.Tensor) or tuple(t.shape) != tuple(shape):
+        got = tuple(t.shape) if isinstance(t, torch.Tensor) else type(t).__name__
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {got}")
+
+
 def _dev_tensor(t: torch.Tensor, dtype, name: str):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -252,10 +260,22 @@ def project(a: torch.Tensor, w: torch.Tensor, *, out_per_head: bool = False, res
     (same layout as out, may be ``out`` itself) and s (float32 [B]) are
     optional; samples with s_b < drop_threshold are left unwritten.
     """
+    if not isinstance(a, torch.Tensor) or a.dim() != 4:
+        raise ValueError("a must be a [B, H, N, d] tensor")
+    B, H, N, d = a.shape
+    if not isinstance(w, torch.Tensor) or w.dim() != 2:
+        raise ValueError("w must be a [H*d, n_out] tensor")
+    n_out = w.shape[-1]
+    _shape(w, (H * d, n_out), "w")
+    out_shape = (B, H, N, d) if out_per_head else (B, N, n_out)
+    if out is not None:
+        _shape(out, out_shape, "out")
+    if resid is not None:
+        _shape(resid, out_shape, "resid")
+    if s is not None:
+        _shape(s, (B,), "s")
     _dev_tensor(a, torch.bfloat16, "a")
     _dev_tensor(w, torch.bfloat16, "w")
-    B, H, N, d = a.shape
-    n_out = w.shape[-1]
     if out is None:
         out = torch.empty((B, H, N, d) if out_per_head else (B, N, n_out), dtype=torch.bfloat16,
                           device=a.device)
@@ -326,11 +346,36 @@ class ForwardPlan:
                  rope3d: bool = False, rope_base: float = 10000.0, o=None,
                  s_out=None, idx_out=None, block: int = 64, w_lin_full=None, w_out=None,
                  out=None):
+        # Shapes first (a wrong size would make a kernel read past a tensor).
+        if not isinstance(q, torch.Tensor) or q.dim() != 4:
+            raise ValueError("q must be a [B, H, N, d] tensor")
+        B, H, N, d = q.shape
+        _shape(k, q.shape, "k")
+        _shape(v, q.shape, "v")
+        if not isinstance(x, torch.Tensor) or x.dim() != 3:
+            raise ValueError("x must be a [B, N, D] tensor")
+        _shape(x, (B, N, x.shape[-1]), "x")
+        _shape(w_gate, (x.shape[-1],), "w_gate")
+        if w_lin is not None:
+            _shape(w_lin, (H, d, d), "w_lin")
+        if w_lin_full is not None:
+            _shape(w_lin_full, (H * d, H * d), "w_lin_full")
+        if w_out is not None:
+            if w_out.dim() != 2:
+                raise ValueError("w_out must be a [H*d, d_out] tensor")
+            _shape(w_out, (H * d, w_out.shape[-1]), "w_out")
+            if out is not None:
+                _shape(out, (B, N, w_out.shape[-1]), "out")
+        if o is not None:
+            _shape(o, q.shape, "o")
+        if s_out is not None:
+            _shape(s_out, (B,), "s_out")
+        if idx_out is not None and mode == "topk":
+            _shape(idx_out, (B, H, (N + block - 1) // block, int(topk)), "idx_out")
         for n, t in (("q", q), ("k", k), ("v", v), ("x", x), ("w_gate", w_gate),
                      ("w_lin", w_lin), ("w_lin_full", w_lin_full), ("w_out", w_out)):
             if t is not None or n in ("q", "k", "v", "x", "w_gate"):
                 _dev_tensor(t, torch.bfloat16, n)
-        B, H, N, d = q.shape
         self.tensors = dict(q=q, k=k, v=v, x=x, w_gate=w_gate, w_lin=w_lin,
                             w_lin_full=w_lin_full, w_out=w_out)
         # Output projection (optional): out [B,N,d_out] = cat_heads(O) w_out.

@@ -1,0 +1,77 @@
+"""The binding checks every tensor's shape before anything reaches the device
+(a wrong size would make a kernel read past a tensor).  On the CPU the checks
+run on host tensors: a well-formed call stops at the device check, a
+malformed one at the shape check."""
+import pytest
+import torch
+
+import sparse_linear_hybrid_top_b200 as salad
+from synth import WORKLOADS, generate, generate_projections
+from tests.test_gpu_attention import SWA_SMALL
+from tests.test_gpu_kernels import CASES
+
+
+def _expect_device_error(fn):
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fn()
+
+
+def _expect_shape_error(fn, name):
+    with pytest.raises(ValueError, match=f"{name} must"):
+        fn()
+
+
+def _plan(w, inp, **kw):
+    extra = dict(window=w.window, space_major_heads=w.space_major_heads, F=w.F, Hh=w.Hh,
+                 Wh=w.Wh) if w.mode == "swa" else {}
+    return salad.ForwardPlan(inp["q"], inp["k"], inp["v"], inp["x"], inp["w_gate"],
+                             kw.pop("w_lin", inp["w_lin"]), mode=w.mode, topk=w.topk,
+                             bias=w.bias, eps=w.eps, **extra, **kw)
+
+
+@pytest.mark.parametrize("w", CASES + [SWA_SMALL], ids=lambda w: w.name)
+def test_forward_plan_shapes_accepted(w):
+    inp = generate(w)
+    nb = w.nb
+    idx = torch.empty(w.B, w.H, nb, max(w.topk, 1), dtype=torch.int32) if w.mode == "topk" \
+        else None
+    s_out = torch.empty(w.B, dtype=torch.float32)
+    _expect_device_error(lambda: _plan(w, inp, idx_out=idx, s_out=s_out))
+    proj = generate_projections(w, d_out=256)
+    _expect_device_error(lambda: _plan(w, inp, w_lin=None, w_lin_full=proj["w_lin_full"],
+                                       w_out=proj["w_out"], idx_out=idx, s_out=s_out))
+
+
+def test_forward_plan_shapes_rejected():
+    w = WORKLOADS["tiny"]
+    inp = generate(w)
+    bad = dict(inp)
+    bad["k"] = inp["k"][:, :, :-1]
+    _expect_shape_error(lambda: _plan(w, bad), "k")
+    bad = dict(inp)
+    bad["w_gate"] = inp["w_gate"][:-8]
+    _expect_shape_error(lambda: _plan(w, bad), "w_gate")
+    _expect_shape_error(lambda: _plan(w, inp, w_lin=inp["w_lin"][:, :, :-1]), "w_lin")
+    proj = generate_projections(w)
+    _expect_shape_error(lambda: _plan(w, inp, w_lin_full=proj["w_lin_full"][:-64]), "w_lin_full")
+    _expect_shape_error(lambda: _plan(w, inp, w_out=proj["w_out"][:-64]), "w_out")
+    _expect_shape_error(lambda: _plan(w, inp, w_out=proj["w_out"],
+                                      out=torch.empty(w.B, w.N, 64, dtype=torch.bfloat16)), "out")
+    _expect_shape_error(lambda: _plan(w, inp, idx_out=torch.empty(w.B, w.H, w.nb, w.topk + 1,
+                                                                  dtype=torch.int32)), "idx_out")
+    _expect_shape_error(lambda: _plan(w, inp, s_out=torch.empty(w.B + 1)), "s_out")
+
+
+def test_project_shapes():
+    B, H, N, d = 2, 3, 50, 64
+    a = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
+    w = torch.zeros(H * d, 192, dtype=torch.bfloat16)
+    res = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
+    s = torch.zeros(B)
+    _expect_device_error(lambda: salad.project(a, w, out_per_head=True, resid=res, s=s))
+    _expect_device_error(lambda: salad.project(a, torch.zeros(H * d, 320, dtype=torch.bfloat16)))
+    _expect_shape_error(lambda: salad.project(a, w[:-64]), "w")
+    _expect_shape_error(lambda: salad.project(a, w, out_per_head=True, resid=res[:, :, :-1]),
+                        "resid")
+    _expect_shape_error(lambda: salad.project(a, w, out=torch.zeros(B, N, 64)), "out")
+    _expect_shape_error(lambda: salad.project(a, w, s=torch.zeros(B + 1)), "s")

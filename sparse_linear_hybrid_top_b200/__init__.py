@@ -156,6 +156,11 @@ def _shape(t, shape, name: str):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {got}")
 
 
+def _dims(t, n: int, name: str, layout: str):
+    if not isinstance(t, torch.Tensor) or t.dim() != n:
+        raise ValueError(f"{name} must be a {layout} tensor")
+
+
 def _dev_tensor(t: torch.Tensor, dtype, name: str):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -190,8 +195,12 @@ def _flags(space_major_heads, H: int):
 def gate(x: torch.Tensor, w: torch.Tensor, bias: float = 0.0, *, s=None, workspace=None,
          stream=None) -> torch.Tensor:
     """s[b] = sigmoid(w . mean_n x[b, n, :] + bias); x bf16 [B,N,D], w bf16 [D]."""
-    _dev_tensor(x, torch.bfloat16, "x"); _dev_tensor(w, torch.bfloat16, "w")
+    _dims(x, 3, "x", "[B, N, D]")
     B, N, D = x.shape
+    _shape(w, (D,), "w")
+    if s is not None:
+        _shape(s, (B,), "s")
+    _dev_tensor(x, torch.bfloat16, "x"); _dev_tensor(w, torch.bfloat16, "w")
     s = torch.empty(B, dtype=torch.float32, device=x.device) if s is None else s
     ws = _workspace(lib.salad_gate_workspace_bytes(B, N, D), x.device, workspace)
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
@@ -205,8 +214,12 @@ def gate_noalloc(x: torch.Tensor, w: torch.Tensor, bias: float = 0.0, *, s=None,
     """The gate for callers that cannot allocate scratch: same result as
     gate(), partial sums kept in the library's own fixed device array
     (B <= 256; calls that overlap on the GPU race on that array)."""
-    _dev_tensor(x, torch.bfloat16, "x"); _dev_tensor(w, torch.bfloat16, "w")
+    _dims(x, 3, "x", "[B, N, D]")
     B, N, D = x.shape
+    _shape(w, (D,), "w")
+    if s is not None:
+        _shape(s, (B,), "s")
+    _dev_tensor(x, torch.bfloat16, "x"); _dev_tensor(w, torch.bfloat16, "w")
     s = torch.empty(B, dtype=torch.float32, device=x.device) if s is None else s
     _check(lib.salad_gate_noalloc(_ptr(x), _ptr(w), float(bias), B, N, D, _ptr(s),
                                   _stream(stream)), "salad_gate_noalloc")
@@ -216,9 +229,13 @@ def gate_noalloc(x: torch.Tensor, w: torch.Tensor, bias: float = 0.0, *, s=None,
 def select_blocks(q: torch.Tensor, k: torch.Tensor, topk: int, *, block: int = 64, idx=None,
                   workspace=None, stream=None) -> torch.Tensor:
     """Top-K key blocks per query block: int32 [B, H, nb, topk], ascending."""
-    _dev_tensor(q, torch.bfloat16, "q"); _dev_tensor(k, torch.bfloat16, "k")
+    _dims(q, 4, "q", "[B, H, N, d]")
     B, H, N, d = q.shape
     nb = (N + block - 1) // block
+    _shape(k, q.shape, "k")
+    if idx is not None:
+        _shape(idx, (B, H, nb, int(topk)), "idx")
+    _dev_tensor(q, torch.bfloat16, "q"); _dev_tensor(k, torch.bfloat16, "k")
     idx = torch.empty(B, H, nb, topk, dtype=torch.int32, device=q.device) if idx is None else idx
     ws = _workspace(lib.salad_select_workspace_bytes(B, H, N, d, block), q.device, workspace)
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
@@ -229,6 +246,8 @@ def select_blocks(q: torch.Tensor, k: torch.Tensor, topk: int, *, block: int = 6
 
 def linear_state(k: torch.Tensor, v: torch.Tensor, *, workspace=None, stream=None):
     """(H, Z): float32 [B,H,d,d] = relu(K)^T V and [B,H,d] = relu(K)^T 1."""
+    _dims(k, 4, "k", "[B, H, N, d]")
+    _shape(v, k.shape, "v")
     _dev_tensor(k, torch.bfloat16, "k"); _dev_tensor(v, torch.bfloat16, "v")
     B, H, N, d = k.shape
     Hst = torch.empty(B, H, d, d, dtype=torch.float32, device=k.device)
@@ -243,9 +262,14 @@ def linear_state(k: torch.Tensor, v: torch.Tensor, *, workspace=None, stream=Non
 def linear_apply(q: torch.Tensor, Hst: torch.Tensor, Z: torch.Tensor, eps: float = 1e-6, *,
                  o=None, stream=None) -> torch.Tensor:
     """relu(q) H / (relu(q) . Z + eps) as bf16 [B,H,N,d]."""
+    _dims(q, 4, "q", "[B, H, N, d]")
+    B, H, N, d = q.shape
+    _shape(Hst, (B, H, d, d), "Hst")
+    _shape(Z, (B, H, d), "Z")
+    if o is not None:
+        _shape(o, q.shape, "o")
     _dev_tensor(q, torch.bfloat16, "q")
     _dev_tensor(Hst, torch.float32, "Hst"); _dev_tensor(Z, torch.float32, "Z")
-    B, H, N, d = q.shape
     o = torch.empty_like(q) if o is None else o
     _check(lib.salad_linear_apply(_ptr(q), _ptr(Hst), _ptr(Z), float(eps), B, H, N, d, _ptr(o),
                                   _stream(stream)), "salad_linear_apply")
@@ -293,6 +317,10 @@ def project(a: torch.Tensor, w: torch.Tensor, *, out_per_head: bool = False, res
 def permute_tokens(src: torch.Tensor, F: int, Hh: int, Wh: int, *, inverse: bool = False,
                    dst=None, stream=None) -> torch.Tensor:
     """Frame-major <-> space-major row order of [..., N, d] slabs."""
+    if not isinstance(src, torch.Tensor) or src.dim() < 2:
+        raise ValueError("src must be a [..., N, d] tensor")
+    if dst is not None:
+        _shape(dst, src.shape, "dst")
     _dev_tensor(src, torch.bfloat16, "src")
     N, d = src.shape[-2:]
     S = src.numel() // (N * d)
@@ -306,9 +334,16 @@ def sparse_attn(q, k, v, mode: str = "topk", *, topk: int = 0, idx=None, window:
                 space_major_heads: Optional[Sequence[int]] = None, F: int = 0, Hh: int = 0,
                 Wh: int = 0, block: int = 64, o=None, workspace=None, stream=None):
     """Normalised sparse-branch attention output, bf16 [B,H,N,d]."""
+    _dims(q, 4, "q", "[B, H, N, d]")
+    B, H, N, d = q.shape
+    _shape(k, q.shape, "k")
+    _shape(v, q.shape, "v")
+    if o is not None:
+        _shape(o, q.shape, "o")
+    if mode == "topk" and idx is not None:
+        _shape(idx, (B, H, (N + block - 1) // block, int(topk)), "idx")
     for n, t in (("q", q), ("k", k), ("v", v)):
         _dev_tensor(t, torch.bfloat16, n)
-    B, H, N, d = q.shape
     m = _MODES[mode]
     flags, fptr = _flags(space_major_heads, H)
     o = torch.empty_like(q) if o is None else o
@@ -323,6 +358,11 @@ def sparse_attn(q, k, v, mode: str = "topk", *, topk: int = 0, idx=None, window:
 
 def dense_attn(q, k, v, *, o=None, stream=None):
     """Dense flash attention softmax(Q K^T / sqrt(d)) V, bf16 [B,H,N,d]."""
+    _dims(q, 4, "q", "[B, H, N, d]")
+    _shape(k, q.shape, "k")
+    _shape(v, q.shape, "v")
+    if o is not None:
+        _shape(o, q.shape, "o")
     for n, t in (("q", q), ("k", k), ("v", v)):
         _dev_tensor(t, torch.bfloat16, n)
     B, H, N, d = q.shape

@@ -75,3 +75,43 @@ def test_project_shapes():
                         "resid")
     _expect_shape_error(lambda: salad.project(a, w, out=torch.zeros(B, N, 64)), "out")
     _expect_shape_error(lambda: salad.project(a, w, s=torch.zeros(B + 1)), "s")
+
+
+def test_piecewise_calls_shapes():
+    w = WORKLOADS["tiny"]
+    inp = generate(w)
+    q, k, v, x, wg = inp["q"], inp["k"], inp["v"], inp["x"], inp["w_gate"]
+    B, H, N, d = q.shape
+    nb = w.nb
+    # Well-formed calls stop at the device check.
+    _expect_device_error(lambda: salad.gate(x, wg, 0.0))
+    _expect_device_error(lambda: salad.gate_noalloc(x, wg, 0.0, s=torch.zeros(B)))
+    _expect_device_error(lambda: salad.select_blocks(q, k, w.topk))
+    _expect_device_error(lambda: salad.select_blocks(
+        q, k, 2, idx=torch.zeros(B, H, nb, 2, dtype=torch.int32)))
+    _expect_device_error(lambda: salad.linear_state(k, v))
+    _expect_device_error(lambda: salad.linear_apply(q, torch.zeros(B, H, d, d), torch.zeros(B, H, d)))
+    _expect_device_error(lambda: salad.permute_tokens(torch.zeros(2, N, d, dtype=torch.bfloat16),
+                                                      w.F, w.Hh, w.Wh))
+    idx = torch.zeros(B, H, nb, w.topk, dtype=torch.int32)
+    _expect_device_error(lambda: salad.sparse_attn(q, k, v, "topk", topk=w.topk, idx=idx))
+    _expect_device_error(lambda: salad.sparse_attn(q, k, v, "swa", window=8))
+    _expect_device_error(lambda: salad.dense_attn(q, k, v))
+    # Malformed ones stop at the shape check.
+    _expect_shape_error(lambda: salad.gate(x, wg[:-8], 0.0), "w")
+    _expect_shape_error(lambda: salad.gate(x, wg, 0.0, s=torch.zeros(B + 1)), "s")
+    _expect_shape_error(lambda: salad.select_blocks(q, k[:, :, :-1], w.topk), "k")
+    _expect_shape_error(lambda: salad.select_blocks(
+        q, k, 2, idx=torch.zeros(B, H, nb, 3, dtype=torch.int32)), "idx")
+    _expect_shape_error(lambda: salad.linear_state(k, v[..., :-1]), "v")
+    _expect_shape_error(lambda: salad.linear_apply(q, torch.zeros(B, H, d, d - 1),
+                                                   torch.zeros(B, H, d)), "Hst")
+    _expect_shape_error(lambda: salad.linear_apply(q, torch.zeros(B, H, d, d),
+                                                   torch.zeros(B, H + 1, d)), "Z")
+    _expect_shape_error(lambda: salad.permute_tokens(
+        torch.zeros(2, N, d, dtype=torch.bfloat16), w.F, w.Hh, w.Wh,
+        dst=torch.zeros(2, N - 1, d, dtype=torch.bfloat16)), "dst")
+    _expect_shape_error(lambda: salad.sparse_attn(q, k, v, "topk", topk=w.topk,
+                                                  idx=idx[:, :, :-1]), "idx")
+    _expect_shape_error(lambda: salad.sparse_attn(q, k, v[:, :1], "swa", window=8), "v")
+    _expect_shape_error(lambda: salad.dense_attn(q, k, v, o=q[:, :, :-1]), "o")

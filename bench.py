@@ -67,6 +67,39 @@ def step_flops(w) -> dict:
             "attn_kernel": attn_kernel, "dense": dense}
 
 
+def input_bytes(w) -> int:
+    """Bytes of one layer's inputs: Q, K, V, X, the gate weight and W_lin (bf16)."""
+    return 2 * (3 * w.B * w.H * w.N * w.d + w.B * w.N * w.D + w.D + w.H * w.d * w.d)
+
+
+def config_of(w, world: int) -> dict:
+    """The workload's `config` dict, identical in both arms of the benchmark."""
+    fl = step_flops(w)
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+            "block": w.block, "mode": w.mode, "topk": w.topk, "window": w.window,
+            "nb": w.nb, "D": w.D,
+            "sparsity": round(1 - fl["sparse"] / fl["dense"], 4),
+            "parallelism": f"replicas{world}",
+            "l2": "no flush: inputs (Q,K,V,X) %.0f MB > 126 MB L2" % (input_bytes(w) / 1e6)}
+
+
+def choose_peak(peaks: dict, timed_ms: float, clk: dict):
+    """The bf16 peak a kernel timed inside this run is held to.
+
+    The burst figure (a GEMM timed alone at full clocks) applies when the
+    timed region is short -- under a second -- and the SM clock sampled
+    during it stayed at its maximum; a seconds-long region, or one whose
+    clock sagged under the power cap, is held to the sustained figure.
+    Returns (peak, label)."""
+    burst = float(peaks["bf16_tflops"])
+    sustained = float(peaks.get("bf16_tflops_sustained") or burst)
+    mhz, mx = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    at_max = mhz is not None and mx is not None and mhz >= 0.97 * mx
+    if timed_ms < 1000.0 and (at_max or mhz is None):
+        return burst, "bf16 burst"
+    return sustained, "bf16 sustained"
+
+
 def launches_per_step(w) -> int:
     # gate (2) + [pool, score, topk, pair_union | gather] + linear state and
     # reduce+fold (2) + attention (1)
@@ -462,19 +495,14 @@ def run_ours(args, w) -> int:
     del sets, plans, outs
 
     peaks, peaks_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    peak, peak_kind = choose_peak(peaks, local_ms, clk)
     achieved = fl["attn_kernel"] / (attn_ms * 1e-3) / 1e12
     line = {
         "metric": METRIC, "value": round(agg["value"], 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "block": w.block, "mode": w.mode, "topk": w.topk, "window": w.window,
-                   "nb": w.nb, "D": w.D,
-                   "sparsity": round(1 - fl["sparse"] / fl["dense"], 4),
-                   "parallelism": f"replicas{world}",
-                   "l2": "no flush: inputs (Q,K,V,X) %.0f MB > 126 MB L2" % (h2d / 1e6)},
+        "config": config_of(w, world),
         "ms_per_layer": round(agg["ms_per_step"], 5),
         "phases_ms": {k: round(v, 5) for k, v in phases.items()},
         "dense_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / agg["ms_per_step"], 3),
@@ -487,7 +515,12 @@ def run_ours(args, w) -> int:
         "flops_per_step": fl["total"],
         "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,hybrid>",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "peak_source": f"bf16 sustained, {peaks_src}",
+                     "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_kind}, {peaks_src} (timed region {local_ms:.1f} ms, "
+                                    f"median SM clock {clk.get('sm_mhz')} of {clk.get('sm_max_mhz')} MHz)",
+                     "frac_of_burst": round(achieved / float(peaks["bf16_tflops"]), 4),
+                     "frac_of_sustained": round(
+                         achieved / float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]), 4),
                      "traffic": committed_traffic(w.name),
                      "algorithmic_flops_per_launch": fl["attn_kernel"]},
         "e2e": {"value": round(e2e["value"], 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -535,8 +568,7 @@ def run_reference(args, w) -> int:
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(t_secs * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "block": w.block, "mode": w.mode, "topk": w.topk, "window": w.window},
+        "config": config_of(w, world),
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cpu_threads(),
                          "kind": "oracle",
                          "sample": f"per step: gate over all X; 1 head: selection, linear "

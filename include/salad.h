@@ -24,8 +24,9 @@
  *     synchronises.  Scratch memory is a caller-provided device workspace
  *     whose size is returned by the matching *_workspace_bytes query;
  *     256-byte alignment is required.  salad_forward alone creates, on its
- *     first call on a device, two streams and three events of its own (kept
- *     until the process exits) to run independent steps side by side.
+ *     first call on each caller stream, two streams and three events of its
+ *     own (kept until the process exits) to run independent steps side by
+ *     side.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) in call order.  All argument checks run on the host before any
  *     launch: an invalid call returns an error and enqueues nothing.
@@ -79,10 +80,15 @@ salad_status salad_gate(const void* x, const void* w, float bias, int B, int N, 
  * Gate with no scratch argument, for callers that cannot allocate device
  * memory at all (a plug-in that receives only its input and output buffers,
  * or code on a path where an allocator call is not permitted).  No passage of
- * the paper corresponds to it: it computes exactly what salad_gate computes,
- * but keeps its per-CTA partial sums in a fixed 64 KB array inside the
- * library (present on every GPU that loads the library, until the process
- * exits) instead of a caller workspace.
+ * the paper corresponds to it.  It keeps its per-CTA partial sums in a fixed
+ * 64 KB array inside the library (present on every GPU that loads the
+ * library, until the process exits) instead of a caller workspace.
+ *   - Result: the value salad_gate computes, from the same kernels and the
+ *     same partition of the tokens whenever that partition's B x parts
+ *     partial sums fit the array's 16384 floats -- on a 148-SM B200 that
+ *     holds for every accepted B, N and D, and the two results are then
+ *     bit-identical.  (Were it not to fit, fewer parts per sample would be
+ *     used, which changes only the float32 rounding of the partial sums.)
  *   - B may be at most 256; larger batches return SALAD_ERR_INVALID_ARG
  *     before any launch.  Other arguments as for salad_gate.
  *   - The first call on each device looks up the array's device address;
@@ -123,9 +129,15 @@ salad_status salad_linear_state(const void* k, const void* v, int B, int H, int 
                                 salad_stream stream);
 
 /*
- * Linear-attention output: o_lin[b,h,n,:] = relu(q) Hst / (relu(q) . Z + eps).
- * q: bf16 [B,H,N,d]; Hst, Z: float32 as produced above; o_lin: bf16 [B,H,N,d]
- * (out).  Needs no workspace.
+ * Linear-attention output (paper.rainbus.top 前置知识 Linear Attention, the
+ * output phi(Q) H / (phi(Q) Z) of the state above; 方法步骤详情 step 3, the
+ * linear branch on the layer's own Q):
+ *   o_lin[b,h,n,:] = relu(q) Hst / (relu(q) . Z + eps).
+ * eps (>= 0, finite) keeps a row with relu(q) = 0 at zero instead of 0/0.
+ * q: bf16 [B,H,N,d] device; Hst, Z: float32 device, as produced by
+ * salad_linear_state; o_lin: bf16 [B,H,N,d] device (out), must not overlap q.
+ * Needs no workspace.  Errors: SALAD_ERR_INVALID_ARG for a null or
+ * misaligned pointer, a bad size or eps; nothing is enqueued then.
  */
 salad_status salad_linear_apply(const void* q, const float* Hst, const float* Z, float eps,
                                 int B, int H, int N, int d, void* o_lin, salad_stream stream);
@@ -201,9 +213,15 @@ salad_status salad_project(const void* a, int B, int H, int N, int d, const void
  * The sparse pattern runs on `stream`; the gate and the linear branch run on
  * two streams of the library forked from `stream` by an event and joined
  * back to it before the attention kernel, so all work is ordered after the
- * caller's earlier work on `stream` and before its later work.  Calls on one
- * device are serialised on the host while they enqueue (the fork and join
- * events are shared).
+ * caller's earlier work on `stream` and before its later work.
+ * Reentrant: each caller stream gets its own two side streams and fork/join
+ * events (created by the first call on that stream -- make it before the
+ * stream is captured into a CUDA graph -- and kept until the process exits;
+ * up to 32 caller streams per device, after which a call enqueues every step
+ * on `stream` itself, in order).  So calls from several threads on different
+ * streams neither wait for one another on the host nor depend on one another
+ * on the GPU; calls on the same stream are serialised while they enqueue.
+ * Concurrent calls must not share a workspace or an output buffer.
  */
 typedef struct salad_forward_args {
     const void* q;              /* bf16 [B,H,N,d] device */

@@ -162,9 +162,17 @@ def _dims(t, n: int, name: str, layout: str):
 
 
 def _dev_tensor(t: torch.Tensor, dtype, name: str):
+    """A tensor the library reads or writes: on the current CUDA device (the
+    library launches there), of the documented dtype, contiguous.  Checked
+    for inputs and caller-supplied outputs alike, before any launch: a host
+    tensor would hand the kernel a host pointer, a tensor of another device
+    would be used on the wrong GPU, and a wrong dtype would be misread."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
-    if t.dtype != dtype:
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
+    if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
@@ -174,6 +182,7 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> Option
     if nbytes == 0:
         return workspace
     if workspace is not None:
+        _dev_tensor(workspace, None, "workspace")
         if workspace.numel() * workspace.element_size() < nbytes:
             raise ValueError("workspace too small")
         return workspace
@@ -201,6 +210,8 @@ def gate(x: torch.Tensor, w: torch.Tensor, bias: float = 0.0, *, s=None, workspa
     if s is not None:
         _shape(s, (B,), "s")
     _dev_tensor(x, torch.bfloat16, "x"); _dev_tensor(w, torch.bfloat16, "w")
+    if s is not None:
+        _dev_tensor(s, torch.float32, "s")
     s = torch.empty(B, dtype=torch.float32, device=x.device) if s is None else s
     ws = _workspace(lib.salad_gate_workspace_bytes(B, N, D), x.device, workspace)
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
@@ -220,6 +231,8 @@ def gate_noalloc(x: torch.Tensor, w: torch.Tensor, bias: float = 0.0, *, s=None,
     if s is not None:
         _shape(s, (B,), "s")
     _dev_tensor(x, torch.bfloat16, "x"); _dev_tensor(w, torch.bfloat16, "w")
+    if s is not None:
+        _dev_tensor(s, torch.float32, "s")
     s = torch.empty(B, dtype=torch.float32, device=x.device) if s is None else s
     _check(lib.salad_gate_noalloc(_ptr(x), _ptr(w), float(bias), B, N, D, _ptr(s),
                                   _stream(stream)), "salad_gate_noalloc")
@@ -236,6 +249,8 @@ def select_blocks(q: torch.Tensor, k: torch.Tensor, topk: int, *, block: int = 6
     if idx is not None:
         _shape(idx, (B, H, nb, int(topk)), "idx")
     _dev_tensor(q, torch.bfloat16, "q"); _dev_tensor(k, torch.bfloat16, "k")
+    if idx is not None:
+        _dev_tensor(idx, torch.int32, "idx")
     idx = torch.empty(B, H, nb, topk, dtype=torch.int32, device=q.device) if idx is None else idx
     ws = _workspace(lib.salad_select_workspace_bytes(B, H, N, d, block), q.device, workspace)
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
@@ -270,6 +285,8 @@ def linear_apply(q: torch.Tensor, Hst: torch.Tensor, Z: torch.Tensor, eps: float
         _shape(o, q.shape, "o")
     _dev_tensor(q, torch.bfloat16, "q")
     _dev_tensor(Hst, torch.float32, "Hst"); _dev_tensor(Z, torch.float32, "Z")
+    if o is not None:
+        _dev_tensor(o, torch.bfloat16, "o")
     o = torch.empty_like(q) if o is None else o
     _check(lib.salad_linear_apply(_ptr(q), _ptr(Hst), _ptr(Z), float(eps), B, H, N, d, _ptr(o),
                                   _stream(stream)), "salad_linear_apply")
@@ -322,6 +339,8 @@ def permute_tokens(src: torch.Tensor, F: int, Hh: int, Wh: int, *, inverse: bool
     if dst is not None:
         _shape(dst, src.shape, "dst")
     _dev_tensor(src, torch.bfloat16, "src")
+    if dst is not None:
+        _dev_tensor(dst, torch.bfloat16, "dst")
     N, d = src.shape[-2:]
     S = src.numel() // (N * d)
     dst = torch.empty_like(src) if dst is None else dst
@@ -344,6 +363,10 @@ def sparse_attn(q, k, v, mode: str = "topk", *, topk: int = 0, idx=None, window:
         _shape(idx, (B, H, (N + block - 1) // block, int(topk)), "idx")
     for n, t in (("q", q), ("k", k), ("v", v)):
         _dev_tensor(t, torch.bfloat16, n)
+    if o is not None:
+        _dev_tensor(o, torch.bfloat16, "o")
+    if mode == "topk" and idx is not None:
+        _dev_tensor(idx, torch.int32, "idx")
     m = _MODES[mode]
     flags, fptr = _flags(space_major_heads, H)
     o = torch.empty_like(q) if o is None else o
@@ -365,6 +388,8 @@ def dense_attn(q, k, v, *, o=None, stream=None):
         _shape(o, q.shape, "o")
     for n, t in (("q", q), ("k", k), ("v", v)):
         _dev_tensor(t, torch.bfloat16, n)
+    if o is not None:
+        _dev_tensor(o, torch.bfloat16, "o")
     B, H, N, d = q.shape
     o = torch.empty_like(q) if o is None else o
     _check(lib.salad_dense_attn(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(o), _stream(stream)),
@@ -416,6 +441,10 @@ class ForwardPlan:
                      ("w_lin", w_lin), ("w_lin_full", w_lin_full), ("w_out", w_out)):
             if t is not None or n in ("q", "k", "v", "x", "w_gate"):
                 _dev_tensor(t, torch.bfloat16, n)
+        for n, t, dt in (("o", o, torch.bfloat16), ("out", out, torch.bfloat16),
+                         ("s_out", s_out, torch.float32), ("idx_out", idx_out, torch.int32)):
+            if t is not None:
+                _dev_tensor(t, dt, n)
         self.tensors = dict(q=q, k=k, v=v, x=x, w_gate=w_gate, w_lin=w_lin,
                             w_lin_full=w_lin_full, w_out=w_out)
         # Output projection (optional): out [B,N,d_out] = cat_heads(O) w_out.

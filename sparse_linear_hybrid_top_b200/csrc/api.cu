@@ -27,31 +27,62 @@ struct DevInfo {
   bool supported = false;
   int num_sms = 0;
   unsigned* err = nullptr;
-  // salad_forward's side streams and fork/join events (created on first use).
-  bool side_ready = false;
-  cudaStream_t side[2] = {nullptr, nullptr};
-  cudaEvent_t fork = nullptr, join_gate = nullptr, join_lin = nullptr;
-  std::mutex enqueue_mu;      // one forward at a time records and waits on the events
 };
 DevInfo g_dev[kMaxDevices];
 std::mutex g_mu;
 
-// The side streams and events of the current device, created once.
-DevInfo* side_resources() {
+// salad_forward's side streams and fork/join events, one set per caller
+// stream (created on first use, kept until the process exits).  Calls on
+// different caller streams use different sets, so they neither wait for each
+// other on the host nor gain false dependencies on the GPU, and a stream being
+// captured into a CUDA graph never shares a side stream with another caller.
+// Calls on the same caller stream are ordered anyway; the set's mutex keeps
+// their fork/join records from interleaving.
+struct SideSet {
+  cudaStream_t caller = nullptr;
+  cudaStream_t side[2] = {nullptr, nullptr};
+  cudaEvent_t fork = nullptr, join_gate = nullptr, join_lin = nullptr;
+  std::mutex enqueue_mu;
+};
+constexpr int kMaxSideSets = 32;   // per device; beyond this a call runs on one stream
+struct SideTable {
+  SideSet sets[kMaxSideSets];
+  int used = 0;
+};
+SideTable g_side[kMaxDevices];
+
+// The side set of `caller` on the current device, or null when the table is
+// full (the call then enqueues every step on the caller's stream, in order).
+// A CUDA failure while creating a set is reported through *cuda_failed.
+SideSet* side_resources(cudaStream_t caller, bool* cuda_failed) {
+  *cuda_failed = false;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_mu);
-  DevInfo& d = g_dev[dev];
-  if (!d.side_ready) {
-    for (int i = 0; i < 2; ++i)
-      if (cudaStreamCreateWithFlags(&d.side[i], cudaStreamNonBlocking) != cudaSuccess)
-        return nullptr;
-    if (cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&d.join_gate, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&d.join_lin, cudaEventDisableTiming) != cudaSuccess)
-      return nullptr;
-    d.side_ready = true;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *cuda_failed = true;
+    return nullptr;
   }
+  std::lock_guard<std::mutex> lock(g_mu);
+  SideTable& t = g_side[dev];
+  for (int i = 0; i < t.used; ++i)
+    if (t.sets[i].caller == caller) return &t.sets[i];
+  if (t.used == kMaxSideSets) return nullptr;
+  SideSet& d = t.sets[t.used];
+  bool ok = true;
+  for (int i = 0; i < 2 && ok; ++i)
+    ok = cudaStreamCreateWithFlags(&d.side[i], cudaStreamNonBlocking) == cudaSuccess;
+  ok = ok && cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming) == cudaSuccess &&
+       cudaEventCreateWithFlags(&d.join_gate, cudaEventDisableTiming) == cudaSuccess &&
+       cudaEventCreateWithFlags(&d.join_lin, cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    for (cudaStream_t& x : d.side)
+      if (x != nullptr) { cudaStreamDestroy(x); x = nullptr; }
+    for (cudaEvent_t* e : {&d.fork, &d.join_gate, &d.join_lin})
+      if (*e != nullptr) { cudaEventDestroy(*e); *e = nullptr; }
+    *cuda_failed = true;
+    return nullptr;
+  }
+  d.caller = caller;
+  ++t.used;
   return &d;
 }
 
@@ -251,7 +282,7 @@ const char* salad_status_string(salad_status s) {
   }
 }
 
-int salad_version(void) { return 400; }
+int salad_version(void) { return 40100; }
 
 // ------------------------------------------------------------------ gate --
 size_t salad_gate_workspace_bytes(int B, int N, int D) {
@@ -523,11 +554,14 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   Ctx c;
   if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
 
-  DevInfo* dv = side_resources();
-  if (dv == nullptr) return SALAD_ERR_CUDA;
-  // Fork/join on per-device events: enqueues of concurrent calls must not
-  // interleave.
-  std::lock_guard<std::mutex> enqueue_lock(dv->enqueue_mu);
+  bool side_failed = false;
+  SideSet* dv = side_resources(c.stream, &side_failed);
+  if (side_failed) return SALAD_ERR_CUDA;
+  // Fork/join on this caller stream's events: enqueues of concurrent calls on
+  // the same caller stream must not interleave.  Without a side set (table
+  // full) there is nothing to fork: every step goes on the caller's stream.
+  std::unique_lock<std::mutex> enqueue_lock;
+  if (dv != nullptr) enqueue_lock = std::unique_lock<std::mutex>(dv->enqueue_mu);
 
   char* ws = static_cast<char*>(a->workspace);
   const int B = a->B, H = a->H, N = a->N, d = a->d;
@@ -537,16 +571,18 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   // it; the attention waits for both.  The side chains are joined back even
   // when a launch fails, so the caller's stream never runs ahead of them.
   Ctx cg = c, cl = c;
-  cg.stream = dv->side[0];
-  cl.stream = dv->side[1];
+  if (dv != nullptr) {
+    cg.stream = dv->side[0];
+    cl.stream = dv->side[1];
+  }
   auto mark = [&](int i, cudaStream_t st) -> bool {
     if (a->phase_events == nullptr || a->phase_events[i] == nullptr) return true;
     return cudaEventRecord(static_cast<cudaEvent_t>(a->phase_events[i]), st) == cudaSuccess;
   };
   if (!mark(0, c.stream)) return SALAD_ERR_CUDA;
-  if (cudaEventRecord(dv->fork, c.stream) != cudaSuccess ||
-      cudaStreamWaitEvent(cg.stream, dv->fork, 0) != cudaSuccess ||
-      cudaStreamWaitEvent(cl.stream, dv->fork, 0) != cudaSuccess)
+  if (dv != nullptr && (cudaEventRecord(dv->fork, c.stream) != cudaSuccess ||
+                        cudaStreamWaitEvent(cg.stream, dv->fork, 0) != cudaSuccess ||
+                        cudaStreamWaitEvent(cl.stream, dv->fork, 0) != cudaSuccess))
     return SALAD_ERR_CUDA;
   bool ok = true;
   auto check = [&](cudaError_t e) { ok = ok && e == cudaSuccess; };
@@ -556,7 +592,7 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   if (override_gate) check(launch_fill_f32(cg, s, a->gate_override, B));
   else check(launch_gate(cg, a->x, a->w_gate, a->gate_bias, B, N, a->D, s, ws + L.gate));
   ok = ok && mark(1, cg.stream);
-  check(cudaEventRecord(dv->join_gate, cg.stream));
+  if (dv != nullptr) check(cudaEventRecord(dv->join_gate, cg.stream));
 
   AttnArgs at;
   std::memset(&at, 0, sizeof(at));
@@ -578,7 +614,7 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   BranchDrop drop;   // default: never drop, reads nothing
   if (at.drop > 0.0f) {
     // Only here does this chain read s: it waits for the gate first.
-    check(cudaStreamWaitEvent(cl.stream, dv->join_gate, 0));
+    if (dv != nullptr) check(cudaStreamWaitEvent(cl.stream, dv->join_gate, 0));
     drop.s = s;
     drop.thr = at.drop;
   }
@@ -600,7 +636,7 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
                                 drop, rope));
     if (ok) check(launch_linear_apply(cl, a->q, Hst, Z, a->eps, B, H, N, d, olin, rope));
   }
-  check(cudaEventRecord(dv->join_lin, cl.stream));
+  if (dv != nullptr) check(cudaEventRecord(dv->join_lin, cl.stream));
 
   // 2. sparse-branch pattern (ijyty.com 1.1 / 1.2), the caller's stream
   if (a->mode == SALAD_MODE_TOPK) {
@@ -636,8 +672,9 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
 
   // Join the side chains, then 4. sparse attention with the gated residual
   // epilogue (steps 2, 6).
-  const bool joined = cudaStreamWaitEvent(c.stream, dv->join_gate, 0) == cudaSuccess &&
-                      cudaStreamWaitEvent(c.stream, dv->join_lin, 0) == cudaSuccess;
+  const bool joined = dv == nullptr ||
+                      (cudaStreamWaitEvent(c.stream, dv->join_gate, 0) == cudaSuccess &&
+                       cudaStreamWaitEvent(c.stream, dv->join_lin, 0) == cudaSuccess);
   if (!ok || !joined || !mark(3, c.stream)) return SALAD_ERR_CUDA;
   if (launch_attention(c, at) != cudaSuccess || !mark(4, c.stream)) return SALAD_ERR_CUDA;
 

@@ -167,13 +167,19 @@ size_t gate_ws_bytes(int B, int N, int D) {
   return align256(static_cast<size_t>(B) * parts * sizeof(float));
 }
 
-cudaError_t launch_gate(const Ctx& c, const void* x, const void* w, float bias, int B, int N,
-                        int D, float* s, void* ws) {
+// Enqueues the partial-sum kernel and the final kernel with the partial sums
+// in `partial`.  At most `max_parts_total` partials (B x parts) are used: the
+// regular gate passes its workspace's capacity, which its partition never
+// exceeds, so the cap only binds for the fixed array of the allocation-free
+// variant.
+cudaError_t launch_gate_parts(const Ctx& c, const void* x, const void* w, float bias, int B,
+                              int N, int D, float* s, float* partial, long long max_parts_total) {
   const int sms = c.num_sms < 256 ? c.num_sms : 256;
-  float* partial = static_cast<float*>(ws);
+  const long long cap = max_parts_total / B > 0 ? max_parts_total / B : 1;
   int nparts;
   if (gate_rows_ok(D)) {
     nparts = gate_rows_parts(B, N, D, sms);
+    if (nparts > cap) nparts = static_cast<int>(cap);
     // Whole unrolled groups per CTA; no empty CTA.
     const int rows_per = ((N + nparts - 1) / nparts + kGateRowUnroll - 1) / kGateRowUnroll * kGateRowUnroll;
     nparts = (N + rows_per - 1) / rows_per;
@@ -181,12 +187,19 @@ cudaError_t launch_gate(const Ctx& c, const void* x, const void* w, float bias, 
         static_cast<const uint4*>(x), static_cast<const uint4*>(w), N, rows_per, partial);
   } else {
     nparts = gate_ctas_per_b(B, N, D, sms);
+    if (nparts > cap) nparts = static_cast<int>(cap);
     const long long chunks_per_b = static_cast<long long>(N) * (D / 8);
     gate_partial_kernel<<<dim3(nparts, B), kGateThreads, 0, c.stream>>>(
         static_cast<const uint4*>(x), static_cast<const uint4*>(w), chunks_per_b, D / 8, partial);
   }
   gate_final_kernel<<<B, 256, 0, c.stream>>>(partial, nparts, N, bias, s);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gate(const Ctx& c, const void* x, const void* w, float bias, int B, int N,
+                        int D, float* s, void* ws) {
+  return launch_gate_parts(c, x, w, bias, B, N, D, s, static_cast<float*>(ws),
+                           static_cast<long long>(gate_ws_bytes(B, N, D) / sizeof(float)));
 }
 
 cudaError_t launch_fill_f32(const Ctx& c, float* dst, float value, int n) {
@@ -214,8 +227,8 @@ namespace salad {
 namespace {
 
 constexpr int kNoAllocMaxBatch = 256;        // largest B the array serves
-constexpr int kNoAllocPartsPerSample = 64;   // partial sums kept per sample
-constexpr int kNoAllocFloats = kNoAllocMaxBatch * kNoAllocPartsPerSample;
+constexpr int kNoAllocFloats = 16384;        // partial sums the array holds (64 KB)
+static_assert(kNoAllocFloats / kNoAllocMaxBatch >= 64, "at least 64 partial sums per sample");
 
 static __device__ __align__(256) float g_gate_scratch[kNoAllocFloats];
 
@@ -272,15 +285,17 @@ extern "C" salad_status salad_gate_noalloc(const void* x, const void* w, float b
   NoAllocDev* d = nullptr;
   const salad_status st = noalloc_setup(dev, &d);
   if (st != SALAD_OK) return st;
-  int nparts = gate_ctas_per_b(B, N, D, d->num_sms < 256 ? d->num_sms : 256);
-  if (nparts > kNoAllocPartsPerSample) nparts = kNoAllocPartsPerSample;
-  // Every partial slot read by the final kernel is written first by this
+  // The same partition as salad_gate whenever its B x parts partial sums fit
+  // the array (then the result is bit-identical); otherwise fewer parts per
+  // sample, which changes only the float32 rounding of the partial sums.
+  // Every partial slot the final kernel reads is written first by this
   // call's partial kernel, so nothing needs clearing between calls.
-  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const long long chunks_per_b = static_cast<long long>(N) * (D / 8);
-  gate_partial_kernel<<<dim3(nparts, B), kGateThreads, 0, cs>>>(
-      static_cast<const uint4*>(x), static_cast<const uint4*>(w), chunks_per_b, D / 8,
-      d->scratch);
-  gate_final_kernel<<<B, 256, 0, cs>>>(d->scratch, nparts, N, bias, s);
-  return cudaGetLastError() == cudaSuccess ? SALAD_OK : SALAD_ERR_CUDA;
+  Ctx c;
+  c.stream = static_cast<cudaStream_t>(stream);
+  c.err = nullptr;
+  c.num_sms = d->num_sms;
+  c.wait_ns = 0;
+  if (launch_gate_parts(c, x, w, bias, B, N, D, s, d->scratch, kNoAllocFloats) != cudaSuccess)
+    return SALAD_ERR_CUDA;
+  return SALAD_OK;
 }

@@ -34,7 +34,7 @@ def test_header_declarations_match_binding_and_exports():
 def test_library_is_built_for_sm100a_only():
     # The binding loads the in-tree library (no fallback path exists).
     assert os.path.dirname(salad.LIB_PATH) == os.path.join(ROOT, "sparse_linear_hybrid_top_b200")
-    assert salad.version() == 400
+    assert salad.version() == 40100
 
 
 def test_status_strings():

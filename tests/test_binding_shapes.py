@@ -115,3 +115,49 @@ def test_piecewise_calls_shapes():
                                                   idx=idx[:, :, :-1]), "idx")
     _expect_shape_error(lambda: salad.sparse_attn(q, k, v[:, :1], "swa", window=8), "v")
     _expect_shape_error(lambda: salad.dense_attn(q, k, v, o=q[:, :, :-1]), "o")
+
+
+@pytest.mark.gpu
+def test_outputs_checked_like_inputs():
+    # Device inputs with a caller-supplied output on the host, of the wrong
+    # dtype or not contiguous: every call refuses before any launch (a host
+    # pointer handed to a kernel would fault; a wrong dtype would be misread).
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    w = WORKLOADS["tiny"]
+    inp = {k: (t.cuda() if isinstance(t, torch.Tensor) else t) for k, t in generate(w).items()}
+    q, k, v, x, wg = inp["q"], inp["k"], inp["v"], inp["x"], inp["w_gate"]
+    B, H, N, d = q.shape
+    nb = w.nb
+    bad_s = [torch.zeros(B), torch.zeros(B, dtype=torch.float64, device="cuda"),
+             torch.zeros(2 * B, device="cuda")[::2]]
+    for s in bad_s:
+        with pytest.raises(ValueError, match="s must|s is on"):
+            salad.gate(x, wg, 0.0, s=s)
+        with pytest.raises(ValueError, match="s must|s is on"):
+            salad.gate_noalloc(x, wg, 0.0, s=s)
+    for idx in (torch.zeros(B, H, nb, 2, dtype=torch.int32),
+                torch.zeros(B, H, nb, 2, dtype=torch.int64, device="cuda")):
+        with pytest.raises(ValueError, match="idx must"):
+            salad.select_blocks(q, k, 2, idx=idx)
+        with pytest.raises(ValueError, match="idx must"):
+            salad.sparse_attn(q, k, v, "topk", topk=2, idx=idx)
+    for o in (torch.empty_like(q, device="cpu"), torch.empty(q.shape, device="cuda")):
+        with pytest.raises(ValueError, match="o must"):
+            salad.dense_attn(q, k, v, o=o)
+        with pytest.raises(ValueError, match="o must"):
+            salad.sparse_attn(q, k, v, "swa", window=8, o=o)
+        with pytest.raises(ValueError, match="o must"):
+            salad.linear_apply(q, torch.zeros(B, H, d, d, device="cuda"),
+                               torch.zeros(B, H, d, device="cuda"), o=o)
+        with pytest.raises(ValueError, match="o must"):
+            _plan(w, inp, o=o)
+    with pytest.raises(ValueError, match="dst must"):
+        salad.permute_tokens(q.reshape(-1, N, d), w.F, w.Hh, w.Wh,
+                             dst=torch.empty(B * H, N, d, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="s_out must"):
+        _plan(w, inp, s_out=torch.zeros(B))
+    with pytest.raises(ValueError, match="idx_out must"):
+        _plan(w, inp, idx_out=torch.zeros(B, H, nb, w.topk, dtype=torch.int64, device="cuda"))
+    with pytest.raises(ValueError, match="workspace must"):
+        salad.gate(x, wg, 0.0, workspace=torch.zeros(1 << 20, dtype=torch.uint8))

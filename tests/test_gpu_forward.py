@@ -178,11 +178,16 @@ def test_forward_is_deterministic(salad):
 
 
 # ------------------------------------------------------------ full sizes ---
-def _oracle_rows(w, inp, b, h, rows_in_order, idx_row_of, s_b, lin_cache):
-    """Oracle output rows of one head, rows given in the head's attention order."""
+def _oracle_rows(w, inp, b, h, rows_in_order, idx_row_of, s_b, lin_cache, angles=None,
+                 dropped=False):
+    """Oracle output rows of one head, rows given in the head's attention order.
+
+    ``angles``: the 3-D rotary encoding of the linear branch (per frame-major
+    token); ``dropped``: the sample's linear branch is pruned (O = O_sparse).
+    """
     q, k, v = (to64(inp[n][b, h]) for n in ("q", "k", "v"))
     if (b, h) not in lin_cache:
-        lin_cache[(b, h)] = oracle.linear_state(k, v)
+        lin_cache[(b, h)] = oracle.linear_state(k, v, angles)
     Hst, Z = lin_cache[(b, h)]
     if w.mode == "topk":
         blocks = sorted(set(int(r) // w.block for r in rows_in_order))
@@ -197,20 +202,35 @@ def _oracle_rows(w, inp, b, h, rows_in_order, idx_row_of, s_b, lin_cache):
         rows = np.asarray(rows_in_order)
         o_s = oracle.swa_attention_rows(qo, ko, vo, w.window, rows)
         tok = perm[rows]
-    o_l = oracle.linear_apply(q[tok], Hst, Z, w.eps)
+    if dropped:
+        return tok, o_s
+    o_l = oracle.linear_apply(q[tok], Hst, Z, w.eps, None if angles is None else angles[tok])
     o = oracle.combine(o_s, o_l, to64(inp["w_lin"][h]), s_b)
     return tok, o
 
 
-def _sampled_check(salad, w, n_samples, seed=0, full=False):
-    inp = generate(w)
+def _sampled_check(salad, w, n_samples, seed=0, full=False, rope3d=False, drop_threshold=0.0,
+                   inp=None):
+    """The forward pass at full size, in the launch configuration the
+    benchmark times, compared with the oracle on seeded query blocks (plus the
+    ragged last block) or on every output."""
+    inp = generate(w) if inp is None else inp
     dev = device_inputs(inp)
-    plan = _plan(salad, w, dev)
+    kw = {}
+    if rope3d:
+        kw["rope3d"] = True
+        if w.mode != "swa":
+            kw.update(F=w.F, Hh=w.Hh, Wh=w.Wh)
+    if drop_threshold:
+        kw["drop_threshold"] = drop_threshold
+    plan = _plan(salad, w, dev, **kw)
     o = plan.run()
     torch.cuda.synchronize()
     salad.check_error()
     s_ref = oracle.gate(inp["x"], inp["w_gate"], inp["bias"])
     np.testing.assert_allclose(to64(plan.s_out), s_ref, rtol=0, atol=1e-5)
+    dropped = s_ref < drop_threshold
+    angles = oracle.rope3d_angles(w.N, w.d, w.F, w.Hh, w.Wh) if rope3d else None
     idx = _selection_used(w, inp, plan.idx_out) if w.mode == "topk" else None
     o_cpu = o.cpu()
     rng = np.random.default_rng(seed)
@@ -229,7 +249,7 @@ def _sampled_check(salad, w, n_samples, seed=0, full=False):
         rows = np.concatenate([np.arange(i * w.block, min(w.N, (i + 1) * w.block))
                                for i in sorted(blocks)])
         tok, want = _oracle_rows(w, inp, b, h, rows, None if idx is None else idx[b, h],
-                                 s_ref[b], lin_cache)
+                                 s_ref[b], lin_cache, angles, bool(dropped[b]))
         got_all.append(o_cpu[b, h, torch.from_numpy(tok)])
         want_all.append(want)
     got = torch.cat(got_all)
@@ -249,6 +269,96 @@ def test_forward_topk720_sampled(salad):
     _sampled_check(salad, WORKLOADS["topk720"], 64, seed=2)
 
 
+# The optional parts of the layer at the size the benchmark times them: the
+# 3-D rotary encoding of the linear branch ("SALAD ... (paper.rainbus.top)"
+# 方法步骤详情 step 3) and post-training branch dropping (step 8; a threshold
+# above every gate value prunes every sample's linear branch, as the
+# benchmark's branch-dropped variant does).
+@pytest.fixture(scope="module")
+def inp480():
+    return generate(WORKLOADS["topk480"])
+
+
+def test_forward_topk480_rope3d_sampled(salad, inp480):
+    _sampled_check(salad, WORKLOADS["topk480"], 96, seed=4, rope3d=True, inp=inp480)
+
+
+def test_forward_topk480_branch_dropped_sampled(salad, inp480):
+    _sampled_check(salad, WORKLOADS["topk480"], 96, seed=5, drop_threshold=1.0, inp=inp480)
+
+
+def test_forward_topk480_branch_kept_below_threshold_sampled(salad, inp480):
+    # A threshold below the sample's gate value keeps the branch.
+    s = float(oracle.gate(inp480["x"], inp480["w_gate"], inp480["bias"])[0])
+    _sampled_check(salad, WORKLOADS["topk480"], 32, seed=6, drop_threshold=0.5 * s, inp=inp480)
+
+
+def test_forward_swa480_rope3d_sampled(salad):
+    _sampled_check(salad, WORKLOADS["swa480"], 96, seed=7, rope3d=True)
+
+
 @pytest.mark.parametrize("name", ["cfg_b2h40_s80", "cfg_b2h40_s95", "cfg_b2h40_all"])
 def test_forward_b2h40_sampled(salad, name):
     _sampled_check(salad, WORKLOADS[name], 48, seed=3)
+
+
+# ------------------------------------------------------------ reentrancy ---
+def test_forward_on_two_streams_at_once(salad):
+    # Two independent layers enqueued on two caller streams, back to back, so
+    # their kernels may overlap on the GPU: each caller stream has its own
+    # side streams and fork/join events, and each output must match the
+    # oracle for its own inputs.
+    wa = RAGGED128
+    wb = dataclasses.replace(RAGGED128, name="ragged128_seed9", seeds=(9,))
+    inps = [generate(wa), generate(wb)]
+    devs = [device_inputs(i) for i in inps]
+    plans = [_plan(salad, w, d) for w, d in zip((wa, wb), devs)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for p, st in zip(plans, streams):
+            p.run(st)
+    torch.cuda.synchronize()
+    salad.check_error()
+    for w, inp, p in zip((wa, wb), inps, plans):
+        ref = oracle.forward(inp, mode="topk", block=w.block, topk=w.topk, eps=w.eps,
+                             idx_override=_selection_used(w, inp, p.idx_out))
+        assert_close(p.o, ref["o"], f"forward on its own stream ({w.name})")
+
+
+def test_forward_from_two_host_threads(salad):
+    # Two host threads, each driving its own plan on its own stream many
+    # times: the enqueues run concurrently (the binding releases the GIL in
+    # the C call) and every result equals the single-threaded one bit for bit.
+    import threading
+    ws = [RAGGED128, dataclasses.replace(RAGGED128, name="ragged128_seed9", seeds=(9,))]
+    devs = [device_inputs(generate(w)) for w in ws]
+    plans = [_plan(salad, w, d) for w, d in zip(ws, devs)]
+    want = [p.run().clone() for p in plans]
+    torch.cuda.synchronize()
+    outs = [[], []]
+    errors = []
+
+    def drive(i):
+        try:
+            st = torch.cuda.Stream()
+            with torch.cuda.stream(st):
+                for _ in range(20):
+                    plans[i].run(st)
+                    outs[i].append(plans[i].o.clone())
+            st.synchronize()
+        except Exception as e:  # surfaced below
+            errors.append(e)
+
+    threads = [threading.Thread(target=drive, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    torch.cuda.synchronize()
+    salad.check_error()
+    assert not errors, errors
+    for i in range(2):
+        assert len(outs[i]) == 20
+        for o in outs[i]:
+            assert torch.equal(o, want[i])

@@ -5,14 +5,19 @@ only its input and output buffers, or code running where an allocator call is
 not permitted -- so they cannot provide the workspace salad_gate needs.  The
 no-allocation variant keeps its partial sums in a fixed array inside the
 library.  This test calls it through the C ABI twice in a row, on different
-inputs, and checks each result against salad_gate within the gate tests'
-tolerance (1e-5 absolute on s).  It also checks that a batch larger than the
-array serves is refused before any launch.
+inputs, and checks each result against salad_gate and against the float64
+oracle within the gate tests' tolerance (1e-5 absolute on s); on a 148-SM
+B200 the two CUDA gates share one partition, so they must agree bit for bit.
+It also checks that a batch larger than the array serves is refused before
+any launch.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
+
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -49,12 +54,16 @@ def test_noalloc_gate_matches_gate_on_two_calls_in_a_row(salad):
         x, w = _inputs(B, N, D, seed)
         s_new = _noalloc(salad, x, w, bias)
         s_ref = salad.gate(x, w, bias)
-        outs.append((s_new, s_ref))
+        outs.append((s_new, s_ref, oracle.gate(x.cpu(), w.cpu(), bias)))
     torch.cuda.synchronize()
     salad.check_error()
-    for s_new, s_ref in outs:
+    same_partition = torch.cuda.get_device_properties(0).multi_processor_count == 148
+    for s_new, s_ref, s_oracle in outs:
         assert torch.isfinite(s_new).all()
         torch.testing.assert_close(s_new, s_ref, rtol=0, atol=1e-5)
+        np.testing.assert_allclose(s_new.cpu().double().numpy(), s_oracle, rtol=0, atol=1e-5)
+        if same_partition:
+            assert torch.equal(s_new, s_ref)
 
 
 def test_noalloc_gate_refuses_batches_beyond_its_array(salad):

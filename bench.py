@@ -101,10 +101,10 @@ def choose_peak(peaks: dict, timed_ms: float, clk: dict):
 
 
 def launches_per_step(w) -> int:
-    # gate (2) + [pool, score, topk, pair_union | gather] + linear state and
-    # reduce+fold (2) + attention (1)
+    # gate (2) + [pool, fused select | gather] + linear state and reduce+fold
+    # (2) + attention (1)
     if w.mode == "topk":
-        return 2 + 4 + 2 + 1
+        return 2 + 2 + 2 + 1
     if w.mode == "swa":
         return 2 + (1 if w.space_major_heads else 0) + 2 + 1
     return 2 + 2 + 1
@@ -291,6 +291,82 @@ def cpu_threads() -> int:
     except Exception:
         pass
     return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------- sweep ---
+SWEEP = ("swa480", "topk720", "cfg_b2h40_s80", "cfg_b2h40_s90", "cfg_b2h40_s95", "cfg_b2h40_all")
+
+
+def run_sweep(names, device, stream, peaks, steps: int = 5, warmup: int = 2) -> dict:
+    """The other workloads of the method's video shapes, each timed like the
+    headline (one salad_forward per step, CUDA events on the launch stream)
+    next to the same library's dense attention on the same Q, K, V.  Inputs
+    are drawn on the device with the synthetic recipe (``generate_device``:
+    same distributions and frame structure, not the host generator's bytes,
+    whose draws take minutes at these sizes)."""
+    import torch
+    import sparse_linear_hybrid_top_b200 as salad
+    from synth import WORKLOADS, generate_device
+    out = {}
+    burst = float(peaks["bf16_tflops"])
+    sustained = float(peaks.get("bf16_tflops_sustained") or burst)
+    for name in names:
+        w = WORKLOADS[name]
+        dev = generate_device(w, device, seed=w.seeds[0])
+        extra = {}
+        if w.mode == "swa":
+            extra = dict(window=w.window, space_major_heads=w.space_major_heads, F=w.F,
+                         Hh=w.Hh, Wh=w.Wh)
+        plan = salad.ForwardPlan(dev["q"], dev["k"], dev["v"], dev["x"], dev["w_gate"],
+                                 dev["w_lin"], mode=w.mode, topk=w.topk, bias=w.bias, eps=w.eps,
+                                 **extra)
+        for _ in range(warmup):
+            plan.run(stream)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for e5 in ev:
+            for e in e5:
+                e.record(stream)
+        torch.cuda.synchronize(device)
+        t0.record(stream)
+        for i in range(steps):
+            plan.set_phase_events(ev[i])
+            plan.run(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+        plan.set_phase_events(None)
+        salad.check_error(stream)
+        ms = t0.elapsed_time(t1) / steps
+        attn = statistics.fmean(e5[3].elapsed_time(e5[4]) for e5 in ev)
+        pre = statistics.fmean(e5[0].elapsed_time(e5[3]) for e5 in ev)
+        salad.dense_attn(dev["q"], dev["k"], dev["v"], stream=stream)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nd = 2
+        d0.record(stream)
+        for _ in range(nd):
+            salad.dense_attn(dev["q"], dev["k"], dev["v"], stream=stream)
+        d1.record(stream)
+        torch.cuda.synchronize(device)
+        dense_ms = d0.elapsed_time(d1) / nd
+        fl = step_flops(w)
+        ach = fl["attn_kernel"] / (attn * 1e-3) / 1e12
+        out[name] = {
+            "B": w.B, "H": w.H, "N": w.N, "mode": w.mode, "topk": w.topk, "window": w.window,
+            "sparsity": round(1 - fl["sparse"] / fl["dense"], 4),
+            "ms_per_layer": round(ms, 4),
+            "value": round(fl["total"] / (ms * 1e-3) / 1e12, 2),
+            "phases_ms": {"pre_attention": round(pre, 4), "attention": round(attn, 4)},
+            "attention_tflops": round(ach, 1),
+            "attention_frac_of_burst": round(ach / burst, 4),
+            "attention_frac_of_sustained": round(ach / sustained, 4),
+            "dense_ms": round(dense_ms, 3),
+            "dense_tflops": round(fl["dense"] / (dense_ms * 1e-3) / 1e12, 1),
+            "speedup_vs_dense": round(dense_ms / ms, 3),
+            "attention_speedup_vs_dense": round(dense_ms / attn, 3),
+        }
+        del plan, dev
+        torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------------------ runs ---
@@ -532,6 +608,10 @@ def run_ours(args, w) -> int:
         "gpu_launches": launches_per_step(w) * args.steps,
         "clocks": clk,
     }
+    if world == 1 and not args.no_sweep:
+        # Timed after the headline line's numbers were taken.
+        line["workloads"] = run_sweep([n for n in SWEEP if n != w.name], device, stream, peaks)
+        line["workloads_inputs"] = "device-drawn with the synthetic recipe (synth.generate_device)"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         del dev
         flops, secs = cpu_sample_work(w, host, n_heads=args.cpu_heads, blocks_per_head=args.cpu_blocks)
@@ -591,6 +671,8 @@ def main(argv=None) -> int:
     ap.add_argument("--cpu-blocks", type=int, default=488, help="query blocks per head in cpu_baseline")
     ap.add_argument("--ref-blocks", type=int, default=16, help="query blocks per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the other workloads (ST-SWA 480p, 720p, B=2 H=40 sparsity sweep)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

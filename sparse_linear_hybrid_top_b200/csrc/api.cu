@@ -643,8 +643,8 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
     int32_t* idx = a->idx_out != nullptr ? a->idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
     int32_t* lists = reinterpret_cast<int32_t*>(ws + L.lists);
     int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
-    if (ok) check(launch_select(c, a->q, a->k, B, H, N, d, a->topk, idx, ws + L.sel));
-    if (ok) check(launch_pair_union(c, idx, B * H, nb, a->topk, lists, counts));
+    if (ok) check(launch_select(c, a->q, a->k, B, H, N, d, a->topk, idx, ws + L.sel, lists,
+                                counts));
     at.mode = kModeTopk;
     at.lists = lists;
     at.counts = counts;

@@ -8,13 +8,16 @@
 // block index.
 //
 // Precision: block sums of bf16 values are formed in float64 (exact for bf16
-// inputs in any realistic range), divided by the row count, and the scores
-// are float64 dot products, so the kept set is decided in float64.
+// inputs in any realistic range) and divided by the row count; the kept set
+// is the one float64 dot products of these means decide.  The scores are
+// formed in float32 with a certified error bound, and only the blocks the
+// bound leaves undecided are scored again in float64 (select_fused_kernel).
 //
-// Kernels: pool (HBM-bound: reads Q and K once), score (small float64 GEMM
-// per head, nb x nb x d), topk (one warp per query block: radix select on
-// order-preserving 64-bit keys, then an ordered compaction), pair_union
-// (one warp per pair of query blocks: bitmap merge of the two kept lists).
+// Kernels: pool (HBM-bound: reads Q and K once), select_fused (per chunk of
+// query blocks of a head: float32 scores in shared memory, a radix select,
+// the float64 recheck, the ascending kept lists and the union of each pair
+// of query blocks' lists for the attention kernel), pair_union (the same
+// union for caller-supplied lists).
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,11 +27,16 @@ namespace {
 constexpr int kBlock = 64;
 
 // ------------------------------------------------------------------ pool --
+// CTA (i, bh, z): the mean of block i of head bh of Q (z = 0) or K (z = 1),
+// summed in float64 over the valid rows, written in float64 and rounded once
+// to float32 (the selection's float32 pass reads the latter).
 template <int D>
 __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
                                                    const uint4* __restrict__ k, int N, int nb,
                                                    double* __restrict__ qbar,
-                                                   double* __restrict__ kbar) {
+                                                   double* __restrict__ kbar,
+                                                   float* __restrict__ qbar32,
+                                                   float* __restrict__ kbar32) {
   constexpr int CPR = D / 8;     // 16-byte chunks per row
   constexpr int RPI = 128 / CPR; // rows per iteration
   __shared__ double red[RPI][D];
@@ -36,6 +44,7 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
   const long long bh = blockIdx.y;
   const uint4* src = blockIdx.z == 0 ? q : k;
   double* dst = blockIdx.z == 0 ? qbar : kbar;
+  float* dst32 = blockIdx.z == 0 ? qbar32 : kbar32;
   const int row0 = i * kBlock;
   const int rows = min(kBlock, N - row0);
   const int chunk = threadIdx.x % CPR;
@@ -62,153 +71,125 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
     double s = 0.0;
 #pragma unroll
     for (int r = 0; r < RPI; ++r) s += red[r][c];
-    dst[(bh * nb + i) * D + c] = s / static_cast<double>(rows);
+    const double m = s / static_cast<double>(rows);
+    dst[(bh * nb + i) * D + c] = m;
+    dst32[(bh * nb + i) * D + c] = static_cast<float>(m);
   }
 }
 
-// ----------------------------------------------------------------- score --
-// S[bh][i][j] = sum_c qbar[bh][i][c] * kbar[bh][j][c] in float64, each sum
-// taken in ascending c.  64 x 64 tile per CTA of 128 threads, 8 (rows) x 4
-// (columns) outputs per thread: rows 2*ty + {0,1} + 16a, columns 2*tx +
-// {0,1} + 32b, so each 16-byte shared load of a half-warp covers contiguous
-// banks.  The c dimension is staged 16 at a time through two shared buffers;
-// the next chunk is read from global memory into registers while the current
-// one is multiplied.
-constexpr int kST = 64;    // tile edge
-constexpr int kSK = 16;    // c-chunk staged per step
-constexpr int kSPad = 2;   // row padding (keeps 16-byte alignment, spreads banks)
-__global__ void __launch_bounds__(128, 4) score_kernel(const double* __restrict__ qbar,
-                                                    const double* __restrict__ kbar, int nb,
-                                                    int D, double* __restrict__ S) {
-  __shared__ __align__(16) double qs[2][kSK][kST + kSPad];
-  __shared__ __align__(16) double ks[2][kSK][kST + kSPad];
-  const long long bh = blockIdx.z;
-  const int i0 = blockIdx.y * kST, j0 = blockIdx.x * kST;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  const double* qb = qbar + bh * nb * D;
-  const double* kb = kbar + bh * nb * D;
-  // Staging: thread t moves elements (row t/8 + 16v, c-pair t%8) of each
-  // operand, v = 0..3: 16-byte reads, 128 bytes per row.
-  const int sr = threadIdx.x / 8, sc = 2 * (threadIdx.x % 8);
-  double2 gq[4], gk[4];
-  auto fetch = [&](int c0) {
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int r = sr + 16 * v;
-      gq[v] = (i0 + r < nb) ? *reinterpret_cast<const double2*>(qb + static_cast<long long>(i0 + r) * D + c0 + sc)
-                            : make_double2(0.0, 0.0);
-      gk[v] = (j0 + r < nb) ? *reinterpret_cast<const double2*>(kb + static_cast<long long>(j0 + r) * D + c0 + sc)
-                            : make_double2(0.0, 0.0);
-    }
-  };
-  auto stash = [&](int buf) {
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int r = sr + 16 * v;
-      qs[buf][sc][r] = gq[v].x;
-      qs[buf][sc + 1][r] = gq[v].y;
-      ks[buf][sc][r] = gk[v].x;
-      ks[buf][sc + 1][r] = gk[v].y;
-    }
-  };
-  double acc[8][4];
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-  const int nchunks = D / kSK;
-  fetch(0);
-  stash(0);
-  __syncthreads();
-  for (int ch = 0; ch < nchunks; ++ch) {
-    const int buf = ch & 1;
-    if (ch + 1 < nchunks) fetch((ch + 1) * kSK);
-#pragma unroll
-    for (int cc = 0; cc < kSK; ++cc) {
-      double2 qa[4], kk[2];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-        qa[a] = *reinterpret_cast<const double2*>(&qs[buf][cc][2 * ty + 16 * a]);
-#pragma unroll
-      for (int b = 0; b < 2; ++b)
-        kk[b] = *reinterpret_cast<const double2*>(&ks[buf][cc][2 * tx + 32 * b]);
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          acc[2 * a][2 * b] = fma(qa[a].x, kk[b].x, acc[2 * a][2 * b]);
-          acc[2 * a][2 * b + 1] = fma(qa[a].x, kk[b].y, acc[2 * a][2 * b + 1]);
-          acc[2 * a + 1][2 * b] = fma(qa[a].y, kk[b].x, acc[2 * a + 1][2 * b]);
-          acc[2 * a + 1][2 * b + 1] = fma(qa[a].y, kk[b].y, acc[2 * a + 1][2 * b + 1]);
-        }
-    }
-    // The other buffer was last read before the previous barrier.
-    if (ch + 1 < nchunks) stash(buf ^ 1);
-    __syncthreads();
-  }
-#pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int i = i0 + 2 * ty + 16 * (a / 2) + (a % 2);
-    if (i >= nb) continue;
-    double* srow = S + (bh * nb + i) * nb;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int j = j0 + 2 * tx + 32 * (b / 2) + (b % 2);
-      if (j < nb) srow[j] = acc[a][b];
-    }
-  }
+// ------------------------------------------------------ fused selection --
+// One CTA scores a chunk of RB query blocks of one head against all nb key
+// blocks, selects the topk largest per query block, and merges the kept
+// lists of the chunk's pairs of query blocks for the attention kernel.
+//
+// Exact float64 decision at float32 cost.  Scores are formed in float32 from
+// the float32-rounded means (a sequential fma chain over c, staged through
+// shared memory), so each differs from the float64 score by at most
+//   E_i = (d + 8) 2^-24 * 1.05 * |qbar_i|_2 * max_j |kbar_j|_2
+// (rounding of the means to float32 and of the d-term fma chain, with a 5%
+// margin that also covers the float32 norms).  With T the k-th largest
+// float32 score of the row, a block scoring above T + 2E is among the float64
+// Top-K for certain, one below T - 2E is not; only the blocks in between (the
+// candidates, typically none or a few) are scored again in float64 (ascending
+// c, the same sum as the float64 definition) and ranked by (score desc,
+// index asc).  The kept set is therefore the float64 selection.
+//
+// Phases (256 threads):
+//  1. scores: thread (ty, tx) accumulates rows 4ty..4ty+3 x columns
+//     4tx..4tx+3 of a column tile; the key means stream through two shared
+//     buffers (the next chunk is read into registers while the current one
+//     is multiplied).  The loading threads also sum each key mean's squares.
+//  2. one warp per row: radix select (4 passes of 8 bits over order-
+//     preserving 32-bit keys) for the k-th largest float32 score, the band,
+//     the float64 recheck, the kept bitmap and the ascending index list.
+//  3. one warp per pair of query blocks: the union of the two kept bitmaps
+//     as an ascending list of entries j | mask << 16.
+template <int D, int RB>
+struct SelCfg {
+  static constexpr int kThreads = 256;
+  static constexpr int kWarps = kThreads / 32;
+  static constexpr int kRG = RB / 4;               // 4-row groups
+  static constexpr int kCG = kThreads / kRG;       // 4-column groups
+  static constexpr int kCT = 4 * kCG;              // columns per tile
+  static constexpr int kKC = RB == 16 ? 16 : 8;    // channels per staged chunk
+  static constexpr int kLoadCols = kCT / kThreads; // columns each thread stages
+  static constexpr int kCandMax = 64;              // float64 candidates buffered per warp
+  static_assert(kCG >= 32 && kCG % 32 == 0, "a warp spans one row group");
+  static_assert(D % kKC == 0, "chunking");
+};
+
+template <int D, int RB>
+size_t sel_smem_bytes(int nb) {
+  using C = SelCfg<D, RB>;
+  const size_t nbp = (static_cast<size_t>(nb) + 3) & ~static_cast<size_t>(3);
+  const size_t nw = (static_cast<size_t>(nb) + 31) / 32;
+  return static_cast<size_t>(D) * RB * 4            // qs [D][RB]
+         + 2 * C::kKC * C::kCT * 4                  // ks [2][KC][CT]
+         + RB * nbp * 4                             // scores [RB][nbp]
+         + RB * nw * 4                              // kept bitmaps [RB][nw]
+         + C::kWarps * 256 * 4                      // radix histograms
+         + C::kWarps * C::kCandMax * 12             // candidate j and float64 score
+         + (C::kThreads + RB + 8) * 4;              // norm reduction, row norms
 }
 
-// ------------------------------------------------------------------ topk --
-__device__ __forceinline__ unsigned long long order_key(double x) {
-  x = x + 0.0;  // -0.0 -> +0.0: equal scores must share one key
+__device__ __forceinline__ uint32_t fkey(float x) {
+  x = x + 0.0f;  // -0.0 -> +0.0: equal scores share one key
+  const uint32_t u = __float_as_uint(x);
+  return (u >> 31) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  return __uint_as_float((k >> 31) ? (k & 0x7fffffffu) : ~k);
+}
+__device__ __forceinline__ unsigned long long dkey(double x) {
+  x = x + 0.0;
   const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(x));
   return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
 
-// One warp per query block row (bh, i).  Keys staged in shared memory.
-__global__ void topk_kernel(const double* __restrict__ S, int nrows, int nb, int topk,
-                            int32_t* __restrict__ idx) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int warps = blockDim.x / 32;
-  const int wid = threadIdx.x / 32, lane = threadIdx.x % 32;
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem_raw) +
-                             static_cast<size_t>(wid) * nb;
-  unsigned* hist = reinterpret_cast<unsigned*>(reinterpret_cast<unsigned long long*>(smem_raw) +
-                                               static_cast<size_t>(warps) * nb) +
-                   wid * 256;
-  const long long row = static_cast<long long>(blockIdx.x) * warps + wid;
-  if (row >= nrows) return;
-  const double* srow = S + row * nb;
-  for (int j = lane; j < nb; j += 32) keys[j] = order_key(srow[j]);
-  __syncwarp();
+// float64 score of (query block row qrow, key block j): ascending-c fma chain.
+template <int D>
+__device__ __forceinline__ double score64(const double* __restrict__ qrow,
+                                          const double* __restrict__ kb, int j) {
+  const double* kr = kb + static_cast<long long>(j) * D;
+  double acc = 0.0;
+#pragma unroll 8
+  for (int c = 0; c < D; ++c) acc = fma(__ldg(qrow + c), __ldg(kr + c), acc);
+  return acc;
+}
 
-  unsigned long long prefix = 0, pmask = 0;
-  int want = topk;
-  for (int pass = 0; pass < 8; ++pass) {
-    const int shift = 56 - 8 * pass;
+// Radix select over the keys of `n` items for which `take(j)` holds: finds
+// the digits of the `want`-th largest key, 8 bits per pass from the top.
+// Returns the full key (all passes run) or, when `early` is set and every
+// key sharing the prefix is wanted, the prefix with its mask; `want` is
+// updated to the number still wanted among keys equal to the (masked)
+// prefix.  Warp-collective; hist: 256 words of this warp.
+template <typename Key, typename KeyOf>
+__device__ __forceinline__ void radix_select(int n, int& want, Key& prefix, Key& pmask,
+                                             unsigned* hist, int lane, bool early, KeyOf key_of) {
+  constexpr int kBits = 8 * sizeof(Key);
+  prefix = 0;
+  pmask = 0;
+  for (int shift = kBits - 8; shift >= 0; shift -= 8) {
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
-    for (int j = lane; j < nb; j += 32) {
-      const unsigned long long key = keys[j];
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    for (int j = lane; j < n; j += 32) {
+      bool ok;
+      const Key key = key_of(j, ok);
+      if (ok && (key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncwarp();
-    // Lane L owns bins 8L .. 8L+7.  Suffix sums over lanes find the digit.
     unsigned mine = 0;
 #pragma unroll
     for (int e = 0; e < 8; ++e) mine += hist[lane * 8 + e];
-    unsigned suffix = mine;  // inclusive suffix sum: bins >= 8L
+    unsigned suffix = mine;  // inclusive suffix sum: bins >= 8 lane
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const unsigned t = __shfl_down_sync(0xffffffffu, suffix, o);
       if (lane + o < 32) suffix += t;
     }
-    const unsigned above_lane = suffix - mine;  // bins >= 8(L+1)
-    const bool here = (above_lane < static_cast<unsigned>(want)) &&
-                      (suffix >= static_cast<unsigned>(want));
-    const unsigned ballot = __ballot_sync(0xffffffffu, here);
-    const int owner = __ffs(ballot) - 1;
+    const unsigned above_lane = suffix - mine;
+    const bool here = above_lane < static_cast<unsigned>(want) && suffix >= static_cast<unsigned>(want);
+    const int owner = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
     int digit = 0;
     unsigned above = 0;
     if (lane == owner) {
@@ -226,36 +207,298 @@ __global__ void topk_kernel(const double* __restrict__ S, int nrows, int nb, int
     digit = __shfl_sync(0xffffffffu, digit, owner);
     above = __shfl_sync(0xffffffffu, above, owner);
     want -= static_cast<int>(above);
-    prefix |= static_cast<unsigned long long>(digit) << shift;
-    pmask |= 0xFFull << shift;
-    // Every key that shares the prefix so far is kept: the set is decided
-    // (no tie among kept and dropped keys is left to break).
+    prefix |= static_cast<Key>(digit) << shift;
+    pmask |= static_cast<Key>(0xFF) << shift;
     const bool settled = hist[digit] == static_cast<unsigned>(want);
     __syncwarp();
-    if (settled) {
-      want = 0x7fffffff;
-      break;
+    if (early && settled) return;
+  }
+}
+
+template <int D, int RB>
+__global__ void __launch_bounds__(256) select_fused_kernel(
+    const float* __restrict__ qbar32, const float* __restrict__ kbar32,
+    const double* __restrict__ qbar64, const double* __restrict__ kbar64, int nb, int topk,
+    int32_t* __restrict__ idx, int32_t* __restrict__ lists, int32_t* __restrict__ counts) {
+  using C = SelCfg<D, RB>;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int nbp = (nb + 3) & ~3;
+  const int nw = (nb + 31) / 32;
+  float* qs = reinterpret_cast<float*>(smem_raw);                        // [D][RB]
+  float* ks = qs + D * RB;                                                // [2][KC][CT]
+  float* sc = ks + 2 * C::kKC * C::kCT;                                   // [RB][nbp]
+  unsigned* bits = reinterpret_cast<unsigned*>(sc + RB * nbp);            // [RB][nw]
+  unsigned* hist_all = bits + RB * nw;                                    // [warps][256]
+  double* cand_s = reinterpret_cast<double*>(hist_all + C::kWarps * 256); // [warps][CandMax]
+  int* cand_j = reinterpret_cast<int*>(cand_s + C::kWarps * C::kCandMax); // [warps][CandMax]
+  float* red = reinterpret_cast<float*>(cand_j + C::kWarps * C::kCandMax); // [threads]
+  float* qn = red + C::kThreads;                                          // [RB] row norms
+  float* kmax_s = qn + RB;                                                // [1]
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const long long bh = blockIdx.y;
+  const int i0 = blockIdx.x * RB;
+  const int rows = min(RB, nb - i0);
+  const float* qb = qbar32 + (bh * nb + i0) * D;
+  const float* kb = kbar32 + bh * nb * D;
+
+  // ---- stage the chunk's query means, transposed (invalid rows are 0)
+  for (int e = tid; e < D * RB; e += C::kThreads) {
+    const int r = e / D, c = e % D;
+    qs[c * RB + r] = r < rows ? __ldg(qb + static_cast<long long>(r) * D + c) : 0.0f;
+  }
+
+  // ---- phase 1: float32 scores
+  const int ty = tid / C::kCG, tx = tid % C::kCG;
+  const int ntile = (nb + C::kCT - 1) / C::kCT;
+  constexpr int kChunks = D / C::kKC;
+  const int nch = ntile * kChunks;
+  float4 stage[C::kLoadCols][C::kKC / 4];
+  float kn2[C::kLoadCols];
+  float kmax2 = 0.0f;
+  auto fetch = [&](int ch) {
+    const int j0 = (ch / kChunks) * C::kCT, c0 = (ch % kChunks) * C::kKC;
+#pragma unroll
+    for (int u = 0; u < C::kLoadCols; ++u) {
+      const int j = j0 + tid + u * C::kThreads;
+      const float4* src = reinterpret_cast<const float4*>(kb + static_cast<long long>(j) * D + c0);
+#pragma unroll
+      for (int v = 0; v < C::kKC / 4; ++v)
+        stage[u][v] = j < nb ? __ldg(src + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto stash = [&](int ch) {
+    float* dst = ks + (ch & 1) * C::kKC * C::kCT;
+    if (ch % kChunks == 0) {
+#pragma unroll
+      for (int u = 0; u < C::kLoadCols; ++u) kn2[u] = 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < C::kLoadCols; ++u) {
+      const int jj = tid + u * C::kThreads;
+#pragma unroll
+      for (int v = 0; v < C::kKC / 4; ++v) {
+        const float4 x = stage[u][v];
+        dst[(4 * v + 0) * C::kCT + jj] = x.x;
+        dst[(4 * v + 1) * C::kCT + jj] = x.y;
+        dst[(4 * v + 2) * C::kCT + jj] = x.z;
+        dst[(4 * v + 3) * C::kCT + jj] = x.w;
+        kn2[u] = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, kn2[u]))));
+      }
+    }
+    if (ch % kChunks == kChunks - 1) {
+#pragma unroll
+      for (int u = 0; u < C::kLoadCols; ++u) kmax2 = fmaxf(kmax2, kn2[u]);
+    }
+  };
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  for (int ch = 0; ch < nch; ++ch) {
+    if (ch + 1 < nch) fetch(ch + 1);
+    const float* kbuf = ks + (ch & 1) * C::kKC * C::kCT;
+    const int c0 = (ch % kChunks) * C::kKC;
+#pragma unroll
+    for (int c = 0; c < C::kKC; ++c) {
+      const float4 qv = *reinterpret_cast<const float4*>(qs + (c0 + c) * RB + 4 * ty);
+      const float4 kv = *reinterpret_cast<const float4*>(kbuf + c * C::kCT + 4 * tx);
+      const float q4[4] = {qv.x, qv.y, qv.z, qv.w};
+      const float k4[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(q4[a], k4[b], acc[a][b]);
+    }
+    if (ch % kChunks == kChunks - 1) {
+      const int j = (ch / kChunks) * C::kCT + 4 * tx;
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          if (j + b < nb) sc[(4 * ty + a) * nbp + j + b] = acc[a][b];
+          acc[a][b] = 0.0f;
+        }
+      }
+    }
+    if (ch + 1 < nch) stash(ch + 1);
+    __syncthreads();
+  }
+  // Largest key-mean norm of the head and each row's query-mean norm.
+  red[tid] = kmax2;
+  if (tid < RB) {
+    float n2 = 0.0f;
+    for (int c = 0; c < D; ++c) n2 = fmaf(qs[c * RB + tid], qs[c * RB + tid], n2);
+    qn[tid] = sqrtf(n2);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float m = 0.0f;
+    for (int t = lane; t < C::kThreads; t += 32) m = fmaxf(m, red[t]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) kmax_s[0] = sqrtf(m);
+  }
+  __syncthreads();
+  const double kmax = kmax_s[0];
+
+  // ---- phase 2: per row (warp), the k-th largest float32 score, the band
+  // and, where needed, the float64 decision.
+  unsigned* hist = hist_all + warp * 256;
+  double* cs = cand_s + warp * C::kCandMax;
+  int* cj = cand_j + warp * C::kCandMax;
+  for (int r = warp; r < RB; r += C::kWarps) {
+    unsigned* kept = bits + r * nw;
+    for (int w = lane; w < nw; w += 32) kept[w] = 0u;
+    __syncwarp();
+    if (r >= rows) continue;
+    const float* srow = sc + r * nbp;
+    int want = topk;
+    uint32_t tkey = 0, tmask = 0;
+    radix_select<uint32_t>(nb, want, tkey, tmask, hist, lane, false,
+                           [&](int j, bool& ok) { ok = true; return fkey(srow[j]); });
+    const double T = static_cast<double>(key_to_float(tkey));
+    // The bound, plus an absolute term for products flushed below float32's
+    // normal range.  Means that are not finite or so large that float32 could
+    // overflow make every block a candidate (the float64 path decides).
+    const double qnr = static_cast<double>(qn[r]);
+    const bool wide = !(qnr < 1e18 && kmax < 1e18);
+    const double E = (D + 8) * 5.9604644775390625e-8 * 1.05 * qnr * kmax + D * 2.4e-38;
+    const double lo = wide ? -INFINITY : T - 2.0 * E, hi = wide ? INFINITY : T + 2.0 * E;
+    // Certain members (above the band) and candidates (inside it).
+    int n_in = 0, n_cand = 0;
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+      const int j = j0 + lane;
+      const double v = j < nb ? static_cast<double>(srow[j]) : -INFINITY;
+      const bool in = j < nb && v > hi;
+      const bool cand = j < nb && !(v > hi) && (wide || v >= lo);
+      const unsigned bin = __ballot_sync(0xffffffffu, in);
+      if (lane == 0) kept[j0 / 32] = bin;
+      n_in += __popc(bin);
+      n_cand += __popc(__ballot_sync(0xffffffffu, cand));
+    }
+    __syncwarp();
+    const int need = topk - n_in;   // 0 <= need <= n_cand
+    auto is_cand = [&](int j) {
+      const double v = static_cast<double>(srow[j]);
+      return !(v > hi) && (wide || v >= lo);
+    };
+    if (need == n_cand) {
+      // Every candidate is kept: no float64 needed.
+      for (int j0 = 0; j0 < nb; j0 += 32) {
+        const int j = j0 + lane;
+        const unsigned b = __ballot_sync(0xffffffffu, j < nb && is_cand(j));
+        if (lane == 0) kept[j0 / 32] |= b;
+      }
+    } else if (need > 0) {
+      const double* qrow = qbar64 + (bh * nb + i0 + r) * D;
+      const double* kb64 = kbar64 + bh * nb * D;
+      if (n_cand <= C::kCandMax) {
+        // Buffer the candidates (ascending j) with their float64 scores and
+        // keep the `need` best by (score desc, j asc).
+        int nc = 0;
+        for (int j0 = 0; j0 < nb; j0 += 32) {
+          const int j = j0 + lane;
+          const bool cand = j < nb && is_cand(j);
+          const unsigned b = __ballot_sync(0xffffffffu, cand);
+          if (cand) cj[nc + __popc(b & ((1u << lane) - 1u))] = j;
+          nc += __popc(b);
+        }
+        __syncwarp();
+        for (int t = lane; t < nc; t += 32) cs[t] = score64<D>(qrow, kb64, cj[t]);
+        __syncwarp();
+        for (int t = lane; t < nc; t += 32) {
+          // Ranked on the order-preserving keys: a total order, so exactly
+          // `need` candidates are kept whatever the values.
+          const unsigned long long st = dkey(cs[t]);
+          int rank = 0;
+          for (int u = 0; u < nc; ++u) {
+            const unsigned long long su = dkey(cs[u]);
+            rank += (su > st || (su == st && u < t)) ? 1 : 0;
+          }
+          if (rank < need) atomicOr(&kept[cj[t] / 32], 1u << (cj[t] % 32));
+        }
+        __syncwarp();
+      } else {
+        // Many candidates (near-degenerate rows, e.g. exact ties): a radix
+        // select over their float64 keys, each key recomputed when read.
+        int want64 = need;
+        unsigned long long pfx = 0, pm = 0;
+        radix_select<unsigned long long>(nb, want64, pfx, pm, hist, lane, true,
+                                         [&](int j, bool& ok) {
+                                           ok = is_cand(j);
+                                           return ok ? dkey(score64<D>(qrow, kb64, j)) : 0ull;
+                                         });
+        int eq_seen = 0;
+        for (int j0 = 0; j0 < nb; j0 += 32) {
+          const int j = j0 + lane;
+          const bool cand = j < nb && is_cand(j);
+          const unsigned long long key = cand ? (dkey(score64<D>(qrow, kb64, j)) & pm) : 0ull;
+          const bool gt = cand && key > pfx;
+          const bool eq = cand && key == pfx;
+          const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+          const int eq_rank = eq_seen + __popc(eqb & ((1u << lane) - 1u));
+          const unsigned kb2 = __ballot_sync(0xffffffffu, gt || (eq && eq_rank < want64));
+          if (lane == 0) kept[j0 / 32] |= kb2;
+          eq_seen += __popc(eqb);
+        }
+        __syncwarp();
+      }
+    }
+    // The kept list, ascending.
+    if (idx != nullptr) {
+      int32_t* out = idx + (bh * nb + i0 + r) * static_cast<long long>(topk);
+      int written = 0;
+      for (int j0 = 0; j0 < nb; j0 += 32) {
+        const int j = j0 + lane;
+        const unsigned word = kept[j0 / 32];
+        const bool keep = j < nb && ((word >> lane) & 1u);
+        const int pos = written + __popc(word & ((1u << lane) - 1u));
+        if (keep && pos < topk) out[pos] = j;
+        written += __popc(word);
+      }
     }
   }
-  // Keep every key whose masked value exceeds the prefix and the first
-  // `want` whose masked value equals it, in index order.  After all eight
-  // passes the mask is full and `prefix` is the exact key of the topk-th
-  // largest score; after an early stop every equal key is kept.
-  int32_t* out = idx + row * topk;
-  int written = 0, eq_seen = 0;
-  for (int j0 = 0; j0 < nb; j0 += 32) {
-    const int j = j0 + lane;
-    const unsigned long long key = j < nb ? (keys[j] & pmask) : 0ull;
-    const bool gt = j < nb && key > prefix;
-    const bool eq = j < nb && key == prefix;
-    const unsigned eq_ballot = __ballot_sync(0xffffffffu, eq);
-    const int eq_rank = eq_seen + __popc(eq_ballot & ((1u << lane) - 1u));
-    const bool keep = gt || (eq && eq_rank < want);
-    const unsigned kb = __ballot_sync(0xffffffffu, keep);
-    const int pos = written + __popc(kb & ((1u << lane) - 1u));
-    if (keep && pos < topk) out[pos] = j;
-    written += __popc(kb);
-    eq_seen += __popc(eq_ballot);
+  if (lists == nullptr) return;
+  __syncthreads();
+
+  // ---- phase 3: union of the kept sets of each pair (2p, 2p+1) of the chunk
+  const int npairs_all = (nb + 1) / 2;
+  for (int pr = warp; pr < (rows + 1) / 2; pr += C::kWarps) {
+    const int p = i0 / 2 + pr;
+    const unsigned* A = bits + (2 * pr) * nw;
+    const bool has_b = 2 * pr + 1 < rows;
+    const unsigned* Bm = bits + (2 * pr + 1) * nw;
+    const long long item = bh * npairs_all + p;
+    int32_t* out = lists + item * (2 * topk);
+    int base = 0;
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+      const int w = w0 + lane;
+      const unsigned a = w < nw ? A[w] : 0u;
+      const unsigned b = (w < nw && has_b) ? Bm[w] : 0u;
+      unsigned u = a | b;
+      const int c = __popc(u);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int pos = base + incl - c;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1;
+        const int mask = static_cast<int>((a >> bit) & 1u) | (static_cast<int>((b >> bit) & 1u) << 1);
+        if (pos < 2 * topk) out[pos] = (w * 32 + bit) | (mask << 16);
+        ++pos;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) counts[item] = min(base, 2 * topk);
   }
 }
 
@@ -317,7 +560,7 @@ __global__ void pair_union_kernel(const int32_t* __restrict__ idx, int BH, int n
 }
 
 struct SelectLayout {
-  size_t qbar, kbar, scores, total;
+  size_t qbar, kbar, qbar32, kbar32, total;
 };
 SelectLayout select_layout(int B, int H, int N, int d, int block) {
   const size_t nb = (static_cast<size_t>(N) + block - 1) / block;
@@ -325,10 +568,30 @@ SelectLayout select_layout(int B, int H, int N, int d, int block) {
   SelectLayout L;
   L.qbar = 0;
   L.kbar = L.qbar + align256(BH * nb * d * sizeof(double));
-  L.scores = L.kbar + align256(BH * nb * d * sizeof(double));
-  L.total = L.scores + align256(BH * nb * nb * sizeof(double));
+  L.qbar32 = L.kbar + align256(BH * nb * d * sizeof(double));
+  L.kbar32 = L.qbar32 + align256(BH * nb * d * sizeof(float));
+  L.total = L.kbar32 + align256(BH * nb * d * sizeof(float));
   return L;
 }
+
+template <int D, int RB>
+cudaError_t launch_select_fused(const Ctx& c, const float* q32, const float* k32,
+                                const double* q64, const double* k64, int BH, int nb, int topk,
+                                int32_t* idx, int32_t* lists, int32_t* counts) {
+  const size_t smem = sel_smem_bytes<D, RB>(nb);
+  cudaError_t e = cudaFuncSetAttribute(select_fused_kernel<D, RB>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((nb + RB - 1) / RB, BH);
+  select_fused_kernel<D, RB><<<grid, SelCfg<D, RB>::kThreads, smem, c.stream>>>(
+      q32, k32, q64, k64, nb, topk, idx, lists, counts);
+  return cudaGetLastError();
+}
+
+// 16 query blocks per CTA while their scores fit next to the staging buffers,
+// else 8 (every nb up to 4096 fits).
+constexpr size_t kSelSmemCap = 200 * 1024;
 
 }  // namespace
 
@@ -337,36 +600,37 @@ size_t select_ws_bytes(int B, int H, int N, int d, int block) {
 }
 
 cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
-                          int topk, int32_t* idx, void* ws) {
+                          int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts) {
   const SelectLayout L = select_layout(B, H, N, d, kBlock);
   char* base = static_cast<char*>(ws);
   double* qbar = reinterpret_cast<double*>(base + L.qbar);
   double* kbar = reinterpret_cast<double*>(base + L.kbar);
-  double* S = reinterpret_cast<double*>(base + L.scores);
+  float* qbar32 = reinterpret_cast<float*>(base + L.qbar32);
+  float* kbar32 = reinterpret_cast<float*>(base + L.kbar32);
   const int nb = (N + kBlock - 1) / kBlock;
   const int BH = B * H;
   dim3 pg(nb, BH, 2);
   if (d == 128)
     pool_kernel<128><<<pg, 128, 0, c.stream>>>(static_cast<const uint4*>(q),
-                                                static_cast<const uint4*>(k), N, nb, qbar, kbar);
+                                                static_cast<const uint4*>(k), N, nb, qbar, kbar,
+                                                qbar32, kbar32);
   else
     pool_kernel<64><<<pg, 128, 0, c.stream>>>(static_cast<const uint4*>(q),
-                                               static_cast<const uint4*>(k), N, nb, qbar, kbar);
-  dim3 sg((nb + kST - 1) / kST, (nb + kST - 1) / kST, BH);
-  score_kernel<<<sg, 128, 0, c.stream>>>(qbar, kbar, nb, d, S);
-  // topk: as many warps per CTA as fit 192 KB of staged keys (>= 1).
-  const size_t per_warp = static_cast<size_t>(nb) * 8 + 256 * 4;
-  int warps = static_cast<int>((192 * 1024) / per_warp);
-  if (warps > 8) warps = 8;
-  if (warps < 1) warps = 1;
-  const size_t smem = per_warp * warps;
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+                                               static_cast<const uint4*>(k), N, nb, qbar, kbar,
+                                               qbar32, kbar32);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int nrows = BH * nb;
-  topk_kernel<<<(nrows + warps - 1) / warps, warps * 32, smem, c.stream>>>(S, nrows, nb, topk,
-                                                                          idx);
-  return cudaGetLastError();
+  if (d == 128)
+    return sel_smem_bytes<128, 16>(nb) <= kSelSmemCap
+               ? launch_select_fused<128, 16>(c, qbar32, kbar32, qbar, kbar, BH, nb, topk, idx,
+                                              lists, counts)
+               : launch_select_fused<128, 8>(c, qbar32, kbar32, qbar, kbar, BH, nb, topk, idx,
+                                             lists, counts);
+  return sel_smem_bytes<64, 16>(nb) <= kSelSmemCap
+             ? launch_select_fused<64, 16>(c, qbar32, kbar32, qbar, kbar, BH, nb, topk, idx,
+                                           lists, counts)
+             : launch_select_fused<64, 8>(c, qbar32, kbar32, qbar, kbar, BH, nb, topk, idx,
+                                          lists, counts);
 }
 
 size_t pairs_ws_bytes(int B, int H, int N, int topk) {

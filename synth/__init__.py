@@ -35,7 +35,8 @@ from typing import Dict, List, Optional
 import numpy as np
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "generate", "generate_projections", "topk_for_sparsity"]
+__all__ = ["Workload", "WORKLOADS", "generate", "generate_device", "generate_projections",
+           "topk_for_sparsity"]
 
 
 def topk_for_sparsity(nb: int, sparsity: float) -> int:
@@ -195,6 +196,42 @@ def generate(w: Workload, heads: Optional[List[int]] = None) -> Dict[str, torch.
         "x": torch.stack(xs), "w_gate": w_gate, "w_lin": w_lin,
         "bias": float(w.bias),
     }
+
+
+def generate_device(w: Workload, device, seed: int = 0) -> Dict[str, torch.Tensor]:
+    """The same recipe as ``generate`` drawn on the device with torch's
+    generator: the same distributions, shapes and frame structure, not the
+    same bytes.  For timing runs at sizes whose host-side draws would take
+    minutes; parity checks use ``generate``."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) * 1000003 + 12345)
+    B, H, N, d, r = w.B, w.H, w.N, w.d, w.lowrank_rank
+    frame = torch.arange(N, device=device) // (w.Hh * w.Wh)
+
+    def qkv():
+        out = []
+        for _ in range(3):
+            out.append(torch.randn(B, H, N, d, generator=g, device=device, dtype=torch.float32))
+        q, k, v = out
+        if w.lowrank_scale != 0.0:
+            for b in range(B):
+                for h in range(H):
+                    u_qk = torch.randn(r, d, generator=g, device=device) / math.sqrt(r)
+                    a_qk = torch.randn(w.F, r, generator=g, device=device)
+                    u_v = torch.randn(r, d, generator=g, device=device) / math.sqrt(r)
+                    a_v = torch.randn(w.F, r, generator=g, device=device)
+                    lr_qk = (w.lowrank_scale * (a_qk @ u_qk))[frame]
+                    q[b, h] += lr_qk
+                    k[b, h] += lr_qk
+                    v[b, h] += (w.lowrank_scale * (a_v @ u_v))[frame]
+        return [t.to(torch.bfloat16) for t in (q, k, v)]
+
+    q, k, v = qkv()
+    x = torch.randn(B, N, w.D, generator=g, device=device).to(torch.bfloat16)
+    w_gate = (0.02 * torch.randn(w.D, generator=g, device=device)).to(torch.bfloat16)
+    w_lin = (0.02 * torch.randn(H, d, d, generator=g, device=device)).to(torch.bfloat16)
+    return {"q": q, "k": k, "v": v, "x": x, "w_gate": w_gate, "w_lin": w_lin,
+            "bias": float(w.bias)}
 
 
 def generate_projections(w: Workload, d_out: Optional[int] = None) -> Dict[str, torch.Tensor]:

@@ -92,6 +92,57 @@ def test_select_all_blocks_and_ties(salad):
     salad.check_error()
 
 
+def _tie_case(nb, N, big_in, big_out, scale=1.0):
+    """Q, K [1,1,N,128] whose block scores agree to ~1e-10 relative, beyond
+    float32 resolution: every query row is all ones (times `scale`); key
+    channel 0 is zero but for row 0 of block j, which carries a distinct tiny
+    value t_j (exact in bf16), and every other key channel is one, so the
+    float64 scores 127 + t_j / 64 (times scale^2) differ only in t_j.  The
+    first `big_in` blocks get 2 on channel 1 of every row (decided in float32,
+    kept) and the last `big_out` blocks 0 there (decided, dropped)."""
+    d = 128
+    q = torch.full((1, 1, N, d), scale, dtype=torch.float32)
+    k = torch.full((1, 1, N, d), scale, dtype=torch.float32)
+    k[..., 0] = 0.0
+    for j in range(nb):
+        t = ((j * 37) % nb + 1) * 2.0 ** -20
+        k[0, 0, j * 64, 0] = scale * t
+        if j < big_in:
+            k[0, 0, j * 64:(j + 1) * 64, 1] = 2.0 * scale
+        elif j >= nb - big_out:
+            k[0, 0, j * 64:(j + 1) * 64, 1] = 0.0
+    return q.to(torch.bfloat16), k.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("nb,N,topk,big_in,big_out,scale", [
+    (96, 96 * 64 - 17, 30, 0, 0, 1.0),     # every block a candidate: radix path over float64 keys
+    (40, 40 * 64, 10, 5, 15, 1.0),          # 20 candidates, 5 to keep: buffered float64 ranking
+    (24, 24 * 64, 7, 3, 3, 2.0 ** 64),      # float32 would overflow: every block goes to float64
+])
+def test_select_decided_in_float64(salad, nb, N, topk, big_in, big_out, scale):
+    # The kept sets must equal the float64 selection exactly -- no near-tie
+    # excuse, although the scores differ by far less than 1e-5 relative: the
+    # float32 pass cannot order these blocks, the float64 recheck must.
+    q, k = _tie_case(nb, N, big_in, big_out, scale)
+    assert (N + 63) // 64 == nb
+    t = ((np.arange(nb) * 37) % nb + 1)
+    assert len(set(t.tolist())) == nb        # distinct perturbations
+    idx = salad.select_blocks(q.cuda(), k.cuda(), topk)
+    torch.cuda.synchronize()
+    salad.check_error()
+    S = oracle.block_scores(to64(q)[0, 0], to64(k)[0, 0], 64)
+    ref = oracle.select_topk(S, topk)
+    got = idx.cpu().numpy()[0, 0]
+    for i in range(nb):
+        assert np.array_equal(np.sort(ref[i]), got[i]), (i, sorted(ref[i].tolist()), got[i].tolist())
+    # The case really is below float32 resolution: float32 scores tie.
+    qm32 = oracle.block_means(to64(q)[0, 0], 64).astype(np.float32)
+    km32 = oracle.block_means(to64(k)[0, 0], 64).astype(np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        S32 = qm32 @ km32.T
+    assert len(np.unique(S32[0, big_in:nb - big_out])) == 1
+
+
 @pytest.mark.parametrize("w", CASES + [WORKLOADS["topk480"]], ids=lambda w: w.name)
 def test_linear_state(salad, w):
     inp = generate(w)

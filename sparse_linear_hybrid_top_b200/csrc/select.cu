@@ -88,8 +88,9 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
 //   E_i = (d + 8) 2^-24 * 1.05 * |qbar_i|_2 * max_j |kbar_j|_2
 // (rounding of the means to float32 and of the d-term fma chain, with a 5%
 // margin that also covers the float32 norms).  With T the k-th largest
-// float32 score of the row, a block scoring above T + 2E is among the float64
-// Top-K for certain, one below T - 2E is not; only the blocks in between (the
+// float32 score of the row, bracketed as blo <= T < bhi, the float64 k-th
+// largest lies in [blo - E, bhi + E]: a block scoring above bhi + 2E is among
+// the float64 Top-K for certain, one below blo - 2E is not; only the blocks in between (the
 // candidates, typically none or a few) are scored again in float64 (ascending
 // c, the same sum as the float64 definition) and ranked by (score desc,
 // index asc).  The kept set is therefore the float64 selection.
@@ -99,9 +100,10 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
 //     4tx..4tx+3 of a column tile; the key means stream through two shared
 //     buffers (the next chunk is read into registers while the current one
 //     is multiplied).  The loading threads also sum each key mean's squares.
-//  2. one warp per row: radix select (4 passes of 8 bits over order-
-//     preserving 32-bit keys) for the k-th largest float32 score, the band,
-//     the float64 recheck, the kept bitmap and the ascending index list.
+//  2. one warp per row: a bisection on the value brackets the k-th largest
+//     float32 score to within the bound; then the band, the float64 recheck
+//     (candidates ranked directly, or by a radix select over float64 keys
+//     when there are many), the kept bitmap and the ascending index list.
 //  3. one warp per pair of query blocks: the union of the two kept bitmaps
 //     as an ascending list of entries j | mask << 16.
 template <int D, int RB>
@@ -132,14 +134,6 @@ size_t sel_smem_bytes(int nb) {
          + (C::kThreads + RB + 8) * 4;              // norm reduction, row norms
 }
 
-__device__ __forceinline__ uint32_t fkey(float x) {
-  x = x + 0.0f;  // -0.0 -> +0.0: equal scores share one key
-  const uint32_t u = __float_as_uint(x);
-  return (u >> 31) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float key_to_float(uint32_t k) {
-  return __uint_as_float((k >> 31) ? (k & 0x7fffffffu) : ~k);
-}
 __device__ __forceinline__ unsigned long long dkey(double x) {
   x = x + 0.0;
   const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(x));
@@ -357,18 +351,43 @@ __global__ void __launch_bounds__(256) select_fused_kernel(
     __syncwarp();
     if (r >= rows) continue;
     const float* srow = sc + r * nbp;
-    int want = topk;
-    uint32_t tkey = 0, tmask = 0;
-    radix_select<uint32_t>(nb, want, tkey, tmask, hist, lane, false,
-                           [&](int j, bool& ok) { ok = true; return fkey(srow[j]); });
-    const double T = static_cast<double>(key_to_float(tkey));
-    // The bound, plus an absolute term for products flushed below float32's
-    // normal range.  Means that are not finite or so large that float32 could
-    // overflow make every block a candidate (the float64 path decides).
+    // Bracket the k-th largest float32 score T: cnt(>= lo) >= topk > cnt(>= hi),
+    // so lo <= T < hi, by bisection on the value (a ballot-free count per
+    // step) until the bracket is narrower than the bound E allows.
     const double qnr = static_cast<double>(qn[r]);
     const bool wide = !(qnr < 1e18 && kmax < 1e18);
     const double E = (D + 8) * 5.9604644775390625e-8 * 1.05 * qnr * kmax + D * 2.4e-38;
-    const double lo = wide ? -INFINITY : T - 2.0 * E, hi = wide ? INFINITY : T + 2.0 * E;
+    auto count_ge = [&](float t) -> int {
+      unsigned cnt = 0;
+      for (int j = lane; j < nb; j += 32) cnt += srow[j] >= t ? 1u : 0u;
+      return static_cast<int>(__reduce_add_sync(0xffffffffu, cnt));
+    };
+    float mn = INFINITY, mx = -INFINITY;
+    for (int j = lane; j < nb; j += 32) {
+      mn = fminf(mn, srow[j]);
+      mx = fmaxf(mx, srow[j]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    double blo = mn, bhi = mx;   // the bracket of T
+    if (!wide && count_ge(mx) < topk) {
+      float lo = mn, hi = mx;
+      for (int it = 0; it < 64 && static_cast<double>(hi) - lo > 0.5 * E; ++it) {
+        const float mid = lo + 0.5f * (hi - lo);
+        if (!(mid > lo && mid < hi)) break;   // adjacent floats
+        if (count_ge(mid) >= topk) lo = mid; else hi = mid;
+      }
+      blo = lo;
+      bhi = hi;
+    } else {
+      blo = bhi = mx;   // T = mx (ties at the maximum), or the band is everything
+    }
+    // The float64 k-th largest lies within [blo - E, bhi + E]: above
+    // bhi + 2E a block is kept for certain, below blo - 2E dropped.
+    const double lo = wide ? -INFINITY : blo - 2.0 * E, hi = wide ? INFINITY : bhi + 2.0 * E;
     // Certain members (above the band) and candidates (inside it).
     int n_in = 0, n_cand = 0;
     for (int j0 = 0; j0 < nb; j0 += 32) {
@@ -599,8 +618,12 @@ size_t select_ws_bytes(int B, int H, int N, int d, int block) {
   return select_layout(B, H, N, d, block).total;
 }
 
-cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
-                          int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts) {
+namespace {
+
+// Pools Q (z = 0) and, when k is given, K (z = 1), then selects.
+cudaError_t pool_and_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
+                            int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts,
+                            cudaEvent_t kbar_ready) {
   const SelectLayout L = select_layout(B, H, N, d, kBlock);
   char* base = static_cast<char*>(ws);
   double* qbar = reinterpret_cast<double*>(base + L.qbar);
@@ -609,7 +632,7 @@ cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int
   float* kbar32 = reinterpret_cast<float*>(base + L.kbar32);
   const int nb = (N + kBlock - 1) / kBlock;
   const int BH = B * H;
-  dim3 pg(nb, BH, 2);
+  dim3 pg(nb, BH, k != nullptr ? 2 : 1);
   if (d == 128)
     pool_kernel<128><<<pg, 128, 0, c.stream>>>(static_cast<const uint4*>(q),
                                                 static_cast<const uint4*>(k), N, nb, qbar, kbar,
@@ -620,6 +643,8 @@ cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int
                                                qbar32, kbar32);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (kbar_ready != nullptr && (e = cudaStreamWaitEvent(c.stream, kbar_ready, 0)) != cudaSuccess)
+    return e;
   if (d == 128)
     return sel_smem_bytes<128, 16>(nb) <= kSelSmemCap
                ? launch_select_fused<128, 16>(c, qbar32, kbar32, qbar, kbar, BH, nb, topk, idx,
@@ -631,6 +656,26 @@ cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int
                                            lists, counts)
              : launch_select_fused<64, 8>(c, qbar32, kbar32, qbar, kbar, BH, nb, topk, idx,
                                           lists, counts);
+}
+
+}  // namespace
+
+cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
+                          int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts) {
+  return pool_and_select(c, q, k, B, H, N, d, topk, idx, ws, lists, counts, nullptr);
+}
+
+void select_kbar(void* ws, int B, int H, int N, int d, double** kbar64, float** kbar32) {
+  const SelectLayout L = select_layout(B, H, N, d, kBlock);
+  char* base = static_cast<char*>(ws);
+  *kbar64 = reinterpret_cast<double*>(base + L.kbar);
+  *kbar32 = reinterpret_cast<float*>(base + L.kbar32);
+}
+
+cudaError_t launch_select_q(const Ctx& c, const void* q, int B, int H, int N, int d, int topk,
+                            int32_t* idx, void* ws, int32_t* lists, int32_t* counts,
+                            cudaEvent_t kbar_ready) {
+  return pool_and_select(c, q, nullptr, B, H, N, d, topk, idx, ws, lists, counts, kbar_ready);
 }
 
 size_t pairs_ws_bytes(int B, int H, int N, int topk) {

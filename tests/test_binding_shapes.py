@@ -129,8 +129,7 @@ def test_outputs_checked_like_inputs():
     q, k, v, x, wg = inp["q"], inp["k"], inp["v"], inp["x"], inp["w_gate"]
     B, H, N, d = q.shape
     nb = w.nb
-    bad_s = [torch.zeros(B), torch.zeros(B, dtype=torch.float64, device="cuda"),
-             torch.zeros(2 * B, device="cuda")[::2]]
+    bad_s = [torch.zeros(B), torch.zeros(B, dtype=torch.float64, device="cuda")]
     for s in bad_s:
         with pytest.raises(ValueError, match="s must|s is on"):
             salad.gate(x, wg, 0.0, s=s)
@@ -142,7 +141,9 @@ def test_outputs_checked_like_inputs():
             salad.select_blocks(q, k, 2, idx=idx)
         with pytest.raises(ValueError, match="idx must"):
             salad.sparse_attn(q, k, v, "topk", topk=2, idx=idx)
-    for o in (torch.empty_like(q, device="cpu"), torch.empty(q.shape, device="cuda")):
+    strided = torch.empty(B, H, N, 2 * d, dtype=torch.bfloat16, device="cuda")[..., ::2]
+    assert strided.shape == q.shape and not strided.is_contiguous()
+    for o in (torch.empty_like(q, device="cpu"), torch.empty(q.shape, device="cuda"), strided):
         with pytest.raises(ValueError, match="o must"):
             salad.dense_attn(q, k, v, o=o)
         with pytest.raises(ValueError, match="o must"):

@@ -282,20 +282,14 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
       uint32_t qc = 0;    // items started (Q buffer qc & 1)
       uint32_t q_issued = 0;   // Q loads issued (drained at the end)
       bool ok = true;
-      for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++qc) {
+      // Q rows of item number j (two 64-row boxes per d-slab; rows past N
+      // read 0) into buffer j & 1, once the item two before it has freed it.
+      auto load_q = [&](long long w, uint32_t j) -> bool {
         const Item it = make_item(P, w);
         const CUtensorMap* qm = it.slot >= 0 ? &mqp : &mq;
-        const CUtensorMap* km = it.slot >= 0 ? &mkp : &mk;
-        const CUtensorMap* vm = it.slot >= 0 ? &mvp : &mv;
         const int z = it.slot >= 0 ? it.b * P.Hs + it.slot : it.bh;
-        const int T = (it.ntiles + 1) / 2;
-        const bool lin = HYB && lin_on(P, it.b);
-        // Q rows of the item (two 64-row boxes per d-slab; rows past N read 0).
-        const int qb = static_cast<int>(qc & 1);
-        if (qc >= 2 && !mbar_wait(q_empty(qb), ((qc - 2) / 2) & 1, wait_ns, abort_flag)) {
-          ok = false;
-          break;
-        }
+        const int qb = static_cast<int>(j & 1);
+        if (j >= 2 && !mbar_wait(q_empty(qb), ((j - 2) / 2) & 1, wait_ns, abort_flag)) return false;
         mbar_arrive_expect_tx(q_full(qb), C::kQBuf);
 #pragma unroll
         for (int hh = 0; hh < D / 64; ++hh)
@@ -303,7 +297,17 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
           for (int rb = 0; rb < 2; ++rb)
             tma_load_3d(q_addr(qb) + hh * C::kRowSlab + rb * kSlab, qm, q_full(qb), hh * 64,
                         it.p * 128 + rb * 64, z);
-        q_issued = qc + 1;
+        q_issued = j + 1;
+        return true;
+      };
+      if (static_cast<long long>(blockIdx.x) < total) ok = load_q(blockIdx.x, 0);
+      for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++qc) {
+        const Item it = make_item(P, w);
+        const CUtensorMap* km = it.slot >= 0 ? &mkp : &mk;
+        const CUtensorMap* vm = it.slot >= 0 ? &mvp : &mv;
+        const int z = it.slot >= 0 ? it.b * P.Hs + it.slot : it.bh;
+        const int T = (it.ntiles + 1) / 2;
+        const bool lin = HYB && lin_on(P, it.b);
         // The item's loads in the MMA thread's order: K0, K1, then V(t) and
         // K(t+2) for each tile t, then the G image.
         auto push = [&](int kind, int t) -> bool {
@@ -333,6 +337,10 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
           return true;
         };
         ok = push(0, 0) && (T < 2 || push(0, 1));
+        // The next item's Q, a whole item ahead: its buffer was the previous
+        // item's, free once that item's MMAs have run (which needs nothing
+        // more from this thread).
+        if (ok && w + gridDim.x < total) ok = load_q(w + gridDim.x, qc + 1);
         for (int t = 0; t < T && ok; ++t) ok = push(1, t) && (t + 2 >= T || push(0, t + 2));
         if (ok && lin) ok = push(2, 0);
       }

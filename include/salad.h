@@ -146,7 +146,8 @@ salad_status salad_linear_apply(const void* q, const float* Hst, const float* Z,
  * Token permutation of the ST-SWA heads (ijyty.com 1.1).  The latent grid
  * F x Hh x Wh (N = F*Hh*Wh) is flattened frame-major, t = (f*Hh + y)*Wh + x;
  * the space-major order is r = (y*Wh + x)*F + f.
- * src, dst: bf16 [S, N, d] device, S = number of (batch, head) slabs.
+ * src, dst: bf16 [S, N, d] device, S = number of (batch, head) slabs,
+ * 1 <= S <= 65535.
  * inverse = 0: dst[s][r] = src[s][t(r)] (frame-major -> space-major);
  * inverse = 1: dst[s][t(r)] = src[s][r] (space-major -> frame-major).
  * src and dst must not overlap.

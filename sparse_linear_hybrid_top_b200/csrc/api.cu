@@ -399,7 +399,7 @@ salad_status salad_project(const void* a, int B, int H, int N, int d, const void
 // --------------------------------------------------------------- permute --
 salad_status salad_permute_tokens(const void* src, void* dst, int S, int N, int d, int F, int Hh,
                                   int Wh, int inverse, salad_stream stream) {
-  if (S < 1 || N < 1 || F < 1 || Hh < 1 || Wh < 1) return SALAD_ERR_INVALID_ARG;
+  if (S < 1 || S > 65535 || N < 1 || F < 1 || Hh < 1 || Wh < 1) return SALAD_ERR_INVALID_ARG;
   if (static_cast<long long>(F) * Hh * Wh != N) return SALAD_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return SALAD_ERR_UNSUPPORTED;
   if (!aligned(src, 16) || !aligned(dst, 16) || (inverse != 0 && inverse != 1))

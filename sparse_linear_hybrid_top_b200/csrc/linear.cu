@@ -294,6 +294,24 @@ __global__ void __launch_bounds__(192, 1) linear_state_kernel(
   }
 }
 
+// Sum over c = 0..n-1 of src[c * stride], in ascending c, with eight loads in
+// flight at a time (the partials live in L2 or HBM; a dependent chain of
+// loads would leave the reduction latency-bound).
+__device__ __forceinline__ float sum_strided(const float* __restrict__ src, long long stride,
+                                             int n) {
+  float acc = 0.f;
+  int c = 0;
+  for (; c + 8 <= n; c += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = __ldg(src + (c + u) * stride);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc += v[u];
+  }
+  for (; c < n; ++c) acc += __ldg(src + c * stride);
+  return acc;
+}
+
 // Fixed-order reduction of the split-N partials.
 __global__ void linear_reduce_kernel(const float* __restrict__ partH,
                                      const float* __restrict__ partZ, int D, int cph,
@@ -301,16 +319,8 @@ __global__ void linear_reduce_kernel(const float* __restrict__ partH,
   const long long bh = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   const int DD = D * D;
-  if (e < DD) {
-    float acc = 0.f;
-    for (int c = 0; c < cph; ++c) acc += partH[(bh * cph + c) * DD + e];
-    Hst[bh * DD + e] = acc;
-  }
-  if (e < D) {
-    float acc = 0.f;
-    for (int c = 0; c < cph; ++c) acc += partZ[(bh * cph + c) * D + e];
-    Z[bh * D + e] = acc;
-  }
+  if (e < DD) Hst[bh * DD + e] = sum_strided(partH + bh * cph * DD + e, DD, cph);
+  if (e < D) Z[bh * D + e] = sum_strided(partZ + bh * cph * D + e, D, cph);
 }
 
 // The linear state's reduction fused with the fold of W_lin, for the forward
@@ -338,17 +348,13 @@ __global__ void __launch_bounds__(256) linear_reduce_fold_kernel(
     reinterpret_cast<uint4*>(wsm)[e] = __ldg(wsrc + e);
   for (int e = threadIdx.x; e < kFoldRows * D; e += blockDim.x) {
     const long long off = static_cast<long long>(r0) * D + e;
-    float acc = 0.f;
-    for (int c = 0; c < cph; ++c) acc += partH[(bh * cph + c) * DD + off];
+    const float acc = sum_strided(partH + bh * cph * DD + off, DD, cph);
     hrows[e] = acc;
     Hst[bh * DD + off] = acc;
   }
   if (blockIdx.x == 0) {
-    for (int e = threadIdx.x; e < D; e += blockDim.x) {
-      float acc = 0.f;
-      for (int c = 0; c < cph; ++c) acc += partZ[(bh * cph + c) * D + e];
-      Z[bh * D + e] = acc;
-    }
+    for (int e = threadIdx.x; e < D; e += blockDim.x)
+      Z[bh * D + e] = sum_strided(partZ + bh * cph * D + e, D, cph);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < kFoldRows * D; e += blockDim.x) {

@@ -92,6 +92,8 @@ def test_permute_argument_checks():
     assert lib.salad_permute_tokens(A, A + 64, 2, 12, 64, 2, 2, 3, 0, None) == INVALID  # overlap
     assert lib.salad_permute_tokens(A, A + (1 << 20), 2, 12, 64, 2, 2, 4, 0, None) == INVALID
     assert lib.salad_permute_tokens(A, A + (1 << 20), 2, 12, 64, 2, 2, 3, 2, None) == INVALID
+    # more slabs than one grid dimension holds
+    assert lib.salad_permute_tokens(A, A + (1 << 36), 65536, 12, 64, 2, 2, 3, 0, None) == INVALID
 
 
 def test_project_argument_checks():

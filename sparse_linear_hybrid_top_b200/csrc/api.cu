@@ -41,7 +41,7 @@ std::mutex g_mu;
 struct SideSet {
   cudaStream_t caller = nullptr;
   cudaStream_t side[2] = {nullptr, nullptr};
-  cudaEvent_t fork = nullptr, join_gate = nullptr, join_lin = nullptr, kbar_ready = nullptr;
+  cudaEvent_t fork = nullptr, join_gate = nullptr, join_lin = nullptr;
   std::mutex enqueue_mu;
 };
 constexpr int kMaxSideSets = 32;   // per device; beyond this a call runs on one stream
@@ -72,12 +72,11 @@ SideSet* side_resources(cudaStream_t caller, bool* cuda_failed) {
     ok = cudaStreamCreateWithFlags(&d.side[i], cudaStreamNonBlocking) == cudaSuccess;
   ok = ok && cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming) == cudaSuccess &&
        cudaEventCreateWithFlags(&d.join_gate, cudaEventDisableTiming) == cudaSuccess &&
-       cudaEventCreateWithFlags(&d.join_lin, cudaEventDisableTiming) == cudaSuccess &&
-       cudaEventCreateWithFlags(&d.kbar_ready, cudaEventDisableTiming) == cudaSuccess;
+       cudaEventCreateWithFlags(&d.join_lin, cudaEventDisableTiming) == cudaSuccess;
   if (!ok) {
     for (cudaStream_t& x : d.side)
       if (x != nullptr) { cudaStreamDestroy(x); x = nullptr; }
-    for (cudaEvent_t* e : {&d.fork, &d.join_gate, &d.join_lin, &d.kbar_ready})
+    for (cudaEvent_t* e : {&d.fork, &d.join_gate, &d.join_lin})
       if (*e != nullptr) { cudaEventDestroy(*e); *e = nullptr; }
     *cuda_failed = true;
     return nullptr;
@@ -622,20 +621,11 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   Rope3D rope;
   if (a->rope3d) rope = make_rope3d(d, a->F, a->Hh, a->Wh, a->rope_base);
   at.rope = rope;
-  // Top-K without dropping: the state kernel, which streams K anyway, also
-  // forms the K block means the selection needs, and the selection pools
-  // only Q (K is read once per layer).  With dropping a dropped sample's
-  // state is skipped, so the selection pools K itself.
-  const bool kbar_in_state = a->mode == SALAD_MODE_TOPK && !(at.drop > 0.0f);
-  double* kb64 = nullptr;
-  float* kb32 = nullptr;
-  if (kbar_in_state) select_kbar(ws + L.sel, B, H, N, d, &kb64, &kb32);
-  cudaEvent_t kbar_ev = (kbar_in_state && dv != nullptr) ? dv->kbar_ready : nullptr;
   void* olin = ws + L.olin;
   if (!full) {
     if (ok)
       check(launch_linear_state(cl, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, a->w_lin, G, drop,
-                                rope, kb64, kb32, kbar_ev));
+                                rope));
     at.Gimg = G;
     at.Z = Z;
   } else {
@@ -643,7 +633,7 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
     // runs plain and the projection GEMM adds s_b (O_l W) afterwards.
     if (ok)
       check(launch_linear_state(cl, a->k, a->v, B, H, N, d, Hst, Z, ws + L.lin, nullptr, nullptr,
-                                drop, rope, kb64, kb32, kbar_ev));
+                                drop, rope));
     if (ok) check(launch_linear_apply(cl, a->q, Hst, Z, a->eps, B, H, N, d, olin, rope));
   }
   if (dv != nullptr) check(cudaEventRecord(dv->join_lin, cl.stream));
@@ -653,13 +643,7 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
     int32_t* idx = a->idx_out != nullptr ? a->idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
     int32_t* lists = reinterpret_cast<int32_t*>(ws + L.lists);
     int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
-    if (ok) {
-      if (kbar_in_state)   // with one stream, the state kernel was enqueued before
-        check(launch_select_q(c, a->q, B, H, N, d, a->topk, idx, ws + L.sel, lists, counts,
-                              kbar_ev));
-      else
-        check(launch_select(c, a->q, a->k, B, H, N, d, a->topk, idx, ws + L.sel, lists, counts));
-    }
+    if (ok) check(launch_select(c, a->q, a->k, B, H, N, d, a->topk, idx, ws + L.sel, lists, counts));
     at.mode = kModeTopk;
     at.lists = lists;
     at.counts = counts;

@@ -32,15 +32,6 @@ size_t select_ws_bytes(int B, int H, int N, int d, int block);
 cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
                           int topk, int32_t* idx, void* ws, int32_t* lists = nullptr,
                           int32_t* counts = nullptr);
-// The same in two parts, for a caller that forms the K means elsewhere
-// (launch_linear_state): select_kbar gives their place in the select
-// workspace; launch_select_q pools Q only and then selects.
-void select_kbar(void* ws, int B, int H, int N, int d, double** kbar64, float** kbar32);
-// kbar_ready (optional): the stream waits for it between the pooling of Q and
-// the selection.
-cudaError_t launch_select_q(const Ctx& c, const void* q, int B, int H, int N, int d, int topk,
-                            int32_t* idx, void* ws, int32_t* lists, int32_t* counts,
-                            cudaEvent_t kbar_ready);
 // Merge the kept lists of query blocks (2p, 2p+1) into one ascending list of
 // entries (j | mask << 16), mask bit 0 = block 2p keeps j, bit 1 = block 2p+1.
 size_t pairs_ws_bytes(int B, int H, int N, int topk);
@@ -91,18 +82,10 @@ struct BranchDrop {
   float gate_override = 0.0f;
   float thr = 0.0f;
 };
-// kbar64/kbar32 (both or neither): the per-block means of K [B*H][nb][d]
-// (valid rows), formed from the tiles the state streams anyway, so that the
-// selection need not read K again.  Not formed for a sample whose branch is
-// dropped (its CTAs leave at once): pass null when dropping is on.
-// state_done (optional) is recorded once the state kernel (and so the means)
-// is done, before the reduction that follows it.
 cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int B, int H, int N,
                                 int d, float* Hst, float* Z, void* ws,
                                 const void* w_lin = nullptr, void* Gimg = nullptr,
-                                BranchDrop drop = BranchDrop(), Rope3D rope = Rope3D(),
-                                double* kbar64 = nullptr, float* kbar32 = nullptr,
-                                cudaEvent_t state_done = nullptr);
+                                BranchDrop drop = BranchDrop(), Rope3D rope = Rope3D());
 cudaError_t launch_linear_apply(const Ctx& c, const void* q, const float* Hst, const float* Z,
                                 float eps, int B, int H, int N, int d, void* o,
                                 Rope3D rope = Rope3D());

@@ -48,8 +48,7 @@ template <int D>
 __global__ void __launch_bounds__(192, 1) linear_state_kernel(
     const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv, int nblk,
     int blocks_per_cta, int ctas_per_head, float* __restrict__ partH, float* __restrict__ partZ,
-    unsigned* err, unsigned long long wait_ns, BranchDrop drop, int H, Rope3D rope, int N,
-    double* __restrict__ kbar64, float* __restrict__ kbar32) {
+    unsigned* err, unsigned long long wait_ns, BranchDrop drop, int H, Rope3D rope, int N) {
   using C = LS<D>;
   // A sample whose linear branch is dropped needs no state: the whole CTA
   // leaves before touching shared memory, barriers or TMEM.
@@ -61,10 +60,8 @@ __global__ void __launch_bounds__(192, 1) linear_state_kernel(
   unsigned char* zero_slab = sm + C::kStages * C::kStage;
   float* zred = reinterpret_cast<float*>(zero_slab + C::kZero);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(zred) + C::kRed);
-  // bars: full[0..S), relu[S..2S), empty[2S..3S), acc, drain, col[3S+2..4S+2); then tmem
-  // holder, abort
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 4 * C::kStages + 2);
-  static_assert((4 * C::kStages + 2) * 8 + 8 <= C::kBars, "barrier region");
+  // bars: full[0..S), relu[S..2S), empty[2S..3S), acc, drain; then tmem holder, abort
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * C::kStages + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   double* theta = reinterpret_cast<double*>(reinterpret_cast<unsigned char*>(bars) + C::kBars);
 
@@ -79,7 +76,6 @@ __global__ void __launch_bounds__(192, 1) linear_state_kernel(
   auto empty = [&](int s) { return smem_u32(bars + 2 * C::kStages + s); };
   const uint32_t acc_bar = smem_u32(bars + 3 * C::kStages);
   const uint32_t drain_bar = smem_u32(bars + 3 * C::kStages + 1);
-  auto col_bar = [&](int s) { return smem_u32(bars + 3 * C::kStages + 2 + s); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -89,7 +85,6 @@ __global__ void __launch_bounds__(192, 1) linear_state_kernel(
     }
     mbar_init(acc_bar, 1);
     mbar_init(drain_bar, 1);
-    for (int s = 0; s < C::kStages; ++s) mbar_init(col_bar(s), 4);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_map(&mk);
@@ -186,32 +181,6 @@ __global__ void __launch_bounds__(192, 1) linear_state_kernel(
         break;
       }
       unsigned char* ktile = stage_base + s * C::kStage;
-      if (kbar64 != nullptr) {
-        // The tile is one 64-token block: its mean of K (valid rows; rows
-        // past N were zero-filled by the load), summed in float64 down each
-        // channel before the in-place ReLU below rewrites the tile.
-        const int blk = b0 + t;
-        if (tid < D) {
-          const unsigned char* col = ktile + (tid / 64) * kSlab;
-          double acc = 0.0;
-#pragma unroll 8
-          for (int r = 0; r < 64; ++r)
-            acc += static_cast<double>(__bfloat162float(
-                *reinterpret_cast<const __nv_bfloat16*>(col + sw128_offset(r, tid % 64))));
-          const double mean = acc / static_cast<double>(min(64, N - blk * 64));
-          const long long o = (static_cast<long long>(bh) * nblk + blk) * D + tid;
-          kbar64[o] = mean;
-          kbar32[o] = static_cast<float>(mean);
-        }
-        // Every warp has read the raw tile before any rewrites it.
-        __syncwarp();
-        if (lane == 0) mbar_arrive(col_bar(s));
-        if (!__all_sync(0xffffffffu, mbar_wait(col_bar(s), (t / C::kStages) & 1, wait_ns, abort_flag))) {
-          raise_timeout(err, abort_flag);
-          ok = false;
-          break;
-        }
-      }
 #pragma unroll
       for (int i = 0; i < (D / 64) * 4; ++i) {
         const int half = i / 4;
@@ -530,8 +499,7 @@ size_t linear_state_ws_bytes(int B, int H, int N, int d) {
 
 cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int B, int H, int N,
                                 int d, float* Hst, float* Z, void* ws, const void* w_lin,
-                                void* Gimg, BranchDrop drop, Rope3D rope, double* kbar64,
-                                float* kbar32, cudaEvent_t state_done) {
+                                void* Gimg, BranchDrop drop, Rope3D rope) {
   const LSPlan p = ls_plan(B, H, N, c.num_sms < 256 ? c.num_sms : 256);
   const int BH = B * H;
   const size_t parts = static_cast<size_t>(BH) * p.ctas_per_head;
@@ -549,18 +517,17 @@ cudaError_t launch_linear_state(const Ctx& c, const void* k, const void* v, int 
     if (e != cudaSuccess) return e;
     linear_state_kernel<128><<<grid, 192, LS<128>::kSmem, c.stream>>>(
         mk, mv, p.nblk, p.blocks_per_cta, p.ctas_per_head, partH, partZ, c.err, c.wait_ns, drop,
-        H, rope, N, kbar64, kbar32);
+        H, rope, N);
   } else {
     e = cudaFuncSetAttribute(linear_state_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              LS<64>::kSmem);
     if (e != cudaSuccess) return e;
     linear_state_kernel<64><<<grid, 192, LS<64>::kSmem, c.stream>>>(
         mk, mv, p.nblk, p.blocks_per_cta, p.ctas_per_head, partH, partZ, c.err, c.wait_ns, drop,
-        H, rope, N, kbar64, kbar32);
+        H, rope, N);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (state_done != nullptr && (e = cudaEventRecord(state_done, c.stream)) != cudaSuccess) return e;
   if (w_lin == nullptr) {
     linear_reduce_kernel<<<dim3((d * d + 255) / 256, BH), 256, 0, c.stream>>>(
         partH, partZ, d, p.ctas_per_head, Hst, Z);

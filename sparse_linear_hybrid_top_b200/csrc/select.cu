@@ -620,10 +620,9 @@ size_t select_ws_bytes(int B, int H, int N, int d, int block) {
 
 namespace {
 
-// Pools Q (z = 0) and, when k is given, K (z = 1), then selects.
+// Pools Q (z = 0) and K (z = 1), then selects.
 cudaError_t pool_and_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
-                            int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts,
-                            cudaEvent_t kbar_ready) {
+                            int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts) {
   const SelectLayout L = select_layout(B, H, N, d, kBlock);
   char* base = static_cast<char*>(ws);
   double* qbar = reinterpret_cast<double*>(base + L.qbar);
@@ -632,7 +631,7 @@ cudaError_t pool_and_select(const Ctx& c, const void* q, const void* k, int B, i
   float* kbar32 = reinterpret_cast<float*>(base + L.kbar32);
   const int nb = (N + kBlock - 1) / kBlock;
   const int BH = B * H;
-  dim3 pg(nb, BH, k != nullptr ? 2 : 1);
+  dim3 pg(nb, BH, 2);
   if (d == 128)
     pool_kernel<128><<<pg, 128, 0, c.stream>>>(static_cast<const uint4*>(q),
                                                 static_cast<const uint4*>(k), N, nb, qbar, kbar,
@@ -643,8 +642,6 @@ cudaError_t pool_and_select(const Ctx& c, const void* q, const void* k, int B, i
                                                qbar32, kbar32);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (kbar_ready != nullptr && (e = cudaStreamWaitEvent(c.stream, kbar_ready, 0)) != cudaSuccess)
-    return e;
   if (d == 128)
     return sel_smem_bytes<128, 16>(nb) <= kSelSmemCap
                ? launch_select_fused<128, 16>(c, qbar32, kbar32, qbar, kbar, BH, nb, topk, idx,
@@ -662,20 +659,7 @@ cudaError_t pool_and_select(const Ctx& c, const void* q, const void* k, int B, i
 
 cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
                           int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts) {
-  return pool_and_select(c, q, k, B, H, N, d, topk, idx, ws, lists, counts, nullptr);
-}
-
-void select_kbar(void* ws, int B, int H, int N, int d, double** kbar64, float** kbar32) {
-  const SelectLayout L = select_layout(B, H, N, d, kBlock);
-  char* base = static_cast<char*>(ws);
-  *kbar64 = reinterpret_cast<double*>(base + L.kbar);
-  *kbar32 = reinterpret_cast<float*>(base + L.kbar32);
-}
-
-cudaError_t launch_select_q(const Ctx& c, const void* q, int B, int H, int N, int d, int topk,
-                            int32_t* idx, void* ws, int32_t* lists, int32_t* counts,
-                            cudaEvent_t kbar_ready) {
-  return pool_and_select(c, q, nullptr, B, H, N, d, topk, idx, ws, lists, counts, kbar_ready);
+  return pool_and_select(c, q, k, B, H, N, d, topk, idx, ws, lists, counts);
 }
 
 size_t pairs_ws_bytes(int B, int H, int N, int topk) {

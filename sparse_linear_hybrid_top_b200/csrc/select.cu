@@ -28,23 +28,27 @@ constexpr int kBlock = 64;
 
 // ------------------------------------------------------------------ pool --
 // CTA (i, bh, z): the mean of block i of head bh of Q (z = 0) or K (z = 1),
-// summed in float64 over the valid rows, written in float64 and rounded once
-// to float32 (the selection's float32 pass reads the latter).
+// summed in float64 over the valid rows and written in float64; rounded once
+// to float32 for the selection's float32 pass: Q row-major [bh][i][c], K
+// channel-major [bh][c][i] (row length nbs, so a chunk of channels is a run
+// of contiguous rows), with the squared norm of each rounded K mean.
 template <int D>
 __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
                                                    const uint4* __restrict__ k, int N, int nb,
-                                                   double* __restrict__ qbar,
+                                                   int nbs, double* __restrict__ qbar,
                                                    double* __restrict__ kbar,
                                                    float* __restrict__ qbar32,
-                                                   float* __restrict__ kbar32) {
+                                                   float* __restrict__ kbar32t,
+                                                   float* __restrict__ kn2) {
   constexpr int CPR = D / 8;     // 16-byte chunks per row
   constexpr int RPI = 128 / CPR; // rows per iteration
   __shared__ double red[RPI][D];
+  __shared__ float nred[4];
   const int i = blockIdx.x;
   const long long bh = blockIdx.y;
-  const uint4* src = blockIdx.z == 0 ? q : k;
-  double* dst = blockIdx.z == 0 ? qbar : kbar;
-  float* dst32 = blockIdx.z == 0 ? qbar32 : kbar32;
+  const bool is_k = blockIdx.z != 0;
+  const uint4* src = is_k ? k : q;
+  double* dst = is_k ? kbar : qbar;
   const int row0 = i * kBlock;
   const int rows = min(kBlock, N - row0);
   const int chunk = threadIdx.x % CPR;
@@ -67,13 +71,27 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
 #pragma unroll
   for (int e = 0; e < 8; ++e) red[rsub][chunk * 8 + e] = acc[e];
   __syncthreads();
+  float part = 0.0f;
   for (int c = threadIdx.x; c < D; c += 128) {
     double s = 0.0;
 #pragma unroll
     for (int r = 0; r < RPI; ++r) s += red[r][c];
     const double m = s / static_cast<double>(rows);
     dst[(bh * nb + i) * D + c] = m;
-    dst32[(bh * nb + i) * D + c] = static_cast<float>(m);
+    const float m32 = static_cast<float>(m);
+    if (is_k) {
+      kbar32t[(bh * D + c) * static_cast<long long>(nbs) + i] = m32;
+      part = fmaf(m32, m32, part);
+    } else {
+      qbar32[(bh * nb + i) * D + c] = m32;
+    }
+  }
+  if (is_k) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((threadIdx.x & 31) == 0) nred[threadIdx.x >> 5] = part;
+    __syncthreads();
+    if (threadIdx.x == 0) kn2[bh * nb + i] = (nred[0] + nred[1]) + (nred[2] + nred[3]);
   }
 }
 
@@ -113,11 +131,14 @@ struct SelCfg {
   static constexpr int kRG = RB / 4;               // 4-row groups
   static constexpr int kCG = kThreads / kRG;       // 4-column groups
   static constexpr int kCT = 4 * kCG;              // columns per tile
-  static constexpr int kKC = RB == 16 ? 16 : 8;    // channels per staged chunk
-  static constexpr int kLoadCols = kCT / kThreads; // columns each thread stages
+  static constexpr int kKC = 8;                    // channels per staged chunk
+  static constexpr int kRing = 4;                  // chunks in flight (cp.async stages)
   static constexpr int kCandMax = 64;              // float64 candidates buffered per warp
+  // The staging ring, reused after the scores by the float64 recheck.
+  static constexpr int kStageFloats = kRing * kKC * kCT;
   static_assert(kCG >= 32 && kCG % 32 == 0, "a warp spans one row group");
   static_assert(D % kKC == 0, "chunking");
+  static_assert(kStageFloats * 4 >= kWarps * (256 * 4 + kCandMax * 12), "recheck scratch");
 };
 
 template <int D, int RB>
@@ -126,11 +147,9 @@ size_t sel_smem_bytes(int nb) {
   const size_t nbp = (static_cast<size_t>(nb) + 3) & ~static_cast<size_t>(3);
   const size_t nw = (static_cast<size_t>(nb) + 31) / 32;
   return static_cast<size_t>(D) * RB * 4            // qs [D][RB]
-         + 2 * C::kKC * C::kCT * 4                  // ks [2][KC][CT]
+         + static_cast<size_t>(C::kStageFloats) * 4 // ks [ring][KC][CT], later the recheck scratch
          + RB * nbp * 4                             // scores [RB][nbp]
          + RB * nw * 4                              // kept bitmaps [RB][nw]
-         + C::kWarps * 256 * 4                      // radix histograms
-         + C::kWarps * C::kCandMax * 12             // candidate j and float64 score
          + (C::kThreads + RB + 8) * 4;              // norm reduction, row norms
 }
 
@@ -151,24 +170,23 @@ __device__ __forceinline__ double score64(const double* __restrict__ qrow,
   return acc;
 }
 
-// Radix select over the keys of `n` items for which `take(j)` holds: finds
-// the digits of the `want`-th largest key, 8 bits per pass from the top.
-// Returns the full key (all passes run) or, when `early` is set and every
-// key sharing the prefix is wanted, the prefix with its mask; `want` is
-// updated to the number still wanted among keys equal to the (masked)
-// prefix.  Warp-collective; hist: 256 words of this warp.
-template <typename Key, typename KeyOf>
-__device__ __forceinline__ void radix_select(int n, int& want, Key& prefix, Key& pmask,
-                                             unsigned* hist, int lane, bool early, KeyOf key_of) {
-  constexpr int kBits = 8 * sizeof(Key);
+// Radix select over 64-bit keys of the items j in [0, n) for which key_of
+// reports ok: finds, 8 bits per pass from the top, the digits of the
+// `want`-th largest key; stops early once every key sharing the prefix is
+// wanted.  On return `want` is the number still wanted among keys equal to
+// the (masked) prefix.  Warp-collective; hist: 256 words of this warp.
+template <typename KeyOf>
+__device__ __forceinline__ void radix_select64(int n, int& want, unsigned long long& prefix,
+                                               unsigned long long& pmask, unsigned* hist, int lane,
+                                               KeyOf key_of) {
   prefix = 0;
   pmask = 0;
-  for (int shift = kBits - 8; shift >= 0; shift -= 8) {
+  for (int shift = 56; shift >= 0; shift -= 8) {
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
     for (int j = lane; j < n; j += 32) {
       bool ok;
-      const Key key = key_of(j, ok);
+      const unsigned long long key = key_of(j, ok);
       if (ok && (key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncwarp();
@@ -201,31 +219,41 @@ __device__ __forceinline__ void radix_select(int n, int& want, Key& prefix, Key&
     digit = __shfl_sync(0xffffffffu, digit, owner);
     above = __shfl_sync(0xffffffffu, above, owner);
     want -= static_cast<int>(above);
-    prefix |= static_cast<Key>(digit) << shift;
-    pmask |= static_cast<Key>(0xFF) << shift;
+    prefix |= static_cast<unsigned long long>(digit) << shift;
+    pmask |= 0xFFull << shift;
     const bool settled = hist[digit] == static_cast<unsigned>(want);
     __syncwarp();
-    if (early && settled) return;
+    if (settled) return;
   }
 }
 
-template <int D, int RB>
-__global__ void __launch_bounds__(256) select_fused_kernel(
-    const float* __restrict__ qbar32, const float* __restrict__ kbar32,
-    const double* __restrict__ qbar64, const double* __restrict__ kbar64, int nb, int topk,
-    int32_t* __restrict__ idx, int32_t* __restrict__ lists, int32_t* __restrict__ counts) {
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// VPL: scores of a row each lane keeps in registers (column j = lane + 32 u).
+template <int D, int RB, int VPL>
+__global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
+    const float* __restrict__ qbar32, const float* __restrict__ kbar32t,
+    const float* __restrict__ kn2, const double* __restrict__ qbar64,
+    const double* __restrict__ kbar64, int nb, int nbs, int topk, int32_t* __restrict__ idx,
+    int32_t* __restrict__ lists, int32_t* __restrict__ counts) {
   using C = SelCfg<D, RB>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int nbp = (nb + 3) & ~3;
   const int nw = (nb + 31) / 32;
   float* qs = reinterpret_cast<float*>(smem_raw);                        // [D][RB]
-  float* ks = qs + D * RB;                                                // [2][KC][CT]
-  float* sc = ks + 2 * C::kKC * C::kCT;                                   // [RB][nbp]
+  float* ks = qs + D * RB;                                                // [ring][KC][CT]
+  float* sc = ks + C::kStageFloats;                                       // [RB][nbp]
   unsigned* bits = reinterpret_cast<unsigned*>(sc + RB * nbp);            // [RB][nw]
-  unsigned* hist_all = bits + RB * nw;                                    // [warps][256]
-  double* cand_s = reinterpret_cast<double*>(hist_all + C::kWarps * 256); // [warps][CandMax]
-  int* cand_j = reinterpret_cast<int*>(cand_s + C::kWarps * C::kCandMax); // [warps][CandMax]
-  float* red = reinterpret_cast<float*>(cand_j + C::kWarps * C::kCandMax); // [threads]
+  float* red = reinterpret_cast<float*>(bits + RB * nw);                  // [threads]
   float* qn = red + C::kThreads;                                          // [RB] row norms
   float* kmax_s = qn + RB;                                                // [1]
 
@@ -234,95 +262,81 @@ __global__ void __launch_bounds__(256) select_fused_kernel(
   const int i0 = blockIdx.x * RB;
   const int rows = min(RB, nb - i0);
   const float* qb = qbar32 + (bh * nb + i0) * D;
-  const float* kb = kbar32 + bh * nb * D;
+  const float* kt = kbar32t + bh * D * static_cast<long long>(nbs);
 
-  // ---- stage the chunk's query means, transposed (invalid rows are 0)
+  // ---- phase 1: float32 scores.  Chunk ch = (column tile, KC channels): KC
+  // rows of CT key means from the channel-major copy, streamed by cp.async
+  // through a ring of kRing chunks, kRing - 1 in flight ahead of the one
+  // being multiplied.
+  const int ty = tid / C::kCG, tx = tid % C::kCG;
+  const int ntile = (nb + C::kCT - 1) / C::kCT;
+  constexpr int kChunks = D / C::kKC;
+  constexpr int kCopies = C::kKC * C::kCT / 4;   // 16-byte copies per chunk
+  const int nch = ntile * kChunks;
+  auto issue = [&](int ch) {
+    float* dst = ks + (ch % C::kRing) * C::kKC * C::kCT;
+    const int j0 = (ch / kChunks) * C::kCT, c0 = (ch % kChunks) * C::kKC;
+    for (int e = tid; e < kCopies; e += C::kThreads) {
+      const int row = e / (C::kCT / 4), col = 4 * (e % (C::kCT / 4));
+      cp_async16(smem_u32(dst + row * C::kCT + col),
+                 kt + static_cast<long long>(c0 + row) * nbs + j0 + col);
+    }
+  };
+#pragma unroll
+  for (int s0 = 0; s0 < C::kRing - 1; ++s0) {
+    if (s0 < nch) issue(s0);
+    cp_async_commit();
+  }
+  // The chunk's query means, transposed (invalid rows are 0), meanwhile.
   for (int e = tid; e < D * RB; e += C::kThreads) {
     const int r = e / D, c = e % D;
     qs[c * RB + r] = r < rows ? __ldg(qb + static_cast<long long>(r) * D + c) : 0.0f;
   }
-
-  // ---- phase 1: float32 scores
-  const int ty = tid / C::kCG, tx = tid % C::kCG;
-  const int ntile = (nb + C::kCT - 1) / C::kCT;
-  constexpr int kChunks = D / C::kKC;
-  const int nch = ntile * kChunks;
-  float4 stage[C::kLoadCols][C::kKC / 4];
-  float kn2[C::kLoadCols];
-  float kmax2 = 0.0f;
-  auto fetch = [&](int ch) {
-    const int j0 = (ch / kChunks) * C::kCT, c0 = (ch % kChunks) * C::kKC;
-#pragma unroll
-    for (int u = 0; u < C::kLoadCols; ++u) {
-      const int j = j0 + tid + u * C::kThreads;
-      const float4* src = reinterpret_cast<const float4*>(kb + static_cast<long long>(j) * D + c0);
-#pragma unroll
-      for (int v = 0; v < C::kKC / 4; ++v)
-        stage[u][v] = j < nb ? __ldg(src + v) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  };
-  auto stash = [&](int ch) {
-    float* dst = ks + (ch & 1) * C::kKC * C::kCT;
-    if (ch % kChunks == 0) {
-#pragma unroll
-      for (int u = 0; u < C::kLoadCols; ++u) kn2[u] = 0.0f;
-    }
-#pragma unroll
-    for (int u = 0; u < C::kLoadCols; ++u) {
-      const int jj = tid + u * C::kThreads;
-#pragma unroll
-      for (int v = 0; v < C::kKC / 4; ++v) {
-        const float4 x = stage[u][v];
-        dst[(4 * v + 0) * C::kCT + jj] = x.x;
-        dst[(4 * v + 1) * C::kCT + jj] = x.y;
-        dst[(4 * v + 2) * C::kCT + jj] = x.z;
-        dst[(4 * v + 3) * C::kCT + jj] = x.w;
-        kn2[u] = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, kn2[u]))));
-      }
-    }
-    if (ch % kChunks == kChunks - 1) {
-#pragma unroll
-      for (int u = 0; u < C::kLoadCols; ++u) kmax2 = fmaxf(kmax2, kn2[u]);
-    }
-  };
   float acc[4][4];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a2 = 0; a2 < 4; ++a2)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-  fetch(0);
-  stash(0);
-  __syncthreads();
+    for (int b2 = 0; b2 < 4; ++b2) acc[a2][b2] = 0.0f;
   for (int ch = 0; ch < nch; ++ch) {
-    if (ch + 1 < nch) fetch(ch + 1);
-    const float* kbuf = ks + (ch & 1) * C::kKC * C::kCT;
+    cp_async_wait<C::kRing - 2>();   // this thread's copies of chunk ch have landed
+    __syncthreads();                 // everyone's have; chunk ch - 1 is no longer read
+    if (ch + C::kRing - 1 < nch) issue(ch + C::kRing - 1);
+    cp_async_commit();
+    const float* kbuf = ks + (ch % C::kRing) * C::kKC * C::kCT;
     const int c0 = (ch % kChunks) * C::kKC;
+    float4 qv[C::kKC], kv[C::kKC];
 #pragma unroll
     for (int c = 0; c < C::kKC; ++c) {
-      const float4 qv = *reinterpret_cast<const float4*>(qs + (c0 + c) * RB + 4 * ty);
-      const float4 kv = *reinterpret_cast<const float4*>(kbuf + c * C::kCT + 4 * tx);
-      const float q4[4] = {qv.x, qv.y, qv.z, qv.w};
-      const float k4[4] = {kv.x, kv.y, kv.z, kv.w};
+      qv[c] = *reinterpret_cast<const float4*>(qs + (c0 + c) * RB + 4 * ty);
+      kv[c] = *reinterpret_cast<const float4*>(kbuf + c * C::kCT + 4 * tx);
+    }
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+    for (int c = 0; c < C::kKC; ++c) {
+      const float q4[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
+      const float k4[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(q4[a], k4[b], acc[a][b]);
+      for (int a2 = 0; a2 < 4; ++a2)
+#pragma unroll
+        for (int b2 = 0; b2 < 4; ++b2) acc[a2][b2] = fmaf(q4[a2], k4[b2], acc[a2][b2]);
     }
     if (ch % kChunks == kChunks - 1) {
       const int j = (ch / kChunks) * C::kCT + 4 * tx;
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
+      for (int a2 = 0; a2 < 4; ++a2) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          if (j + b < nb) sc[(4 * ty + a) * nbp + j + b] = acc[a][b];
-          acc[a][b] = 0.0f;
+        for (int b2 = 0; b2 < 4; ++b2) {
+          if (j + b2 < nb) sc[(4 * ty + a2) * nbp + j + b2] = acc[a2][b2];
+          acc[a2][b2] = 0.0f;
         }
       }
     }
-    if (ch + 1 < nch) stash(ch + 1);
-    __syncthreads();
   }
-  // Largest key-mean norm of the head and each row's query-mean norm.
+  cp_async_wait<0>();
+  __syncthreads();   // the ring is free for the recheck scratch
+  // Largest key-mean norm of the head (from the pooling pass) and each row's
+  // query-mean norm.
+  float kmax2 = 0.0f;
+  for (int j = tid; j < nb; j += C::kThreads) kmax2 = fmaxf(kmax2, __ldg(kn2 + bh * nb + j));
   red[tid] = kmax2;
   if (tid < RB) {
     float n2 = 0.0f;
@@ -341,38 +355,48 @@ __global__ void __launch_bounds__(256) select_fused_kernel(
   const double kmax = kmax_s[0];
 
   // ---- phase 2: per row (warp), the k-th largest float32 score, the band
-  // and, where needed, the float64 decision.
-  unsigned* hist = hist_all + warp * 256;
-  double* cs = cand_s + warp * C::kCandMax;
-  int* cj = cand_j + warp * C::kCandMax;
+  // and, where needed, the float64 decision.  The staging buffers now hold
+  // each warp's radix histogram and candidate buffer.
+  unsigned* hist = reinterpret_cast<unsigned*>(ks) + warp * (256 + C::kCandMax * 3);
+  double* cs = reinterpret_cast<double*>(hist + 256);
+  int* cj = reinterpret_cast<int*>(cs + C::kCandMax);
   for (int r = warp; r < RB; r += C::kWarps) {
     unsigned* kept = bits + r * nw;
     for (int w = lane; w < nw; w += 32) kept[w] = 0u;
     __syncwarp();
     if (r >= rows) continue;
     const float* srow = sc + r * nbp;
+    // The row's scores in registers: column j = lane + 32 u (-inf past nb).
+    float vals[VPL];
+#pragma unroll
+    for (int u = 0; u < VPL; ++u) {
+      const int j = lane + 32 * u;
+      vals[u] = j < nb ? srow[j] : -INFINITY;
+    }
     // Bracket the k-th largest float32 score T: cnt(>= lo) >= topk > cnt(>= hi),
-    // so lo <= T < hi, by bisection on the value (a ballot-free count per
-    // step) until the bracket is narrower than the bound E allows.
+    // so lo <= T < hi, by bisection on the value until the bracket is
+    // narrower than the bound E allows.
     const double qnr = static_cast<double>(qn[r]);
     const bool wide = !(qnr < 1e18 && kmax < 1e18);
     const double E = (D + 8) * 5.9604644775390625e-8 * 1.05 * qnr * kmax + D * 2.4e-38;
     auto count_ge = [&](float t) -> int {
       unsigned cnt = 0;
-      for (int j = lane; j < nb; j += 32) cnt += srow[j] >= t ? 1u : 0u;
+#pragma unroll
+      for (int u = 0; u < VPL; ++u) cnt += vals[u] >= t ? 1u : 0u;
       return static_cast<int>(__reduce_add_sync(0xffffffffu, cnt));
     };
     float mn = INFINITY, mx = -INFINITY;
-    for (int j = lane; j < nb; j += 32) {
-      mn = fminf(mn, srow[j]);
-      mx = fmaxf(mx, srow[j]);
+#pragma unroll
+    for (int u = 0; u < VPL; ++u) {
+      if (lane + 32 * u < nb) mn = fminf(mn, vals[u]);
+      mx = fmaxf(mx, vals[u]);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
-    double blo = mn, bhi = mx;   // the bracket of T
+    double blo = mx, bhi = mx;   // T = mx when at least topk scores tie at the maximum
     if (!wide && count_ge(mx) < topk) {
       float lo = mn, hi = mx;
       for (int it = 0; it < 64 && static_cast<double>(hi) - lo > 0.5 * E; ++it) {
@@ -382,36 +406,37 @@ __global__ void __launch_bounds__(256) select_fused_kernel(
       }
       blo = lo;
       bhi = hi;
-    } else {
-      blo = bhi = mx;   // T = mx (ties at the maximum), or the band is everything
     }
     // The float64 k-th largest lies within [blo - E, bhi + E]: above
     // bhi + 2E a block is kept for certain, below blo - 2E dropped.
     const double lo = wide ? -INFINITY : blo - 2.0 * E, hi = wide ? INFINITY : bhi + 2.0 * E;
-    // Certain members (above the band) and candidates (inside it).
+    auto is_cand_v = [&](float v) {
+      const double dv = static_cast<double>(v);
+      return !(dv > hi) && (wide || dv >= lo);
+    };
+    // Certain members (word u of the kept bitmap is the ballot over u) and
+    // the candidates.
     int n_in = 0, n_cand = 0;
-    for (int j0 = 0; j0 < nb; j0 += 32) {
-      const int j = j0 + lane;
-      const double v = j < nb ? static_cast<double>(srow[j]) : -INFINITY;
-      const bool in = j < nb && v > hi;
-      const bool cand = j < nb && !(v > hi) && (wide || v >= lo);
+    unsigned cand_w[VPL];
+#pragma unroll
+    for (int u = 0; u < VPL; ++u) {
+      const bool valid = lane + 32 * u < nb;
+      const bool in = valid && static_cast<double>(vals[u]) > hi;
+      const bool cand = valid && is_cand_v(vals[u]);
       const unsigned bin = __ballot_sync(0xffffffffu, in);
-      if (lane == 0) kept[j0 / 32] = bin;
+      cand_w[u] = __ballot_sync(0xffffffffu, cand);
+      if (lane == 0 && u < nw) kept[u] = bin;
       n_in += __popc(bin);
-      n_cand += __popc(__ballot_sync(0xffffffffu, cand));
+      n_cand += __popc(cand_w[u]);
     }
     __syncwarp();
     const int need = topk - n_in;   // 0 <= need <= n_cand
-    auto is_cand = [&](int j) {
-      const double v = static_cast<double>(srow[j]);
-      return !(v > hi) && (wide || v >= lo);
-    };
     if (need == n_cand) {
       // Every candidate is kept: no float64 needed.
-      for (int j0 = 0; j0 < nb; j0 += 32) {
-        const int j = j0 + lane;
-        const unsigned b = __ballot_sync(0xffffffffu, j < nb && is_cand(j));
-        if (lane == 0) kept[j0 / 32] |= b;
+      if (lane == 0) {
+#pragma unroll
+        for (int u = 0; u < VPL; ++u)
+          if (u < nw) kept[u] |= cand_w[u];
       }
     } else if (need > 0) {
       const double* qrow = qbar64 + (bh * nb + i0 + r) * D;
@@ -420,11 +445,10 @@ __global__ void __launch_bounds__(256) select_fused_kernel(
         // Buffer the candidates (ascending j) with their float64 scores and
         // keep the `need` best by (score desc, j asc).
         int nc = 0;
-        for (int j0 = 0; j0 < nb; j0 += 32) {
-          const int j = j0 + lane;
-          const bool cand = j < nb && is_cand(j);
-          const unsigned b = __ballot_sync(0xffffffffu, cand);
-          if (cand) cj[nc + __popc(b & ((1u << lane) - 1u))] = j;
+#pragma unroll
+        for (int u = 0; u < VPL; ++u) {
+          const unsigned b = cand_w[u];
+          if ((b >> lane) & 1u) cj[nc + __popc(b & ((1u << lane) - 1u))] = lane + 32 * u;
           nc += __popc(b);
         }
         __syncwarp();
@@ -445,13 +469,13 @@ __global__ void __launch_bounds__(256) select_fused_kernel(
       } else {
         // Many candidates (near-degenerate rows, e.g. exact ties): a radix
         // select over their float64 keys, each key recomputed when read.
+        auto is_cand = [&](int j) { return is_cand_v(srow[j]); };
         int want64 = need;
         unsigned long long pfx = 0, pm = 0;
-        radix_select<unsigned long long>(nb, want64, pfx, pm, hist, lane, true,
-                                         [&](int j, bool& ok) {
-                                           ok = is_cand(j);
-                                           return ok ? dkey(score64<D>(qrow, kb64, j)) : 0ull;
-                                         });
+        radix_select64(nb, want64, pfx, pm, hist, lane, [&](int j, bool& ok) {
+          ok = is_cand(j);
+          return ok ? dkey(score64<D>(qrow, kb64, j)) : 0ull;
+        });
         int eq_seen = 0;
         for (int j0 = 0; j0 < nb; j0 += 32) {
           const int j = j0 + lane;
@@ -468,16 +492,15 @@ __global__ void __launch_bounds__(256) select_fused_kernel(
         __syncwarp();
       }
     }
+    __syncwarp();
     // The kept list, ascending.
     if (idx != nullptr) {
       int32_t* out = idx + (bh * nb + i0 + r) * static_cast<long long>(topk);
       int written = 0;
-      for (int j0 = 0; j0 < nb; j0 += 32) {
-        const int j = j0 + lane;
-        const unsigned word = kept[j0 / 32];
-        const bool keep = j < nb && ((word >> lane) & 1u);
+      for (int w = 0; w < nw; ++w) {
+        const unsigned word = kept[w];
         const int pos = written + __popc(word & ((1u << lane) - 1u));
-        if (keep && pos < topk) out[pos] = j;
+        if (((word >> lane) & 1u) && pos < topk) out[pos] = 32 * w + lane;
         written += __popc(word);
       }
     }
@@ -579,46 +602,59 @@ __global__ void pair_union_kernel(const int32_t* __restrict__ idx, int BH, int n
 }
 
 struct SelectLayout {
-  size_t qbar, kbar, qbar32, kbar32, total;
+  size_t qbar, kbar, qbar32, kbar32t, kn2, total;
+  int nbs;   // row length of the channel-major float32 K means
 };
 SelectLayout select_layout(int B, int H, int N, int d, int block) {
   const size_t nb = (static_cast<size_t>(N) + block - 1) / block;
   const size_t BH = static_cast<size_t>(B) * H;
   SelectLayout L;
+  // Whole 512-column tiles, so a chunk's copies never leave their row.
+  L.nbs = static_cast<int>((nb + 511) / 512 * 512);
   L.qbar = 0;
   L.kbar = L.qbar + align256(BH * nb * d * sizeof(double));
   L.qbar32 = L.kbar + align256(BH * nb * d * sizeof(double));
-  L.kbar32 = L.qbar32 + align256(BH * nb * d * sizeof(float));
-  L.total = L.kbar32 + align256(BH * nb * d * sizeof(float));
+  L.kbar32t = L.qbar32 + align256(BH * nb * d * sizeof(float));
+  L.kn2 = L.kbar32t + align256(BH * d * L.nbs * sizeof(float));
+  L.total = L.kn2 + align256(BH * nb * sizeof(float));
   return L;
 }
 
-template <int D, int RB>
-cudaError_t launch_select_fused(const Ctx& c, const float* q32, const float* k32,
-                                const double* q64, const double* k64, int BH, int nb, int topk,
-                                int32_t* idx, int32_t* lists, int32_t* counts) {
+template <int D, int RB, int VPL>
+cudaError_t launch_select_fused(const Ctx& c, const float* q32, const float* k32t,
+                                const float* kn2, const double* q64, const double* k64, int BH,
+                                int nb, int nbs, int topk, int32_t* idx, int32_t* lists,
+                                int32_t* counts) {
   const size_t smem = sel_smem_bytes<D, RB>(nb);
-  cudaError_t e = cudaFuncSetAttribute(select_fused_kernel<D, RB>,
+  cudaError_t e = cudaFuncSetAttribute(select_fused_kernel<D, RB, VPL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid((nb + RB - 1) / RB, BH);
-  select_fused_kernel<D, RB><<<grid, SelCfg<D, RB>::kThreads, smem, c.stream>>>(
-      q32, k32, q64, k64, nb, topk, idx, lists, counts);
+  select_fused_kernel<D, RB, VPL><<<grid, SelCfg<D, RB>::kThreads, smem, c.stream>>>(
+      q32, k32t, kn2, q64, k64, nb, nbs, topk, idx, lists, counts);
   return cudaGetLastError();
 }
 
-// 16 query blocks per CTA while their scores fit next to the staging buffers,
-// else 8 (every nb up to 4096 fits).
-constexpr size_t kSelSmemCap = 200 * 1024;
-
-}  // namespace
-
-size_t select_ws_bytes(int B, int H, int N, int d, int block) {
-  return select_layout(B, H, N, d, block).total;
+// The chunk size (16 query blocks per CTA while their scores fit next to the
+// staging ring, else 8; every nb up to 4096 fits) and the row's scores per
+// lane kept in registers (nb <= 32 VPL).
+template <int D>
+cudaError_t dispatch_select(const Ctx& c, const float* q32, const float* k32t, const float* kn2,
+                            const double* q64, const double* k64, int BH, int nb, int nbs,
+                            int topk, int32_t* idx, int32_t* lists, int32_t* counts) {
+  const bool rb16 = sel_smem_bytes<D, 16>(nb) <= 200 * 1024;
+  if (nb <= 512)
+    return launch_select_fused<D, 16, 16>(c, q32, k32t, kn2, q64, k64, BH, nb, nbs, topk, idx,
+                                          lists, counts);
+  if (nb <= 2048)
+    return rb16 ? launch_select_fused<D, 16, 64>(c, q32, k32t, kn2, q64, k64, BH, nb, nbs, topk,
+                                                 idx, lists, counts)
+                : launch_select_fused<D, 8, 64>(c, q32, k32t, kn2, q64, k64, BH, nb, nbs, topk,
+                                                idx, lists, counts);
+  return launch_select_fused<D, 8, 128>(c, q32, k32t, kn2, q64, k64, BH, nb, nbs, topk, idx,
+                                        lists, counts);
 }
-
-namespace {
 
 // Pools Q (z = 0) and K (z = 1), then selects.
 cudaError_t pool_and_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
@@ -628,34 +664,33 @@ cudaError_t pool_and_select(const Ctx& c, const void* q, const void* k, int B, i
   double* qbar = reinterpret_cast<double*>(base + L.qbar);
   double* kbar = reinterpret_cast<double*>(base + L.kbar);
   float* qbar32 = reinterpret_cast<float*>(base + L.qbar32);
-  float* kbar32 = reinterpret_cast<float*>(base + L.kbar32);
+  float* kbar32t = reinterpret_cast<float*>(base + L.kbar32t);
+  float* kn2 = reinterpret_cast<float*>(base + L.kn2);
   const int nb = (N + kBlock - 1) / kBlock;
   const int BH = B * H;
   dim3 pg(nb, BH, 2);
   if (d == 128)
     pool_kernel<128><<<pg, 128, 0, c.stream>>>(static_cast<const uint4*>(q),
-                                                static_cast<const uint4*>(k), N, nb, qbar, kbar,
-                                                qbar32, kbar32);
+                                                static_cast<const uint4*>(k), N, nb, L.nbs, qbar,
+                                                kbar, qbar32, kbar32t, kn2);
   else
     pool_kernel<64><<<pg, 128, 0, c.stream>>>(static_cast<const uint4*>(q),
-                                               static_cast<const uint4*>(k), N, nb, qbar, kbar,
-                                               qbar32, kbar32);
+                                               static_cast<const uint4*>(k), N, nb, L.nbs, qbar,
+                                               kbar, qbar32, kbar32t, kn2);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (d == 128)
-    return sel_smem_bytes<128, 16>(nb) <= kSelSmemCap
-               ? launch_select_fused<128, 16>(c, qbar32, kbar32, qbar, kbar, BH, nb, topk, idx,
-                                              lists, counts)
-               : launch_select_fused<128, 8>(c, qbar32, kbar32, qbar, kbar, BH, nb, topk, idx,
-                                             lists, counts);
-  return sel_smem_bytes<64, 16>(nb) <= kSelSmemCap
-             ? launch_select_fused<64, 16>(c, qbar32, kbar32, qbar, kbar, BH, nb, topk, idx,
-                                           lists, counts)
-             : launch_select_fused<64, 8>(c, qbar32, kbar32, qbar, kbar, BH, nb, topk, idx,
-                                          lists, counts);
+    return dispatch_select<128>(c, qbar32, kbar32t, kn2, qbar, kbar, BH, nb, L.nbs, topk, idx,
+                                lists, counts);
+  return dispatch_select<64>(c, qbar32, kbar32t, kn2, qbar, kbar, BH, nb, L.nbs, topk, idx,
+                             lists, counts);
 }
 
 }  // namespace
+
+size_t select_ws_bytes(int B, int H, int N, int d, int block) {
+  return select_layout(B, H, N, d, block).total;
+}
 
 cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
                           int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts) {

@@ -52,8 +52,9 @@ def test_topk_attention_given_selection(salad, w):
 
 
 def test_topk_random_selection_patterns(salad):
-    # Arbitrary (not score-driven) kept sets: disjoint pairs, full overlap,
-    # single blocks -- every mask combination of a query-block pair.
+    # Arbitrary (not score-driven) kept sets: every mask combination of a
+    # query-block pair, tiles only one block of a pair needs, and the ragged
+    # last pair (nb = 15: its second block does not exist).
     w = RAGGED128
     inp = generate(w)
     dev = device_inputs(inp)
@@ -67,6 +68,19 @@ def test_topk_random_selection_patterns(salad):
         want = np.stack([oracle.topk_attention(q[0, h], k[0, h], v[0, h], idx[0, h], w.block)
                          for h in range(w.H)])[None]
         assert_close(o, want, f"random topk k={kk}")
+    # Structured sets: each block keeps only itself, a block far away, or
+    # blocks that differ between the two halves of each group of four.
+    for name, rows in (("diagonal", [[i] for i in range(w.nb)]),
+                       ("far", [[(i + w.nb // 2) % w.nb] for i in range(w.nb)]),
+                       ("slot-disjoint", [[0, 1] if i % 4 < 2 else [w.nb - 2, w.nb - 1]
+                                          for i in range(w.nb)])):
+        kk = len(rows[0])
+        idx = np.array([rows for _ in range(w.H)])[None]
+        idx_t = torch.from_numpy(idx).to(torch.int32).cuda()
+        o = salad.sparse_attn(dev["q"], dev["k"], dev["v"], "topk", topk=kk, idx=idx_t)
+        want = np.stack([oracle.topk_attention(q[0, h], k[0, h], v[0, h], idx[0, h], w.block)
+                         for h in range(w.H)])[None]
+        assert_close(o, want, f"{name} topk k={kk}")
     salad.check_error()
 
 

@@ -117,6 +117,9 @@ WORKLOADS: Dict[str, Workload] = {
                                space_major_heads=tuple(range(6))),
     # 720p-like long sequence: 28x45x80 latent (N=100800, 1575 blocks), k=158.
     "topk720": _topk720(),
+    # The 720p layer with 8 of its 40 heads (the same N, k and values per head):
+    # a case small enough for profiler captures of the 720p kernels.
+    "topk720_h8": _topk720().with_(name="topk720_h8", H=8, D=1024),
     # Batch of two independent samples, 40 heads, sparsity sweep + all blocks.
     "cfg_b2h40_s80": _sweep(0.80),
     "cfg_b2h40_s90": _sweep(0.90),

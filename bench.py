@@ -142,60 +142,124 @@ def committed_traffic(workload: str):
 
 # ---------------------------------------------------------------- clocks ---
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    """SM clock and throttle reasons sampled during a region.
+
+    A thread polls NVML about every half millisecond (a timed region of a
+    few dozen steps lasts only tens of milliseconds, shorter than
+    nvidia-smi's own sampling period); where NVML cannot be opened, an
+    `nvidia-smi -lms 100` child is the fallback and `start()` waits for its
+    first sample. Reading clocks changes nothing on the GPU."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clocks-event reason bits.
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device_index: int):
+        self.dev = device_index
         self.proc = None
-        self.lines = []
         self.thread = None
+        self.stop_flag = threading.Event()
+        self.first = threading.Event()
+        self.sm, self.mx, self.reasons = [], [], set()
+        self.source = None
+        self.nvml = None
+        self.handle = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        p = torch.cuda.get_device_properties(self.dev)
+        pynvml.nvmlInit()
+        for i in range(pynvml.nvmlDeviceGetCount()):
+            h = pynvml.nvmlDeviceGetHandleByIndex(i)
+            pci = pynvml.nvmlDeviceGetPciInfo(h)
+            if (pci.domain, pci.bus, pci.device) == (p.pci_domain_id, p.pci_bus_id, p.pci_device_id):
+                return pynvml, h
+        pynvml.nvmlShutdown()
+        return None, None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, ValueError):
-            self.proc = None
-            return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+            self.nvml, self.handle = self._nvml_handle()
+        except Exception:       # no NVML library or no matching device
+            self.nvml, self.handle = None, None
+        if self.handle is not None:
+            self.source = "nvml"
+            self.mx.append(float(self.nvml.nvmlDeviceGetMaxClockInfo(self.handle,
+                                                                     self.nvml.NVML_CLOCK_SM)))
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+        else:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except (OSError, ValueError):
+                self.proc = None
+                return
+            self.source = "nvidia-smi"
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
+        self.first.wait(timeout=3.0)
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _poll_nvml(self):
+        nv, h = self.nvml, self.handle
+        while not self.stop_flag.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:
+                break
+            for n, bit in self.REASON_BITS.items():
+                if mask & bit:
+                    self.reasons.add(n)
+            self.first.set()
+            time.sleep(0.0005)
 
-    def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        if self.thread is not None:
-            self.thread.join(timeout=5)
-        sm, mx, reasons = [], [], set()
+    def _read_smi(self):
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
+        for ln in self.proc.stdout:
+            parts = [p.strip() for p in ln.strip().split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                sm, mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
+            if self.stop_flag.is_set():
+                continue
+            self.sm.append(sm)
+            self.mx.append(mx)
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
-                    reasons.add(n)
+                    self.reasons.add(n)
+            self.first.set()
+
+    def stop(self) -> dict:
+        if self.thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0,
+                    "reasons": ["no clock source (NVML and nvidia-smi unavailable)"]}
+        self.stop_flag.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.thread.join(timeout=5)
+        if self.nvml is not None:
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+        sm = list(self.sm)
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+                "sm_min_mhz": min(sm) if sm else None,
+                "sm_max_mhz": max(self.mx) if self.mx else None,
+                "samples": len(sm), "source": self.source,
+                "reasons": sorted(self.reasons)}
 
 
 # ---------------------------------------------------------- distributed ---
@@ -400,8 +464,7 @@ def run_ours(args, w) -> int:
     # Phase events: 5 per step, recorded by the library on the launch stream.
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                          else local)
+    clocks = ClockSampler(torch.cuda.current_device())
     for e5 in ev:                 # create the handles before the timed region
         for e in e5:
             e.record(stream)

@@ -40,3 +40,36 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = _run({"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_clock_sampler_reads_nvml_reasons(monkeypatch):
+    """The timed region's clock record: a fake NVML reports a capped clock
+    with the power-cap and hardware-slowdown bits set; the sampler takes
+    several samples inside a 30 ms region and names both reasons."""
+    import threading
+    import time
+    import types
+    sys.path.insert(0, ROOT)
+    import bench
+
+    calls = {"n": 0}
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1,
+        nvmlDeviceGetMaxClockInfo=lambda h, k: 1965,
+        nvmlDeviceGetClockInfo=lambda h, k: (calls.__setitem__("n", calls["n"] + 1), 1800)[1],
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x4 | 0x8,
+        nvmlShutdown=lambda: None)
+    monkeypatch.setattr(bench.ClockSampler, "_nvml_handle", lambda self: (fake, object()))
+    c = bench.ClockSampler(0)
+    c.start()
+    time.sleep(0.03)
+    rec = c.stop()
+    assert rec["source"] == "nvml"
+    assert rec["samples"] >= 5 and rec["samples"] == calls["n"]
+    assert rec["sm_mhz"] == 1800 and rec["sm_max_mhz"] == 1965
+    assert rec["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    assert not any(t.name == c.thread.name and t.is_alive() for t in threading.enumerate())
+    # A capped clock holds the attention kernel to the sustained peak.
+    peak, label = bench.choose_peak({"bf16_tflops": 1636.8, "bf16_tflops_sustained": 1388.9},
+                                    30.0, rec)
+    assert label == "bf16 sustained" and peak == 1388.9

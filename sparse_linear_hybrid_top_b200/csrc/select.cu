@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
 //   E_i = (d + 8) 2^-24 * 1.05 * |qbar_i|_2 * max_j |kbar_j|_2
 // (rounding of the means to float32 and of the d-term fma chain, with a 5%
 // margin that also covers the float32 norms).  With T the k-th largest
-// float32 score of the row, bracketed as blo <= T < bhi, the float64 k-th
+// float32 score of the row, bracketed as blo <= T <= bhi, the float64 k-th
 // largest lies in [blo - E, bhi + E]: a block scoring above bhi + 2E is among
 // the float64 Top-K for certain, one below blo - 2E is not; only the blocks in between (the
 // candidates, typically none or a few) are scored again in float64 (ascending
@@ -114,24 +114,27 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
 // index asc).  The kept set is therefore the float64 selection.
 //
 // Phases (256 threads):
-//  1. scores: thread (ty, tx) accumulates rows 4ty..4ty+3 x columns
-//     4tx..4tx+3 of a column tile; the key means stream through two shared
-//     buffers (the next chunk is read into registers while the current one
-//     is multiplied).  The loading threads also sum each key mean's squares.
+//  1. scores: thread (ty, tx) accumulates RPT rows (RPT ty ..) x 4 columns
+//     (4 tx ..) of a column tile; the channel-major key means stream through
+//     a ring of cp.async chunks.  RPT = 8 where a 512-column tile covers the
+//     row (nb <= 512): each 16-byte key load then feeds 32 fma, not 16.
 //  2. one warp per row: a bisection on the value brackets the k-th largest
-//     float32 score to within the bound; then the band, the float64 recheck
-//     (candidates ranked directly, or by a radix select over float64 keys
-//     when there are many), the kept bitmap and the ascending index list.
+//     float32 score T, until the bracket is narrower than the bound or holds
+//     at most 32 scores -- those are then gathered one per lane and T is
+//     taken exactly; then the band, the float64 recheck (candidates ranked
+//     directly, or by a radix select over float64 keys when there are many),
+//     the kept bitmap and the ascending index list.
 //  3. one warp per pair of query blocks: the union of the two kept bitmaps
 //     as an ascending list of entries j | mask << 16.
-template <int D, int RB>
+template <int D, int RB, int RPT>
 struct SelCfg {
   static constexpr int kThreads = 256;
   static constexpr int kWarps = kThreads / 32;
-  static constexpr int kRG = RB / 4;               // 4-row groups
+  static constexpr int kRPT = RPT;                 // query rows per thread
+  static constexpr int kRG = RB / kRPT;            // row groups
   static constexpr int kCG = kThreads / kRG;       // 4-column groups
   static constexpr int kCT = 4 * kCG;              // columns per tile
-  static constexpr int kKC = 8;                    // channels per staged chunk
+  static constexpr int kKC = kRPT == 8 ? 4 : 8;    // channels per staged chunk
   static constexpr int kRing = 4;                  // chunks in flight (cp.async stages)
   static constexpr int kCandMax = 64;              // float64 candidates buffered per warp
   // The staging ring, reused after the scores by the float64 recheck.
@@ -141,9 +144,9 @@ struct SelCfg {
   static_assert(kStageFloats * 4 >= kWarps * (256 * 4 + kCandMax * 12), "recheck scratch");
 };
 
-template <int D, int RB>
+template <int D, int RB, int RPT>
 size_t sel_smem_bytes(int nb) {
-  using C = SelCfg<D, RB>;
+  using C = SelCfg<D, RB, RPT>;
   const size_t nbp = (static_cast<size_t>(nb) + 3) & ~static_cast<size_t>(3);
   const size_t nw = (static_cast<size_t>(nb) + 31) / 32;
   return static_cast<size_t>(D) * RB * 4            // qs [D][RB]
@@ -239,13 +242,13 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 // VPL: scores of a row each lane keeps in registers (column j = lane + 32 u).
-template <int D, int RB, int VPL>
+template <int D, int RB, int VPL, int RPT>
 __global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
     const float* __restrict__ qbar32, const float* __restrict__ kbar32t,
     const float* __restrict__ kn2, const double* __restrict__ qbar64,
     const double* __restrict__ kbar64, int nb, int nbs, int topk, int32_t* __restrict__ idx,
     int32_t* __restrict__ lists, int32_t* __restrict__ counts) {
-  using C = SelCfg<D, RB>;
+  using C = SelCfg<D, RB, RPT>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int nbp = (nb + 3) & ~3;
   const int nw = (nb + 31) / 32;
@@ -292,9 +295,9 @@ __global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
     const int r = e / D, c = e % D;
     qs[c * RB + r] = r < rows ? __ldg(qb + static_cast<long long>(r) * D + c) : 0.0f;
   }
-  float acc[4][4];
+  float acc[C::kRPT][4];
 #pragma unroll
-  for (int a2 = 0; a2 < 4; ++a2)
+  for (int a2 = 0; a2 < C::kRPT; ++a2)
 #pragma unroll
     for (int b2 = 0; b2 < 4; ++b2) acc[a2][b2] = 0.0f;
   for (int ch = 0; ch < nch; ++ch) {
@@ -304,28 +307,34 @@ __global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
     cp_async_commit();
     const float* kbuf = ks + (ch % C::kRing) * C::kKC * C::kCT;
     const int c0 = (ch % kChunks) * C::kKC;
-    float4 qv[C::kKC], kv[C::kKC];
+    float4 qv[C::kKC][C::kRPT / 4], kv[C::kKC];
 #pragma unroll
     for (int c = 0; c < C::kKC; ++c) {
-      qv[c] = *reinterpret_cast<const float4*>(qs + (c0 + c) * RB + 4 * ty);
+#pragma unroll
+      for (int g = 0; g < C::kRPT / 4; ++g)
+        qv[c][g] = *reinterpret_cast<const float4*>(qs + (c0 + c) * RB + C::kRPT * ty + 4 * g);
       kv[c] = *reinterpret_cast<const float4*>(kbuf + c * C::kCT + 4 * tx);
     }
 #pragma unroll
     for (int c = 0; c < C::kKC; ++c) {
-      const float q4[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
       const float k4[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
 #pragma unroll
-      for (int a2 = 0; a2 < 4; ++a2)
+      for (int g = 0; g < C::kRPT / 4; ++g) {
+        const float q4[4] = {qv[c][g].x, qv[c][g].y, qv[c][g].z, qv[c][g].w};
 #pragma unroll
-        for (int b2 = 0; b2 < 4; ++b2) acc[a2][b2] = fmaf(q4[a2], k4[b2], acc[a2][b2]);
+        for (int a2 = 0; a2 < 4; ++a2)
+#pragma unroll
+          for (int b2 = 0; b2 < 4; ++b2)
+            acc[4 * g + a2][b2] = fmaf(q4[a2], k4[b2], acc[4 * g + a2][b2]);
+      }
     }
     if (ch % kChunks == kChunks - 1) {
       const int j = (ch / kChunks) * C::kCT + 4 * tx;
 #pragma unroll
-      for (int a2 = 0; a2 < 4; ++a2) {
+      for (int a2 = 0; a2 < C::kRPT; ++a2) {
 #pragma unroll
         for (int b2 = 0; b2 < 4; ++b2) {
-          if (j + b2 < nb) sc[(4 * ty + a2) * nbp + j + b2] = acc[a2][b2];
+          if (j + b2 < nb) sc[(C::kRPT * ty + a2) * nbp + j + b2] = acc[a2][b2];
           acc[a2][b2] = 0.0f;
         }
       }
@@ -397,15 +406,43 @@ __global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
     double blo = mx, bhi = mx;   // T = mx when at least topk scores tie at the maximum
-    if (!wide && count_ge(mx) < topk) {
+    int c_hi = 0;
+    if (!wide && (c_hi = count_ge(mx)) < topk) {
       float lo = mn, hi = mx;
-      for (int it = 0; it < 64 && static_cast<double>(hi) - lo > 0.5 * E; ++it) {
+      int c_lo = nb;               // cnt(>= lo) >= topk > cnt(>= hi) = c_hi
+      for (int it = 0; it < 64 && static_cast<double>(hi) - lo > 0.5 * E && c_lo - c_hi > 32;
+           ++it) {
         const float mid = lo + 0.5f * (hi - lo);
         if (!(mid > lo && mid < hi)) break;   // adjacent floats
-        if (count_ge(mid) >= topk) lo = mid; else hi = mid;
+        const int cm = count_ge(mid);
+        if (cm >= topk) { lo = mid; c_lo = cm; } else { hi = mid; c_hi = cm; }
       }
       blo = lo;
       bhi = hi;
+      if (c_lo - c_hi <= 32) {
+        // At most 32 scores lie in [lo, hi): gather them, one per lane, and
+        // take T exactly: the largest x with cnt(>= x) >= topk - c_hi among
+        // them (every score >= hi is counted in c_hi).
+        float* gbuf = reinterpret_cast<float*>(hist);
+        int ng = 0;
+#pragma unroll
+        for (int u = 0; u < VPL; ++u) {
+          const bool g = vals[u] >= lo && vals[u] < hi;
+          const unsigned b = __ballot_sync(0xffffffffu, g);
+          if (g) gbuf[ng + __popc(b & ((1u << lane) - 1u))] = vals[u];
+          ng += __popc(b);
+        }
+        __syncwarp();
+        const float x = lane < ng ? gbuf[lane] : -INFINITY;
+        int cge = 0;
+        for (int u = 0; u < ng; ++u) cge += __shfl_sync(0xffffffffu, x, u) >= x ? 1 : 0;
+        float t = (lane < ng && cge >= topk - c_hi) ? x : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, o));
+        __syncwarp();
+        blo = t;
+        bhi = t;
+      }
     }
     // The float64 k-th largest lies within [blo - E, bhi + E]: above
     // bhi + 2E a block is kept for certain, below blo - 2E dropped.
@@ -620,18 +657,18 @@ SelectLayout select_layout(int B, int H, int N, int d, int block) {
   return L;
 }
 
-template <int D, int RB, int VPL>
+template <int D, int RB, int VPL, int RPT = 4>
 cudaError_t launch_select_fused(const Ctx& c, const float* q32, const float* k32t,
                                 const float* kn2, const double* q64, const double* k64, int BH,
                                 int nb, int nbs, int topk, int32_t* idx, int32_t* lists,
                                 int32_t* counts) {
-  const size_t smem = sel_smem_bytes<D, RB>(nb);
-  cudaError_t e = cudaFuncSetAttribute(select_fused_kernel<D, RB, VPL>,
+  const size_t smem = sel_smem_bytes<D, RB, RPT>(nb);
+  cudaError_t e = cudaFuncSetAttribute(select_fused_kernel<D, RB, VPL, RPT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid((nb + RB - 1) / RB, BH);
-  select_fused_kernel<D, RB, VPL><<<grid, SelCfg<D, RB>::kThreads, smem, c.stream>>>(
+  select_fused_kernel<D, RB, VPL, RPT><<<grid, SelCfg<D, RB, RPT>::kThreads, smem, c.stream>>>(
       q32, k32t, kn2, q64, k64, nb, nbs, topk, idx, lists, counts);
   return cudaGetLastError();
 }
@@ -643,9 +680,9 @@ template <int D>
 cudaError_t dispatch_select(const Ctx& c, const float* q32, const float* k32t, const float* kn2,
                             const double* q64, const double* k64, int BH, int nb, int nbs,
                             int topk, int32_t* idx, int32_t* lists, int32_t* counts) {
-  const bool rb16 = sel_smem_bytes<D, 16>(nb) <= 200 * 1024;
+  const bool rb16 = sel_smem_bytes<D, 16, 4>(nb) <= 200 * 1024;
   if (nb <= 512)
-    return launch_select_fused<D, 16, 16>(c, q32, k32t, kn2, q64, k64, BH, nb, nbs, topk, idx,
+    return launch_select_fused<D, 16, 16, 8>(c, q32, k32t, kn2, q64, k64, BH, nb, nbs, topk, idx,
                                           lists, counts);
   if (nb <= 2048)
     return rb16 ? launch_select_fused<D, 16, 64>(c, q32, k32t, kn2, q64, k64, BH, nb, nbs, topk,

@@ -101,7 +101,19 @@ SWA_SMALL64 = Workload(name="swa_small64", B=2, H=2, d=64, F=5, Hh=4, Wh=7, D=64
                        window=40, space_major_heads=(1,), lowrank_scale=0.5, seeds=(8, 9))  # N=140
 
 
-@pytest.mark.parametrize("w", [SWA_SMALL, SWA_SMALL64], ids=lambda w: w.name)
+# Grids with the frame counts of the 480p and 720p latents (F = 20, 28) and
+# one more (F = 36): a position's F rows straddle the 64-row blocks and the
+# 128-row tiles of the regrouped order differently in each.
+SWA_F20 = Workload(name="swa_f20", B=1, H=3, d=128, F=20, Hh=3, Wh=5, D=64, mode="swa",
+                   window=70, space_major_heads=(0, 2), lowrank_scale=0.5, seeds=(10,))  # N=300
+SWA_F28 = Workload(name="swa_f28", B=2, H=2, d=64, F=28, Hh=2, Wh=5, D=64, mode="swa",
+                   window=100, space_major_heads=(0, 1), lowrank_scale=0.5, seeds=(11, 12))  # N=280
+SWA_F36 = Workload(name="swa_f36", B=1, H=2, d=128, F=36, Hh=2, Wh=3, D=64, mode="swa",
+                   window=50, space_major_heads=(1,), lowrank_scale=0.5, seeds=(13,))  # N=216
+SWA_CASES = [SWA_SMALL, SWA_SMALL64, SWA_F20, SWA_F28, SWA_F36]
+
+
+@pytest.mark.parametrize("w", SWA_CASES, ids=lambda w: w.name)
 @pytest.mark.parametrize("window", [None, 0, 1, 1000000])
 def test_swa_attention(salad, w, window):
     W = w.window if window is None else window

@@ -17,7 +17,7 @@ import torch
 import oracle
 from synth import WORKLOADS, generate
 from tests._parity import assert_close, device_inputs, to64
-from tests.test_gpu_attention import SWA_SMALL, SWA_SMALL64
+from tests.test_gpu_attention import SWA_SMALL, SWA_SMALL64, SWA_F20, SWA_F36
 from tests.test_gpu_kernels import CASES, RAGGED128
 
 pytestmark = pytest.mark.gpu
@@ -58,7 +58,7 @@ def _selection_used(w, inp, idx_gpu):
     return idx
 
 
-@pytest.mark.parametrize("w", CASES + [SWA_SMALL, SWA_SMALL64], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", CASES + [SWA_SMALL, SWA_SMALL64, SWA_F20, SWA_F36], ids=lambda w: w.name)
 def test_forward_small_full_compare(salad, w):
     inp = generate(w)
     dev = device_inputs(inp)
@@ -128,7 +128,7 @@ def test_forward_branch_dropping(salad):
     assert_close(o_mid, ref["o"], "forward with branch dropping")
 
 
-@pytest.mark.parametrize("w", CASES + [SWA_SMALL, SWA_SMALL64], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", CASES + [SWA_SMALL, SWA_SMALL64, SWA_F20, SWA_F36], ids=lambda w: w.name)
 def test_forward_rope3d(salad, w):
     # The linear branch with the 3-D rotary encoding over the workload's grid.
     inp = generate(w)

@@ -358,7 +358,10 @@ def cpu_threads() -> int:
 
 
 # ----------------------------------------------------------------- sweep ---
-SWEEP = ("swa480", "topk720", "cfg_b2h40_s80", "cfg_b2h40_s90", "cfg_b2h40_s95", "cfg_b2h40_all")
+# "name+regroup_in_load": the workload with its ST-SWA heads regrouped inside
+# the attention's loads instead of copied (the library's non-default form).
+SWEEP = ("swa480", "swa480+regroup_in_load", "topk720", "cfg_b2h40_s80", "cfg_b2h40_s90",
+         "cfg_b2h40_s95", "cfg_b2h40_all")
 
 
 def run_sweep(names, device, stream, peaks, steps: int = 5, warmup: int = 2) -> dict:
@@ -375,12 +378,15 @@ def run_sweep(names, device, stream, peaks, steps: int = 5, warmup: int = 2) -> 
     burst = float(peaks["bf16_tflops"])
     sustained = float(peaks.get("bf16_tflops_sustained") or burst)
     for name in names:
-        w = WORKLOADS[name]
+        base, _, option = name.partition("+")
+        w = WORKLOADS[base]
         dev = generate_device(w, device, seed=w.seeds[0])
         extra = {}
         if w.mode == "swa":
             extra = dict(window=w.window, space_major_heads=w.space_major_heads, F=w.F,
                          Hh=w.Hh, Wh=w.Wh)
+        if option == "regroup_in_load":
+            extra["regroup_in_load"] = True
         plan = salad.ForwardPlan(dev["q"], dev["k"], dev["v"], dev["x"], dev["w_gate"],
                                  dev["w_lin"], mode=w.mode, topk=w.topk, bias=w.bias, eps=w.eps,
                                  **extra)
@@ -673,7 +679,8 @@ def run_ours(args, w) -> int:
     }
     if world == 1 and not args.no_sweep:
         # Timed after the headline line's numbers were taken.
-        line["workloads"] = run_sweep([n for n in SWEEP if n != w.name], device, stream, peaks)
+        line["workloads"] = run_sweep([n for n in SWEEP if n.partition("+")[0] != w.name],
+                                      device, stream, peaks)
         line["workloads_inputs"] = "device-drawn with the synthetic recipe (synth.generate_device)"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         del dev

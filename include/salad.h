@@ -286,6 +286,15 @@ typedef struct salad_forward_args {
      * and joined back before the attention, so only the last two events
      * bound one kernel. */
     void* const* phase_events;
+    /* SWA mode, heads regrouped space-major ("视频扩散模型中的稀疏注意力机制解析
+     * (ijyty.com)" 1.1): 0 (default) copies their Q, K, V space-major into
+     * the workspace first; 1 regroups them inside the attention's TMA loads
+     * instead (no copy): their work items and key tiles are floor(128/F)
+     * whole spatial positions, floor(128/F)*F of the 128 MMA rows (requires
+     * F <= 128, else SALAD_ERR_UNSUPPORTED).  Same results within rounding;
+     * on a B200 the copy is faster (480p: attention 0.96 ms with the copy,
+     * 1.45 ms in the loads), so 1 exists for memory-tight callers. */
+    int regroup_in_load;
 } salad_forward_args;
 
 size_t salad_forward_workspace_bytes(const salad_forward_args* args);

@@ -69,6 +69,7 @@ class ForwardArgs(ctypes.Structure):
         ("s_out", ctypes.c_void_p), ("idx_out", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("phase_events", ctypes.c_void_p),
+        ("regroup_in_load", ctypes.c_int),
     ]
 
 
@@ -410,7 +411,7 @@ class ForwardPlan:
                  gate_override: Optional[float] = None, drop_threshold: float = 0.0,
                  rope3d: bool = False, rope_base: float = 10000.0, o=None,
                  s_out=None, idx_out=None, block: int = 64, w_lin_full=None, w_out=None,
-                 out=None):
+                 out=None, regroup_in_load: bool = False):
         # Shapes first (a wrong size would make a kernel read past a tensor).
         if not isinstance(q, torch.Tensor) or q.dim() != 4:
             raise ValueError("q must be a [B, H, N, d] tensor")
@@ -463,6 +464,7 @@ class ForwardPlan:
         a.mode, a.block, a.topk, a.window = _MODES[mode], block, int(topk), int(window)
         a.space_major_heads = fptr
         a.F, a.Hh, a.Wh = F, Hh, Wh
+        a.regroup_in_load = 1 if regroup_in_load else 0
         a.eps = float(eps)
         a.gate_override = float("nan") if gate_override is None else float(gate_override)
         # Post-training branch dropping: sample b's linear branch is skipped

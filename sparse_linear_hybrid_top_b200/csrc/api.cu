@@ -206,6 +206,23 @@ bool make_tmap_bf16_heads4d(CUtensorMap* map, const void* base, int B, int H, in
 
 // Row-major [rows][cols] bf16 viewed as 2-D (cols, rows), box 64 x 64, 128-byte
 // swizzle.
+bool make_tmap_bf16_regroup(CUtensorMap* map, const void* base, int S, int F, int npos, int d,
+                            int box_pos) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr || F < 1 || F > 256 || box_pos < 1 || box_pos > 256) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(F),
+                              static_cast<cuuint64_t>(npos), static_cast<cuuint64_t>(S)};
+  // Byte strides of the frame, position and head dimensions.
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(npos) * d * 2,
+                                 static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(F) * npos * d * 2};
+  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(F), static_cast<cuuint32_t>(box_pos), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, int rows, int cols) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
@@ -254,7 +271,7 @@ static FwdLayout forward_layout(const salad_forward_args* a) {
   for (int h = 0; h < kMaxHeads; ++h) L.slot[h] = -1;
   if (a->mode == SALAD_MODE_SWA && a->H <= kMaxHeads)
     L.Hs = space_major_slots(a->H, a->space_major_heads, L.slot);
-  if (L.Hs > 0) {
+  if (L.Hs > 0 && !a->regroup_in_load) {   // the space-major copies
     const size_t bytes = B * static_cast<size_t>(L.Hs) * N * d * 2;
     L.qp = take(bytes);
     L.kp = take(bytes);
@@ -282,7 +299,7 @@ const char* salad_status_string(salad_status s) {
   }
 }
 
-int salad_version(void) { return 40100; }
+int salad_version(void) { return 40200; }
 
 // ------------------------------------------------------------------ gate --
 size_t salad_gate_workspace_bytes(int B, int N, int D) {
@@ -550,6 +567,9 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   if (L.Hs > 0 && (a->F < 1 || a->Hh < 1 || a->Wh < 1 ||
                    static_cast<long long>(a->F) * a->Hh * a->Wh != a->N))
     return SALAD_ERR_INVALID_ARG;
+  if (a->regroup_in_load != 0 && a->regroup_in_load != 1) return SALAD_ERR_INVALID_ARG;
+  // Regrouping in the loads needs a whole position (F rows) per 128-row tile.
+  if (L.Hs > 0 && a->regroup_in_load && a->F > 128) return SALAD_ERR_UNSUPPORTED;
   if ((st = check_ws(a->workspace, a->workspace_bytes, L.total)) != SALAD_OK) return st;
   Ctx c;
   if ((st = get_ctx(stream, &c)) != SALAD_OK) return st;
@@ -650,7 +670,12 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
     at.list_stride = 2 * a->topk;
   } else if (a->mode == SALAD_MODE_SWA) {
     at.mode = kModeBand;
-    if (L.Hs > 0) {
+    if (L.Hs > 0 && a->regroup_in_load) {
+      // Regrouped inside the attention's loads: whole positions per tile.
+      at.regroup_rows = (128 / a->F) * a->F;
+      at.Hs = L.Hs;
+      at.head_slot = L.slot;
+    } else if (L.Hs > 0) {
       int sel[kMaxHeads];
       for (int h = 0; h < H; ++h)
         if (L.slot[h] >= 0) sel[L.slot[h]] = h;

@@ -92,6 +92,14 @@ struct Params {
   short head_slot[256];       // slot in the regrouped copies, -1 = frame-major head
   int B, H, N, Hs, nb, npairs;
   int mode, window, F, Hh, Wh;
+  // Regrouping inside the loads (kernel instantiation RG): a regrouped head's
+  // items and key tiles are rg_pos whole spatial positions, rg_rows =
+  // rg_pos * F rows of the 128-row MMA, read from the frame-major tensors.
+  int rg_rows, rg_pos;
+  // RG: work items of sample b, head h are [b * per_b + head_base[h],
+  // b * per_b + head_base[h + 1]).
+  int per_b;
+  int head_base[257];
   const int32_t* lists;
   const int32_t* counts;
   int list_stride;
@@ -108,21 +116,48 @@ struct Params {
   unsigned long long wait_ns;
 };
 
+// The kernel's parameters (six tensor maps and Params) stay within the
+// classic 4 KB parameter space.
+static_assert(sizeof(Params) + 6 * sizeof(CUtensorMap) <= 4096, "kernel parameter space");
+
 struct Item {
   int bh, b, h, p;
   int ntiles;
-  int jlo;                // first key block (band / dense)
+  int jlo;                // first key block (band / dense), or key tile (rg)
   const int32_t* list;    // topk entries
   int slot;               // >= 0: regrouped (space-major) head
+  bool rg;                // regrouped in the loads: position-aligned rows and key tiles
 };
 
+// Query rows of an item (and keys of one of its key tiles).
+template <bool RG>
+__device__ __forceinline__ int item_rows(const Params& P, const Item& it) {
+  if constexpr (RG) return it.rg ? P.rg_rows : 128;
+  return 128;
+}
+
+template <bool RG>
 __device__ __forceinline__ Item make_item(const Params& P, long long w) {
   Item it;
-  it.bh = static_cast<int>(w / P.npairs);
-  it.p = static_cast<int>(w % P.npairs);
-  it.b = it.bh / P.H;
-  it.h = it.bh % P.H;
+  if constexpr (RG) {
+    it.b = static_cast<int>(w / P.per_b);
+    const int rem = static_cast<int>(w - static_cast<long long>(it.b) * P.per_b);
+    int lo = 0, hi = P.H;   // head_base[lo] <= rem < head_base[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) / 2;
+      if (P.head_base[mid] <= rem) lo = mid; else hi = mid;
+    }
+    it.h = lo;
+    it.p = rem - P.head_base[lo];
+    it.bh = it.b * P.H + it.h;
+  } else {
+    it.bh = static_cast<int>(w / P.npairs);
+    it.p = static_cast<int>(w % P.npairs);
+    it.b = it.bh / P.H;
+    it.h = it.bh % P.H;
+  }
   it.slot = P.head_slot[it.h];
+  it.rg = RG && it.slot >= 0;
   it.list = nullptr;
   it.jlo = 0;
   if (P.mode == kModeTopk) {
@@ -131,12 +166,19 @@ __device__ __forceinline__ Item make_item(const Params& P, long long w) {
   } else if (P.mode == kModeDense) {
     it.ntiles = P.nb;
   } else {
-    const int r0 = it.p * 128;
-    const int r1 = min(P.N, r0 + 128) - 1;
+    const int rows = item_rows<RG>(P, it);
+    const int r0 = it.p * rows;
+    const int r1 = min(P.N, r0 + rows) - 1;
     const int lo = max(0, r0 - P.window);
     const int hi = min(P.N - 1, r1 + P.window);
-    it.jlo = lo / 64;
-    it.ntiles = hi / 64 - it.jlo + 1;
+    if (RG && it.rg) {
+      // Key tiles of rg_rows keys (whole positions), two half-tiles each.
+      it.jlo = lo / rows;
+      it.ntiles = 2 * (hi / rows - it.jlo + 1);
+    } else {
+      it.jlo = lo / 64;
+      it.ntiles = hi / 64 - it.jlo + 1;
+    }
   }
   return it;
 }
@@ -191,7 +233,19 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-template <int D, bool HYB>
+// Zero [base, base + bytes) (a multiple of 16) with the whole CTA, then order
+// these generic-proxy writes before later async-proxy accesses (TMA, MMA).
+// Out of line: inlined, its loop costs the kernel a register spill.
+__device__ __noinline__ void zero_smem(unsigned char* base, int bytes) {
+  uint4* z = reinterpret_cast<uint4*>(base);
+  for (int i = threadIdx.x; i < bytes / 16; i += blockDim.x) z[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+}
+
+// RG: regrouped ST-SWA heads are read inside the loads (position-aligned
+// items and key tiles, V staged [d-slab][128 rows]); a separate instantiation
+// so that the default kernel carries none of it.
+template <int D, bool HYB, bool RG>
 __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CUtensorMap mq,
                                                       const __grid_constant__ CUtensorMap mk,
                                                       const __grid_constant__ CUtensorMap mv,
@@ -234,8 +288,15 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
   auto st_addr = [&](long long c) { return smem_u32(ring + static_cast<int>(c % NS) * C::kStage); };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const long long total = static_cast<long long>(P.B) * P.H * P.npairs;
+  const long long total = RG ? static_cast<long long>(P.B) * P.per_b
+                             : static_cast<long long>(P.B) * P.H * P.npairs;
   const unsigned long long wait_ns = P.wait_ns;
+
+  // RG: position-aligned items fill rg_rows < 128 rows of Q and of each K/V
+  // tile; the rows past them are read by the MMAs (their P columns are 0,
+  // their output rows are not written) and must hold finite values: zero the
+  // Q buffers and the ring once, before any load lands.
+  if constexpr (RG) zero_smem(qbuf, 2 * C::kQBuf + NS * C::kStage);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -285,11 +346,22 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
       // Q rows of item number j (two 64-row boxes per d-slab; rows past N
       // read 0) into buffer j & 1, once the item two before it has freed it.
       auto load_q = [&](long long w, uint32_t j) -> bool {
-        const Item it = make_item(P, w);
+        const Item it = make_item<RG>(P, w);
         const CUtensorMap* qm = it.slot >= 0 ? &mqp : &mq;
         const int z = it.slot >= 0 ? it.b * P.Hs + it.slot : it.bh;
         const int qb = static_cast<int>(j & 1);
         if (j >= 2 && !mbar_wait(q_empty(qb), ((j - 2) / 2) & 1, wait_ns, abort_flag)) return false;
+        if (RG && it.rg) {
+          // rg_pos whole positions, all F frames each, in space-major order:
+          // one (64 channels, F, rg_pos) box per d-slab of the frame-major Q.
+          mbar_arrive_expect_tx(q_full(qb), (D / 64) * P.rg_rows * 128);
+#pragma unroll
+          for (int hh = 0; hh < D / 64; ++hh)
+            tma_load_4d(q_addr(qb) + hh * C::kRowSlab, qm, q_full(qb), hh * 64, 0,
+                        it.p * P.rg_pos, it.bh);
+          q_issued = j + 1;
+          return true;
+        }
         mbar_arrive_expect_tx(q_full(qb), C::kQBuf);
 #pragma unroll
         for (int hh = 0; hh < D / 64; ++hh)
@@ -302,7 +374,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
       };
       if (static_cast<long long>(blockIdx.x) < total) ok = load_q(blockIdx.x, 0);
       for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++qc) {
-        const Item it = make_item(P, w);
+        const Item it = make_item<RG>(P, w);
         const CUtensorMap* km = it.slot >= 0 ? &mkp : &mk;
         const CUtensorMap* vm = it.slot >= 0 ? &mvp : &mv;
         const int z = it.slot >= 0 ? it.b * P.Hs + it.slot : it.bh;
@@ -322,15 +394,26 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
             bulk_load(dst, P.Gimg + static_cast<long long>(it.bh) * D * D, C::kGImg, full(si));
             return true;
           }
+          if (RG && it.rg) {
+            // Key tile jlo + t: rg_pos whole positions of the frame-major K
+            // or V, [d-slab][rg_rows rows] like every tile of this kernel.
+            mbar_arrive_expect_tx(full(si), (D / 64) * P.rg_rows * 128);
+#pragma unroll
+            for (int hh = 0; hh < D / 64; ++hh)
+              tma_load_4d(dst + hh * C::kRowSlab, kind == 0 ? km : vm, full(si), hh * 64, 0,
+                          (it.jlo + t) * P.rg_pos, it.bh);
+            return true;
+          }
           const int nblk = (2 * t + 1 < it.ntiles) ? 2 : 1;
           mbar_arrive_expect_tx(full(si), nblk * (D / 64) * kSlab);
           for (int x = 0; x < nblk; ++x) {
             const int j = list_entry(it, 2 * t + x, P.mode) & 0xFFFF;
 #pragma unroll
             for (int hh = 0; hh < D / 64; ++hh) {
-              if (kind == 0)   // K: [d-slab][128 rows]; block x from row 64x
-                tma_load_3d(dst + hh * C::kRowSlab + x * kSlab, km, full(si), hh * 64, j * 64, z);
-              else             // V: [block][d-slab][64 rows]
+              if (kind == 0 || RG)   // K (and RG's V): [d-slab][128 rows]; block x from row 64x
+                tma_load_3d(dst + hh * C::kRowSlab + x * kSlab, kind == 0 ? km : vm, full(si),
+                            hh * 64, j * 64, z);
+              else                   // V: [block][d-slab][64 rows]
                 tma_load_3d(dst + x * (D / 64) * kSlab + hh * kSlab, vm, full(si), hh * 64, j * 64, z);
             }
           }
@@ -393,7 +476,7 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         next_stage();
       };
       for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++ic) {
-        const Item it = make_item(P, w);
+        const Item it = make_item<RG>(P, w);
         const int T = (it.ntiles + 1) / 2;
         const bool lin = HYB && lin_on(P, it.b);
         const int qb = static_cast<int>(ic & 1);
@@ -415,13 +498,17 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
           ++pf[slot];
           if (!wait_stage()) { ok = false; break; }
           tc_fence_after();
-          const uint64_t vdesc = sdesc_sw128(ring_base + stage * C::kStage, kSlab, 1024);
+          // V (MN-major): d-slabs kSlab apart ([block][d-slab][64 rows]), or,
+          // in RG, kRowSlab apart ([d-slab][128 rows]).
+          const uint64_t vdesc =
+              sdesc_sw128(ring_base + stage * C::kStage, RG ? C::kRowSlab : kSlab, 1024);
           const uint32_t sa = tmem + C::s_col(slot), oa = tmem + C::o_col(slot);
           const uint32_t acc0 = t >= 2 ? 1u : 0u;
           if (2 * t + 1 < it.ntiles) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {   // K-steps: 16 keys each
-              const uint64_t off = static_cast<uint64_t>(((ks / 4) * (D / 64) * kSlab + (ks % 4) * 2048) >> 4);
+              const uint64_t off = static_cast<uint64_t>(
+                  (RG ? ks * 2048 : (ks / 4) * (D / 64) * kSlab + (ks % 4) * 2048) >> 4);
               mma_ts(oa, sa + ks * 8, vdesc + off, idesc_pv, ks > 0 ? 1u : acc0);
             }
           } else {
@@ -481,9 +568,10 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
     long long pv_base = 0;                        // this slot's PVs completed before this item
     bool ok = true;
     for (long long w = blockIdx.x; w < total && ok; w += gridDim.x, ++ic) {
-      const Item it = make_item(P, w);
-      const int row_pos = it.p * 128 + r;        // position in the head's (possibly regrouped) order
-      const bool row_valid = row_pos < P.N;
+      const Item it = make_item<RG>(P, w);
+      const int rows = item_rows<RG>(P, it);
+      const int row_pos = it.p * rows + r;       // position in the head's (possibly regrouped) order
+      const bool row_valid = (!RG || r < rows) && row_pos < P.N;
       const int T = (it.ntiles + 1) / 2;
       const int nt = (T - slot + 1) / 2;          // this slot's tiles: t = slot, slot + 2, ...
       const bool lin = HYB && lin_on(P, it.b);   // this item adds the linear term
@@ -535,17 +623,26 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         tc_fence_after();
         // The tile's two key blocks; inside each, the row's valid keys form
         // one contiguous range [lo, hi] of the block's 64 columns.
-        const int jb[2] = {e0 & 0xFFFF, e1 & 0xFFFF};
         const int mk[2] = {e0 >> 16, e1 >> 16};
+        // First key of each 64-column half: block j at 64 j, or, on a
+        // position-aligned tile (RG), rg_rows (jlo + t) + 64 x; kend is one
+        // past the tile's last key.
+        int kb[2] = {(e0 & 0xFFFF) * 64, (e1 & 0xFFFF) * 64};
+        int kend = P.N;
+        if (RG && it.rg) {
+          kb[0] = rows * (it.jlo + t);
+          kb[1] = kb[0] + 64;
+          kend = min(P.N, kb[0] + rows);
+        }
         int lo[2], hi[2];
         bool live[2], any[2], part[2];
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           lo[x] = 0;
-          hi[x] = min(63, P.N - 1 - jb[x] * 64);
+          hi[x] = min(63, kend - 1 - kb[x]);
           if (P.mode == kModeBand) {
-            lo[x] = max(lo[x], row_pos - P.window - jb[x] * 64);
-            hi[x] = min(hi[x], row_pos + P.window - jb[x] * 64);
+            lo[x] = max(lo[x], row_pos - P.window - kb[x]);
+            hi[x] = min(hi[x], row_pos + P.window - kb[x]);
           }
           live[x] = row_valid && (mk[x] & half_bit) && lo[x] <= hi[x];
           any[x] = __any_sync(0xffffffffu, live[x]);
@@ -789,7 +886,7 @@ __global__ void debug_wait_kernel(unsigned* err, unsigned long long wait_ns) {
   }
 }
 
-template <int D, bool HYB>
+template <int D, bool HYB, bool RG>
 cudaError_t launch_attn_t(const Ctx& c, const AttnArgs& a, const Params& P) {
   using C = AT<D, HYB>;
   CUtensorMap mq, mk, mv, mqp, mkp, mvp;
@@ -797,7 +894,15 @@ cudaError_t launch_attn_t(const Ctx& c, const AttnArgs& a, const Params& P) {
   if (!make_tmap_bf16_3d(&mq, a.q, BH, a.N, D) || !make_tmap_bf16_3d(&mk, a.k, BH, a.N, D) ||
       !make_tmap_bf16_3d(&mv, a.v, BH, a.N, D))
     return cudaErrorInvalidValue;
-  if (a.Hs > 0) {
+  if (RG) {
+    // Regrouped heads read in the loads: (channel, frame, position, head)
+    // views of the frame-major tensors, one box = rg_pos whole positions.
+    const int npos = a.N / a.F;
+    if (!make_tmap_bf16_regroup(&mqp, a.q, BH, a.F, npos, D, P.rg_pos) ||
+        !make_tmap_bf16_regroup(&mkp, a.k, BH, a.F, npos, D, P.rg_pos) ||
+        !make_tmap_bf16_regroup(&mvp, a.v, BH, a.F, npos, D, P.rg_pos))
+      return cudaErrorInvalidValue;
+  } else if (a.Hs > 0) {
     if (!make_tmap_bf16_3d(&mqp, a.qp, a.B * a.Hs, a.N, D) ||
         !make_tmap_bf16_3d(&mkp, a.kp, a.B * a.Hs, a.N, D) ||
         !make_tmap_bf16_3d(&mvp, a.vp, a.B * a.Hs, a.N, D))
@@ -807,13 +912,14 @@ cudaError_t launch_attn_t(const Ctx& c, const AttnArgs& a, const Params& P) {
     mkp = mk;
     mvp = mv;
   }
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, HYB>,
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, HYB, RG>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  const long long items = static_cast<long long>(BH) * P.npairs;
+  const long long items = RG ? static_cast<long long>(a.B) * P.per_b
+                             : static_cast<long long>(BH) * P.npairs;
   long long grid = items < c.num_sms ? items : c.num_sms;
   if (grid < 1) grid = 1;
-  attn_kernel<D, HYB><<<static_cast<int>(grid), 320, C::kSmem, c.stream>>>(mq, mk, mv, mqp, mkp,
+  attn_kernel<D, HYB, RG><<<static_cast<int>(grid), 320, C::kSmem, c.stream>>>(mq, mk, mv, mqp, mkp,
                                                                              mvp, P);
   return cudaGetLastError();
 }
@@ -833,6 +939,17 @@ cudaError_t launch_attention(const Ctx& c, const AttnArgs& a) {
   P.Hs = a.Hs;
   P.nb = (a.N + 63) / 64;
   P.npairs = (P.nb + 1) / 2;
+  // Regrouping inside the loads: items of rg_pos whole positions for the
+  // regrouped heads, 128-row pairs of query blocks for the others.
+  const bool rg = a.mode == kModeBand && a.Hs > 0 && a.regroup_rows > 0 && a.head_slot != nullptr;
+  P.rg_pos = rg ? a.regroup_rows / a.F : 0;
+  P.rg_rows = P.rg_pos * a.F;
+  P.head_base[0] = 0;
+  for (int h = 0; h < a.H; ++h) {
+    const int n = rg && a.head_slot[h] >= 0 ? (a.N / a.F + P.rg_pos - 1) / P.rg_pos : P.npairs;
+    P.head_base[h + 1] = P.head_base[h] + n;
+  }
+  P.per_b = P.head_base[a.H];
   P.mode = a.mode;
   P.window = a.window;
   P.F = a.F;
@@ -853,8 +970,15 @@ cudaError_t launch_attention(const Ctx& c, const AttnArgs& a) {
   P.err = c.err;
   P.wait_ns = c.wait_ns;
   const bool hyb = a.Gimg != nullptr;
-  if (a.d == 128) return hyb ? launch_attn_t<128, true>(c, a, P) : launch_attn_t<128, false>(c, a, P);
-  return hyb ? launch_attn_t<64, true>(c, a, P) : launch_attn_t<64, false>(c, a, P);
+  if (rg) {
+    if (P.rg_pos < 1) return cudaErrorInvalidValue;
+    if (a.d == 128)
+      return hyb ? launch_attn_t<128, true, true>(c, a, P) : launch_attn_t<128, false, true>(c, a, P);
+    return hyb ? launch_attn_t<64, true, true>(c, a, P) : launch_attn_t<64, false, true>(c, a, P);
+  }
+  if (a.d == 128)
+    return hyb ? launch_attn_t<128, true, false>(c, a, P) : launch_attn_t<128, false, false>(c, a, P);
+  return hyb ? launch_attn_t<64, true, false>(c, a, P) : launch_attn_t<64, false, false>(c, a, P);
 }
 
 cudaError_t launch_debug_wait(const Ctx& c) {

@@ -117,6 +117,10 @@ struct AttnArgs {
   int mode;                   // AttnMode
   int window;                 // band half-width
   int F, Hh, Wh;              // grid of the regrouped heads
+  // > 0: the regrouped heads are read inside the attention's loads, items
+  // and key tiles of floor(regroup_rows / F) whole positions (regroup_rows
+  // <= 128, >= F); qp, kp, vp are then unused.
+  int regroup_rows;
   const int32_t* lists;       // topk: [B*H*npairs][2*topk] entries j | mask<<16
   const int32_t* counts;      // topk: [B*H*npairs]
   int list_stride;            // 2*topk
@@ -139,6 +143,11 @@ cudaError_t launch_debug_wait(const Ctx& c);
 // (64, 64, 1), 128-byte swizzle.  Returns false on failure.
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, int S, int N, int d);
 bool make_tmap_bf16_heads4d(CUtensorMap* map, const void* base, int B, int H, int N, int d);
+// Frame-major [S][F * npos][d] bf16 (token t = f npos + p) viewed as 4-D
+// (d, F, npos, S) with the frame dimension first: box (64, F, box_pos, 1)
+// lands box_pos whole positions, F rows each, in space-major order.
+bool make_tmap_bf16_regroup(CUtensorMap* map, const void* base, int S, int F, int npos, int d,
+                            int box_pos);
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, int rows, int cols);
 
 // ---- full-width projections (proj.cu)

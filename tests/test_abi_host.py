@@ -34,7 +34,7 @@ def test_header_declarations_match_binding_and_exports():
 def test_library_is_built_for_sm100a_only():
     # The binding loads the in-tree library (no fallback path exists).
     assert os.path.dirname(salad.LIB_PATH) == os.path.join(ROOT, "sparse_linear_hybrid_top_b200")
-    assert salad.version() == 40100
+    assert salad.version() == 40200
 
 
 def test_status_strings():
@@ -164,6 +164,18 @@ def test_forward_argument_checks_and_workspace_query():
     none = _fwd_args(mode=1, topk=0, window=10, N=1000)
     assert (lib.salad_forward_workspace_bytes(ctypes.byref(swa)) -
             lib.salad_forward_workspace_bytes(ctypes.byref(none))) == 3 * 2 * 1000 * 64 * 2
+    # Regrouping inside the attention's loads needs no copies; it takes 0 or 1
+    # and a whole position (F <= 128 rows) per 128-row tile.
+    inload = _fwd_args(mode=1, topk=0, window=10, N=1000, F=10, Hh=10, Wh=10, regroup_in_load=1,
+                       space_major_heads=ctypes.cast(flags, ctypes.c_void_p).value)
+    assert (lib.salad_forward_workspace_bytes(ctypes.byref(inload)) ==
+            lib.salad_forward_workspace_bytes(ctypes.byref(none)))
+    ws = lib.salad_forward_workspace_bytes(ctypes.byref(swa))
+    for kw, want in ((dict(regroup_in_load=2, F=10, Hh=10, Wh=10), INVALID),
+                     (dict(regroup_in_load=1, F=250, Hh=2, Wh=2), UNSUP)):
+        bad = _fwd_args(mode=1, topk=0, window=10, N=1000, workspace=A, workspace_bytes=ws,
+                        space_major_heads=ctypes.cast(flags, ctypes.c_void_p).value, **kw)
+        assert lib.salad_forward(ctypes.byref(bad), None) == want, kw
 
 
 def test_valid_call_without_device_reports_cuda_error():

@@ -17,7 +17,7 @@ import torch
 import oracle
 from synth import WORKLOADS, generate
 from tests._parity import assert_close, device_inputs, to64
-from tests.test_gpu_attention import SWA_SMALL, SWA_SMALL64, SWA_F20, SWA_F36
+from tests.test_gpu_attention import SWA_SMALL, SWA_SMALL64, SWA_F20, SWA_F28, SWA_F36
 from tests.test_gpu_kernels import CASES, RAGGED128
 
 pytestmark = pytest.mark.gpu
@@ -210,7 +210,7 @@ def _oracle_rows(w, inp, b, h, rows_in_order, idx_row_of, s_b, lin_cache, angles
 
 
 def _sampled_check(salad, w, n_samples, seed=0, full=False, rope3d=False, drop_threshold=0.0,
-                   inp=None):
+                   inp=None, regroup_in_load=False):
     """The forward pass at full size, in the launch configuration the
     benchmark times, compared with the oracle on seeded query blocks (plus the
     ragged last block) or on every output."""
@@ -223,6 +223,8 @@ def _sampled_check(salad, w, n_samples, seed=0, full=False, rope3d=False, drop_t
             kw.update(F=w.F, Hh=w.Hh, Wh=w.Wh)
     if drop_threshold:
         kw["drop_threshold"] = drop_threshold
+    if regroup_in_load:
+        kw["regroup_in_load"] = True
     plan = _plan(salad, w, dev, **kw)
     o = plan.run()
     torch.cuda.synchronize()
@@ -295,6 +297,37 @@ def test_forward_topk480_branch_kept_below_threshold_sampled(salad, inp480):
 
 def test_forward_swa480_rope3d_sampled(salad):
     _sampled_check(salad, WORKLOADS["swa480"], 96, seed=7, rope3d=True)
+
+
+# ST-SWA heads regrouped inside the attention's TMA loads (position-aligned
+# items and key tiles of floor(128/F) whole positions) instead of copied:
+# the same results within rounding, for every frame count of the small
+# cases (4, 5, 20, 28, 36: 128, 125, 120, 112, 108 rows per tile), with the
+# rotary encoding, and at 480p.
+@pytest.mark.parametrize("w", [SWA_SMALL, SWA_SMALL64, SWA_F20, SWA_F28, SWA_F36],
+                         ids=lambda w: w.name)
+@pytest.mark.parametrize("rope3d", [False, True])
+def test_forward_regroup_in_load(salad, w, rope3d):
+    inp = generate(w)
+    dev = device_inputs(inp)
+    plan = _plan(salad, w, dev, regroup_in_load=True, rope3d=rope3d)
+    o = plan.run().clone()
+    torch.cuda.synchronize()
+    salad.check_error()
+    ref = oracle.forward(inp, mode=w.mode, block=w.block, topk=w.topk, window=w.window,
+                         space_major_heads=w.space_major_heads, F=w.F, Hh=w.Hh, Wh=w.Wh,
+                         eps=w.eps, rope3d=rope3d)
+    assert_close(o, ref["o"], f"forward {w.name} regrouped in the loads")
+    # Frame-major heads take the same tiles either way: bit-identical there.
+    copy = _plan(salad, w, dev, rope3d=rope3d).run()
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        if h not in w.space_major_heads:
+            assert torch.equal(o[:, h], copy[:, h]), h
+
+
+def test_forward_swa480_regroup_in_load_sampled(salad):
+    _sampled_check(salad, WORKLOADS["swa480"], 96, seed=9, regroup_in_load=True)
 
 
 @pytest.mark.parametrize("name", ["cfg_b2h40_s80", "cfg_b2h40_s90", "cfg_b2h40_s95",

@@ -291,9 +291,10 @@ typedef struct salad_forward_args {
      * the workspace first; 1 regroups them inside the attention's TMA loads
      * instead (no copy): their work items and key tiles are floor(128/F)
      * whole spatial positions, floor(128/F)*F of the 128 MMA rows (requires
-     * F <= 128, else SALAD_ERR_UNSUPPORTED).  Same results within rounding;
-     * on a B200 the copy is faster (480p: attention 0.96 ms with the copy,
-     * 1.45 ms in the loads), so 1 exists for memory-tight callers. */
+     * F <= 128, else SALAD_ERR_UNSUPPORTED).  Same results within rounding
+     * (frame-major heads bit-identical); no copy workspace.  On a B200 the
+     * copy is faster (480p ST-SWA layer: 1.02 ms with the copy, 1.63 ms in
+     * the loads), so 1 exists for memory-tight callers. */
     int regroup_in_load;
 } salad_forward_args;
 

@@ -101,10 +101,10 @@ def choose_peak(peaks: dict, timed_ms: float, clk: dict):
 
 
 def launches_per_step(w) -> int:
-    # gate (2) + [pool, fused select | gather] + linear state and reduce+fold
-    # (2) + attention (1)
+    # gate (2) + [pool, scores, selection | gather] + linear state and
+    # reduce+fold (2) + attention (1)
     if w.mode == "topk":
-        return 2 + 2 + 2 + 1
+        return 2 + 3 + 2 + 1
     if w.mode == "swa":
         return 2 + (1 if w.space_major_heads else 0) + 2 + 1
     return 2 + 2 + 1

@@ -174,13 +174,17 @@ int space_major_slots(int H, const uint8_t* flags, int* slot) {
 }  // namespace
 
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, int S, int N, int d) {
+  return make_tmap_bf16_3d_rows(map, base, S, N, d, 64);
+}
+
+bool make_tmap_bf16_3d_rows(CUtensorMap* map, const void* base, int S, int N, int d, int rows) {
   EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
+  if (fn == nullptr || rows < 1 || rows > 256) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                               static_cast<cuuint64_t>(S)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                                  static_cast<cuuint64_t>(N) * d * 2};
-  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kGateThreads) gate_partial_kernel(
 // 1024: thread c owns 16-byte column chunk c of every row, so its 8 weights
 // stay in registers; CTA (part, b) streams rows [part*rows_per, ...) of X[b]
 // with kGateRowUnroll independent 16-byte loads in flight per thread.
-constexpr int kGateRowUnroll = 8;
+constexpr int kGateRowUnroll = 16;
 __global__ void gate_rows_kernel(const uint4* __restrict__ x, const uint4* __restrict__ w, int N,
                                  int rows_per, float* __restrict__ partial) {
   const int CD = blockDim.x;

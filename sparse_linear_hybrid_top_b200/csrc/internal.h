@@ -142,6 +142,8 @@ cudaError_t launch_debug_wait(const Ctx& c);
 // Tensor map for a bf16 [S, N, d] tensor viewed as 3-D (d, N, S), box
 // (64, 64, 1), 128-byte swizzle.  Returns false on failure.
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, int S, int N, int d);
+// The same view with a box of (64, rows, 1), rows <= 256.
+bool make_tmap_bf16_3d_rows(CUtensorMap* map, const void* base, int S, int N, int d, int rows);
 bool make_tmap_bf16_heads4d(CUtensorMap* map, const void* base, int B, int H, int N, int d);
 // Frame-major [S][F * npos][d] bf16 (token t = f npos + p) viewed as 4-D
 // (d, F, npos, S) with the frame dimension first: box (64, F, box_pos, 1)

@@ -10,14 +10,17 @@
 // Precision: block sums of bf16 values are formed in float64 (exact for bf16
 // inputs in any realistic range) and divided by the row count; the kept set
 // is the one float64 dot products of these means decide.  The scores are
-// formed in float32 with a certified error bound, and only the blocks the
-// bound leaves undecided are scored again in float64 (select_fused_kernel).
+// formed on the tensor cores from a two-term bf16 split of each mean with a
+// certified error bound, and only the blocks the bound leaves undecided are
+// scored again in float64 (select_rows_kernel).
 //
-// Kernels: pool (HBM-bound: reads Q and K once), select_fused (per chunk of
-// query blocks of a head: float32 scores in shared memory, a radix select,
-// the float64 recheck, the ascending kept lists and the union of each pair
-// of query blocks' lists for the attention kernel), pair_union (the same
-// union for caller-supplied lists).
+// Kernels: pool (HBM-bound: reads Q and K once; writes the float64 means,
+// their bf16 hi/lo split and squared norms), score (tcgen05: S = Qbar Kbar^T
+// per head, 128 query blocks x 128 key blocks per accumulator, written to the
+// workspace in float32), select_rows (per 16 query blocks of a head: the
+// k-th largest score, the float64 recheck, the ascending kept lists and the
+// union of each pair of query blocks' lists for the attention kernel),
+// pair_union (the same union for caller-supplied lists).
 #include "common.cuh"
 #include "internal.h"
 
@@ -28,27 +31,33 @@ constexpr int kBlock = 64;
 
 // ------------------------------------------------------------------ pool --
 // CTA (i, bh, z): the mean of block i of head bh of Q (z = 0) or K (z = 1),
-// summed in float64 over the valid rows and written in float64; rounded once
-// to float32 for the selection's float32 pass: Q row-major [bh][i][c], K
-// channel-major [bh][c][i] (row length nbs, so a chunk of channels is a run
-// of contiguous rows), with the squared norm of each rounded K mean.
+// summed in float64 over the valid rows and written in float64 [bh][i][c];
+// its two-term bf16 split for the score MMAs, hi = bf16(f), lo = bf16(f - hi)
+// with f the float32 rounding of the mean (hi and lo [bh][i][c], row-major);
+// and its squared norm (float64 sum, stored as float32).
 template <int D>
 __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
                                                    const uint4* __restrict__ k, int N, int nb,
-                                                   int nbs, double* __restrict__ qbar,
+                                                   double* __restrict__ qbar,
                                                    double* __restrict__ kbar,
-                                                   float* __restrict__ qbar32,
-                                                   float* __restrict__ kbar32t,
+                                                   __nv_bfloat16* __restrict__ qhi,
+                                                   __nv_bfloat16* __restrict__ qlo,
+                                                   __nv_bfloat16* __restrict__ khi,
+                                                   __nv_bfloat16* __restrict__ klo,
+                                                   float* __restrict__ qn2,
                                                    float* __restrict__ kn2) {
   constexpr int CPR = D / 8;     // 16-byte chunks per row
   constexpr int RPI = 128 / CPR; // rows per iteration
   __shared__ double red[RPI][D];
-  __shared__ float nred[4];
+  __shared__ double nred[4];
   const int i = blockIdx.x;
   const long long bh = blockIdx.y;
   const bool is_k = blockIdx.z != 0;
   const uint4* src = is_k ? k : q;
   double* dst = is_k ? kbar : qbar;
+  __nv_bfloat16* hi = is_k ? khi : qhi;
+  __nv_bfloat16* lo = is_k ? klo : qlo;
+  float* n2 = is_k ? kn2 : qn2;
   const int row0 = i * kBlock;
   const int rows = min(kBlock, N - row0);
   const int chunk = threadIdx.x % CPR;
@@ -57,9 +66,7 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.0;
   const uint4* base = src + (bh * N + row0) * CPR + chunk;
-#pragma unroll 4
-  for (int r = rsub; r < rows; r += RPI) {
-    const uint4 v = __ldcs(base + static_cast<long long>(r) * CPR);
+  auto add = [&](const uint4& v) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -67,94 +74,266 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
       acc[2 * e] += static_cast<double>(f.x);
       acc[2 * e + 1] += static_cast<double>(f.y);
     }
+  };
+  if (rows == kBlock) {
+    // A full block: every load of the thread in flight before the first add.
+    constexpr int kIt = kBlock / RPI;
+    uint4 v[kIt];
+#pragma unroll
+    for (int t = 0; t < kIt; ++t) v[t] = __ldcs(base + static_cast<long long>(rsub + t * RPI) * CPR);
+#pragma unroll
+    for (int t = 0; t < kIt; ++t) add(v[t]);
+  } else {
+    for (int r = rsub; r < rows; r += RPI) add(__ldcs(base + static_cast<long long>(r) * CPR));
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) red[rsub][chunk * 8 + e] = acc[e];
   __syncthreads();
-  float part = 0.0f;
+  double part = 0.0;
   for (int c = threadIdx.x; c < D; c += 128) {
     double s = 0.0;
 #pragma unroll
     for (int r = 0; r < RPI; ++r) s += red[r][c];
     const double m = s / static_cast<double>(rows);
-    dst[(bh * nb + i) * D + c] = m;
-    const float m32 = static_cast<float>(m);
-    if (is_k) {
-      kbar32t[(bh * D + c) * static_cast<long long>(nbs) + i] = m32;
-      part = fmaf(m32, m32, part);
-    } else {
-      qbar32[(bh * nb + i) * D + c] = m32;
-    }
+    const long long at = (bh * nb + i) * D + c;
+    dst[at] = m;
+    const float f = static_cast<float>(m);
+    const __nv_bfloat16 h = __float2bfloat16_rn(f);
+    hi[at] = h;
+    lo[at] = __float2bfloat16_rn(f - __bfloat162float(h));   // f - h is exact in float32
+    part = fma(m, m, part);
   }
-  if (is_k) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if ((threadIdx.x & 31) == 0) nred[threadIdx.x >> 5] = part;
-    __syncthreads();
-    if (threadIdx.x == 0) kn2[bh * nb + i] = (nred[0] + nred[1]) + (nred[2] + nred[3]);
-  }
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  if ((threadIdx.x & 31) == 0) nred[threadIdx.x >> 5] = part;
+  __syncthreads();
+  if (threadIdx.x == 0) n2[bh * nb + i] = static_cast<float>((nred[0] + nred[1]) + (nred[2] + nred[3]));
 }
 
-// ------------------------------------------------------ fused selection --
-// One CTA scores a chunk of RB query blocks of one head against all nb key
-// blocks, selects the topk largest per query block, and merges the kept
-// lists of the chunk's pairs of query blocks for the attention kernel.
+// ----------------------------------------------------------------- score --
+// S[bh][i][j] = Qbar_i . Kbar_j for 128 query blocks (one CTA, M = 128) and
+// all key blocks, 128 at a time (N = 128, accumulators in four 128-column
+// TMEM buffers), as three bf16 products of the split means:
+//   S~ = qhi khi + qhi klo + qlo khi   (float32 accumulation).
+// The error bound (used by select_rows_kernel): with f = fl32(m), hi =
+// bf16(f), lo = bf16(f - hi), a mean is hi + lo + e with |e| <= 1.02 2^-18 |m|;
+// the dropped qlo klo and the e terms give at most 3.1 2^-18 |q_c||k_c| per
+// channel; the 3d products are exact in float32 (8-bit by 8-bit
+// significands) and their float32 sum, in any order and rounding to nearest
+// or toward zero, is off by at most 3d 2^-23 times the sum of their moduli
+// (<= 1.03 sum_c |q_c||k_c|).  With Cauchy-Schwarz:
+//   |S~ - S| <= (3.1 2^-18 + 3.09 d 2^-23) |qbar_i| |kbar_j|
+// plus an absolute term for values below float32's normal range.  (Reading:
+// the tensor core's float32 accumulation is taken to be no worse than
+// float32 additions; bf16 products are exact.)
 //
-// Exact float64 decision at float32 cost.  Scores are formed in float32 from
-// the float32-rounded means (a sequential fma chain over c, staged through
-// shared memory), so each differs from the float64 score by at most
-//   E_i = (d + 8) 2^-24 * 1.05 * |qbar_i|_2 * max_j |kbar_j|_2
-// (rounding of the means to float32 and of the d-term fma chain, with a 5%
-// margin that also covers the float32 norms).  With T the k-th largest
-// float32 score of the row, bracketed as blo <= T <= bhi, the float64 k-th
-// largest lies in [blo - E, bhi + E]: a block scoring above bhi + 2E is among
-// the float64 Top-K for certain, one below blo - 2E is not; only the blocks in between (the
-// candidates, typically none or a few) are scored again in float64 (ascending
-// c, the same sum as the float64 definition) and ranked by (score desc,
-// index asc).  The kept set is therefore the float64 selection.
-//
-// Phases (256 threads):
-//  1. scores: thread (ty, tx) accumulates RPT rows (RPT ty ..) x 4 columns
-//     (4 tx ..) of a column tile; the channel-major key means stream through
-//     a ring of cp.async chunks.  RPT = 8 where a 512-column tile covers the
-//     row (nb <= 512): each 16-byte key load then feeds 32 fma, not 16.
-//  2. one warp per row: a bisection on the value brackets the k-th largest
-//     float32 score T, until the bracket is narrower than the bound or holds
-//     at most 32 scores -- those are then gathered one per lane and T is
-//     taken exactly; then the band, the float64 recheck (candidates ranked
-//     directly, or by a radix select over float64 keys when there are many),
-//     the kept bitmap and the ascending index list.
-//  3. one warp per pair of query blocks: the union of the two kept bitmaps
-//     as an ascending list of entries j | mask << 16.
-template <int D, int RB, int RPT>
-struct SelCfg {
-  static constexpr int kThreads = 256;
-  static constexpr int kWarps = kThreads / 32;
-  static constexpr int kRPT = RPT;                 // query rows per thread
-  static constexpr int kRG = RB / kRPT;            // row groups
-  static constexpr int kCG = kThreads / kRG;       // 4-column groups
-  static constexpr int kCT = 4 * kCG;              // columns per tile
-  static constexpr int kKC = kRPT == 8 ? 4 : 8;    // channels per staged chunk
-  static constexpr int kRing = 4;                  // chunks in flight (cp.async stages)
-  static constexpr int kCandMax = 64;              // float64 candidates buffered per warp
-  // The staging ring, reused after the scores by the float64 recheck.
-  static constexpr int kStageFloats = kRing * kKC * kCT;
-  static_assert(kCG >= 32 && kCG % 32 == 0, "a warp spans one row group");
-  static_assert(D % kKC == 0, "chunking");
-  static_assert(kStageFloats * 4 >= kWarps * (256 * 4 + kCandMax * 12), "recheck scratch");
+// Warp roles (192 threads): warp 0 lane 0 issues the TMA loads and the MMAs;
+// warp 1 holds the TMEM allocation; warps 2..5 read the accumulators (TMEM
+// lane quarter w % 4) and write the scores.
+template <int D>
+struct SC {
+  static constexpr int kSlabA = 128 * 128;          // 128 rows of one 64-channel slab
+  static constexpr int kA = (D / 64) * kSlabA;      // one operand (hi or lo) of 128 rows
+  static constexpr int kB = kA;                     // 128 key rows
+  static constexpr int kSmemUsed = 1024 + 2 * kA + 2 * 2 * kB + 256;   // A hi/lo, B hi/lo x 2 stages
+  // Over half of the SM's shared memory, so one CTA (and its 512 TMEM
+  // columns) occupies each SM.
+  static constexpr int kSmem = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
 };
 
-template <int D, int RB, int RPT>
-size_t sel_smem_bytes(int nb) {
-  using C = SelCfg<D, RB, RPT>;
-  const size_t nbp = (static_cast<size_t>(nb) + 3) & ~static_cast<size_t>(3);
-  const size_t nw = (static_cast<size_t>(nb) + 31) / 32;
-  return static_cast<size_t>(D) * RB * 4            // qs [D][RB]
-         + static_cast<size_t>(C::kStageFloats) * 4 // ks [ring][KC][CT], later the recheck scratch
-         + RB * nbp * 4                             // scores [RB][nbp]
-         + RB * nw * 4                              // kept bitmaps [RB][nw]
-         + (C::kThreads + RB + 8) * 4;              // norm reduction, row norms
+template <int D>
+__global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ CUtensorMap mqh,
+                                                       const __grid_constant__ CUtensorMap mql,
+                                                       const __grid_constant__ CUtensorMap mkh,
+                                                       const __grid_constant__ CUtensorMap mkl,
+                                                       int nb, int nbs, int splits,
+                                                       float* __restrict__ S, unsigned* err,
+                                                       unsigned long long wait_ns) {
+  using C = SC<D>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* a_hi = sm;
+  unsigned char* a_lo = a_hi + C::kA;
+  unsigned char* b_st = a_lo + C::kA;                    // [2 stages][hi, lo]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(b_st + 2 * 2 * C::kB);
+  // bars: a_full, b_full[2], b_empty[2], acc_full[4], acc_empty[4], drain
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  const uint32_t a_full = smem_u32(bars);
+  auto b_full = [&](int s) { return smem_u32(bars + 1 + s); };
+  auto b_empty = [&](int s) { return smem_u32(bars + 3 + s); };
+  auto acc_full = [&](int b) { return smem_u32(bars + 5 + b); };
+  auto acc_empty = [&](int b) { return smem_u32(bars + 9 + b); };
+  const uint32_t drain = smem_u32(bars + 13);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int i0 = blockIdx.x * 128;
+  const int bh = blockIdx.z;
+  // This CTA's key chunks: [cbeg, cbeg + nch) of the row's 128-column chunks
+  // (the chunks are split over gridDim.y = splits CTAs).
+  const int nchunks = (nb + 127) / 128;
+  const int cbeg = static_cast<int>(static_cast<long long>(nchunks) * blockIdx.y / splits);
+  const int nch = static_cast<int>(static_cast<long long>(nchunks) * (blockIdx.y + 1) / splits) - cbeg;
+
+  if (threadIdx.x == 0) {
+    mbar_init(a_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(b_full(s), 1);
+      mbar_init(b_empty(s), 1);
+    }
+    for (int b = 0; b < 4; ++b) {
+      mbar_init(acc_full(b), 1);
+      mbar_init(acc_empty(b), 4);   // the four epilogue warps
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&mqh);
+    tma_prefetch_map(&mql);
+    tma_prefetch_map(&mkh);
+    tma_prefetch_map(&mkl);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      int loaded = 0, consumed = 0;   // chunks whose K means were requested / have landed
+      auto load_b = [&](int c) {
+        const int s = c & 1;
+        unsigned char* bh_ = b_st + s * 2 * C::kB;
+        mbar_arrive_expect_tx(b_full(s), 2 * C::kB);
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh) {
+          tma_load_3d(smem_u32(bh_ + hh * C::kSlabA), &mkh, b_full(s), hh * 64, (cbeg + c) * 128, bh);
+          tma_load_3d(smem_u32(bh_ + C::kB + hh * C::kSlabA), &mkl, b_full(s), hh * 64,
+                      (cbeg + c) * 128, bh);
+        }
+        loaded = c + 1;
+      };
+      mbar_arrive_expect_tx(a_full, 2 * C::kA);
+#pragma unroll
+      for (int hh = 0; hh < D / 64; ++hh) {
+        tma_load_3d(smem_u32(a_hi + hh * C::kSlabA), &mqh, a_full, hh * 64, i0, bh);
+        tma_load_3d(smem_u32(a_lo + hh * C::kSlabA), &mql, a_full, hh * 64, i0, bh);
+      }
+      load_b(0);
+      if (nch > 1) load_b(1);
+      constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+      ok = mbar_wait(a_full, 0, wait_ns, abort_flag);
+      const uint64_t dah = sdesc_sw128(smem_u32(a_hi), 16, 1024);
+      const uint64_t dal = sdesc_sw128(smem_u32(a_lo), 16, 1024);
+      for (int c = 0; c < nch && ok; ++c) {
+        const int s = c & 1, buf = c & 3;
+        if (!mbar_wait(b_full(s), (c / 2) & 1, wait_ns, abort_flag)) { ok = false; break; }
+        consumed = c + 1;
+        if (c >= 4 && !mbar_wait(acc_empty(buf), ((c - 4) / 4) & 1, wait_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const unsigned char* bs = b_st + s * 2 * C::kB;
+        const uint64_t dbh = sdesc_sw128(smem_u32(bs), 16, 1024);
+        const uint64_t dbl = sdesc_sw128(smem_u32(bs + C::kB), 16, 1024);
+        const uint32_t acc = tmem + 128 * buf;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t off = static_cast<uint64_t>(((ks / 4) * C::kSlabA + (ks % 4) * 32) >> 4);
+          mma_ss(acc, dah + off, dbh + off, idesc, ks > 0 ? 1u : 0u);
+          mma_ss(acc, dah + off, dbl + off, idesc, 1u);
+          mma_ss(acc, dal + off, dbh + off, idesc, 1u);
+        }
+        mma_commit(b_empty(s));
+        mma_commit(acc_full(buf));
+        // The previous chunk's stage is free once its MMAs have read it
+        // (they run ahead of the ones just issued): refill it with chunk c + 1.
+        if (c >= 1 && c + 1 < nch) {
+          if (!mbar_wait(b_empty((c - 1) & 1), ((c - 1) / 2) & 1, wait_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          load_b(c + 1);
+        }
+      }
+      if (!ok) raise_timeout(err, abort_flag);
+      // Leave nothing in flight: requested loads landed, issued MMAs done.
+      for (int c = consumed; c < loaded; ++c)
+        if (!mbar_wait(b_full(c & 1), (c / 2) & 1, wait_ns, nullptr)) atomicOr(err, kErrTimeout);
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0, wait_ns, nullptr)) atomicOr(err, kErrTimeout);
+    }
+  } else if (warp >= 2) {
+    const int quarter = warp % 4;
+    const int r = quarter * 32 + lane;                 // query block i0 + r
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const bool row_ok = i0 + r < nb;
+    float* srow = S + (static_cast<long long>(bh) * nb + (row_ok ? i0 + r : 0)) * nbs;
+    bool ok = true;
+    for (int c = 0; c < nch && ok; ++c) {
+      const int buf = c & 3;
+      if (!__all_sync(0xffffffffu, mbar_wait(acc_full(buf), (c / 4) & 1, wait_ns, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + 128 * buf + c0, v);
+        if (row_ok) {
+          float4* dst = reinterpret_cast<float4*>(srow + (cbeg + c) * 128 + c0);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty(buf));
+    }
+    if (!ok) raise_timeout(err, abort_flag);
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
 }
+
+// ------------------------------------------------------------ selection --
+// One CTA takes RB query blocks of one head: per block (one warp) the kept
+// set from the float32 scores S~ and the bound E above, then the union of
+// each pair of query blocks' kept sets for the attention kernel.
+//
+// Exact float64 decision.  With T the k-th largest score of the row in S~,
+// bracketed as blo <= T <= bhi, the float64 k-th largest lies in
+// [blo - E, bhi + E]: a block scoring above bhi + 2E is among the float64
+// Top-K for certain, one below blo - 2E is not; only the blocks in between
+// (the candidates, typically none or a few) are scored again in float64
+// (ascending c, the same sum as the float64 definition) and ranked by
+// (score desc, index asc).  The kept set is therefore the float64 selection.
+//
+// Per row: the row's scores in registers (column lane + 32 u); a bisection
+// on the value brackets T until the bracket is narrower than the bound or
+// holds at most 8 scores -- those are then gathered one per lane and T is
+// taken exactly; then the band, the float64 recheck (candidates ranked
+// directly, or by a radix select over float64 keys when there are many), the
+// kept bitmap and the ascending index list.  Per pair of query blocks (one
+// warp): the union of the two kept bitmaps as an ascending list of entries
+// j | mask << 16.
+constexpr int kSelThreads = 256;
+constexpr int kWarps = kSelThreads / 32;
+constexpr int kCandMax = 64;              // float64 candidates buffered per warp
 
 __device__ __forceinline__ unsigned long long dkey(double x) {
   x = x + 0.0;
@@ -230,164 +409,80 @@ __device__ __forceinline__ void radix_select64(int n, int& want, unsigned long l
   }
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // VPL: scores of a row each lane keeps in registers (column j = lane + 32 u).
-template <int D, int RB, int VPL, int RPT>
-__global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
-    const float* __restrict__ qbar32, const float* __restrict__ kbar32t,
+template <int D, int RB, int VPL>
+__global__ void __launch_bounds__(kSelThreads, VPL <= 16 ? 3 : 1) select_rows_kernel(
+    const float* __restrict__ S, int nbs, const float* __restrict__ qn2,
     const float* __restrict__ kn2, const double* __restrict__ qbar64,
-    const double* __restrict__ kbar64, int nb, int nbs, int topk, int32_t* __restrict__ idx,
+    const double* __restrict__ kbar64, int nb, int topk, int32_t* __restrict__ idx,
     int32_t* __restrict__ lists, int32_t* __restrict__ counts) {
-  using C = SelCfg<D, RB, RPT>;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int nbp = (nb + 3) & ~3;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int nw = (nb + 31) / 32;
-  float* qs = reinterpret_cast<float*>(smem_raw);                        // [D][RB]
-  float* ks = qs + D * RB;                                                // [ring][KC][CT]
-  float* sc = ks + C::kStageFloats;                                       // [RB][nbp]
-  unsigned* bits = reinterpret_cast<unsigned*>(sc + RB * nbp);            // [RB][nw]
+  unsigned* scratch = reinterpret_cast<unsigned*>(smem_raw);              // [warps][256 + 3 kCandMax]
+  unsigned* bits = scratch + kWarps * (256 + kCandMax * 3);               // [RB][nw]
   float* red = reinterpret_cast<float*>(bits + RB * nw);                  // [threads]
-  float* qn = red + C::kThreads;                                          // [RB] row norms
-  float* kmax_s = qn + RB;                                                // [1]
-
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const long long bh = blockIdx.y;
   const int i0 = blockIdx.x * RB;
   const int rows = min(RB, nb - i0);
-  const float* qb = qbar32 + (bh * nb + i0) * D;
-  const float* kt = kbar32t + bh * D * static_cast<long long>(nbs);
 
-  // ---- phase 1: float32 scores.  Chunk ch = (column tile, KC channels): KC
-  // rows of CT key means from the channel-major copy, streamed by cp.async
-  // through a ring of kRing chunks, kRing - 1 in flight ahead of the one
-  // being multiplied.
-  const int ty = tid / C::kCG, tx = tid % C::kCG;
-  const int ntile = (nb + C::kCT - 1) / C::kCT;
-  constexpr int kChunks = D / C::kKC;
-  constexpr int kCopies = C::kKC * C::kCT / 4;   // 16-byte copies per chunk
-  const int nch = ntile * kChunks;
-  auto issue = [&](int ch) {
-    float* dst = ks + (ch % C::kRing) * C::kKC * C::kCT;
-    const int j0 = (ch / kChunks) * C::kCT, c0 = (ch % kChunks) * C::kKC;
-    for (int e = tid; e < kCopies; e += C::kThreads) {
-      const int row = e / (C::kCT / 4), col = 4 * (e % (C::kCT / 4));
-      cp_async16(smem_u32(dst + row * C::kCT + col),
-                 kt + static_cast<long long>(c0 + row) * nbs + j0 + col);
-    }
-  };
-#pragma unroll
-  for (int s0 = 0; s0 < C::kRing - 1; ++s0) {
-    if (s0 < nch) issue(s0);
-    cp_async_commit();
-  }
-  // The chunk's query means, transposed (invalid rows are 0), meanwhile.
-  for (int e = tid; e < D * RB; e += C::kThreads) {
-    const int r = e / D, c = e % D;
-    qs[c * RB + r] = r < rows ? __ldg(qb + static_cast<long long>(r) * D + c) : 0.0f;
-  }
-  float acc[C::kRPT][4];
-#pragma unroll
-  for (int a2 = 0; a2 < C::kRPT; ++a2)
-#pragma unroll
-    for (int b2 = 0; b2 < 4; ++b2) acc[a2][b2] = 0.0f;
-  for (int ch = 0; ch < nch; ++ch) {
-    cp_async_wait<C::kRing - 2>();   // this thread's copies of chunk ch have landed
-    __syncthreads();                 // everyone's have; chunk ch - 1 is no longer read
-    if (ch + C::kRing - 1 < nch) issue(ch + C::kRing - 1);
-    cp_async_commit();
-    const float* kbuf = ks + (ch % C::kRing) * C::kKC * C::kCT;
-    const int c0 = (ch % kChunks) * C::kKC;
-    float4 qv[C::kKC][C::kRPT / 4], kv[C::kKC];
-#pragma unroll
-    for (int c = 0; c < C::kKC; ++c) {
-#pragma unroll
-      for (int g = 0; g < C::kRPT / 4; ++g)
-        qv[c][g] = *reinterpret_cast<const float4*>(qs + (c0 + c) * RB + C::kRPT * ty + 4 * g);
-      kv[c] = *reinterpret_cast<const float4*>(kbuf + c * C::kCT + 4 * tx);
-    }
-#pragma unroll
-    for (int c = 0; c < C::kKC; ++c) {
-      const float k4[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
-#pragma unroll
-      for (int g = 0; g < C::kRPT / 4; ++g) {
-        const float q4[4] = {qv[c][g].x, qv[c][g].y, qv[c][g].z, qv[c][g].w};
-#pragma unroll
-        for (int a2 = 0; a2 < 4; ++a2)
-#pragma unroll
-          for (int b2 = 0; b2 < 4; ++b2)
-            acc[4 * g + a2][b2] = fmaf(q4[a2], k4[b2], acc[4 * g + a2][b2]);
-      }
-    }
-    if (ch % kChunks == kChunks - 1) {
-      const int j = (ch / kChunks) * C::kCT + 4 * tx;
-#pragma unroll
-      for (int a2 = 0; a2 < C::kRPT; ++a2) {
-#pragma unroll
-        for (int b2 = 0; b2 < 4; ++b2) {
-          if (j + b2 < nb) sc[(C::kRPT * ty + a2) * nbp + j + b2] = acc[a2][b2];
-          acc[a2][b2] = 0.0f;
-        }
-      }
-    }
-  }
-  cp_async_wait<0>();
-  __syncthreads();   // the ring is free for the recheck scratch
-  // Largest key-mean norm of the head (from the pooling pass) and each row's
-  // query-mean norm.
+  // Largest key-mean norm of the head.
   float kmax2 = 0.0f;
-  for (int j = tid; j < nb; j += C::kThreads) kmax2 = fmaxf(kmax2, __ldg(kn2 + bh * nb + j));
+  for (int j = tid; j < nb; j += kSelThreads) kmax2 = fmaxf(kmax2, __ldg(kn2 + bh * nb + j));
   red[tid] = kmax2;
-  if (tid < RB) {
-    float n2 = 0.0f;
-    for (int c = 0; c < D; ++c) n2 = fmaf(qs[c * RB + tid], qs[c * RB + tid], n2);
-    qn[tid] = sqrtf(n2);
-  }
   __syncthreads();
   if (warp == 0) {
     float m = 0.0f;
-    for (int t = lane; t < C::kThreads; t += 32) m = fmaxf(m, red[t]);
+    for (int t = lane; t < kSelThreads; t += 32) m = fmaxf(m, red[t]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) kmax_s[0] = sqrtf(m);
+    if (lane == 0) red[0] = m;
   }
   __syncthreads();
-  const double kmax = kmax_s[0];
+  const double kmax = sqrtf(red[0]);
 
-  // ---- phase 2: per row (warp), the k-th largest float32 score, the band
-  // and, where needed, the float64 decision.  The staging buffers now hold
-  // each warp's radix histogram and candidate buffer.
-  unsigned* hist = reinterpret_cast<unsigned*>(ks) + warp * (256 + C::kCandMax * 3);
+  // ---- per row (warp): the k-th largest float32 score, the band and, where
+  // needed, the float64 decision; each warp's radix histogram and candidate
+  // buffer.
+  unsigned* hist = scratch + warp * (256 + kCandMax * 3);
   double* cs = reinterpret_cast<double*>(hist + 256);
-  int* cj = reinterpret_cast<int*>(cs + C::kCandMax);
-  for (int r = warp; r < RB; r += C::kWarps) {
+  int* cj = reinterpret_cast<int*>(cs + kCandMax);
+  // The row's scores in registers: column j = lane + 32 u (-inf past nb).
+  // With few per lane, the warp's next row is read while this one is
+  // processed.
+  constexpr bool kAhead = VPL <= 16;
+  auto load_row = [&](int r, float (&v)[VPL]) {
+    const float* srow = S + (bh * nb + i0 + r) * static_cast<long long>(nbs);
+#pragma unroll
+    for (int u = 0; u < VPL; ++u) {
+      const int j = lane + 32 * u;
+      v[u] = (r < rows && j < nb) ? __ldg(srow + j) : -INFINITY;
+    }
+  };
+  float ahead[kAhead ? VPL : 1];
+  if constexpr (kAhead) load_row(warp, ahead);
+  for (int r = warp; r < RB; r += kWarps) {
     unsigned* kept = bits + r * nw;
     for (int w = lane; w < nw; w += 32) kept[w] = 0u;
     __syncwarp();
     if (r >= rows) continue;
-    const float* srow = sc + r * nbp;
-    // The row's scores in registers: column j = lane + 32 u (-inf past nb).
+    const float* srow = S + (bh * nb + i0 + r) * static_cast<long long>(nbs);
     float vals[VPL];
+    if constexpr (kAhead) {
 #pragma unroll
-    for (int u = 0; u < VPL; ++u) {
-      const int j = lane + 32 * u;
-      vals[u] = j < nb ? srow[j] : -INFINITY;
+      for (int u = 0; u < VPL; ++u) vals[u] = ahead[u];
+      if (r + kWarps < rows) load_row(r + kWarps, ahead);
+    } else {
+      load_row(r, vals);
     }
     // Bracket the k-th largest float32 score T: cnt(>= lo) >= topk > cnt(>= hi),
     // so lo <= T < hi, by bisection on the value until the bracket is
     // narrower than the bound E allows.
-    const double qnr = static_cast<double>(qn[r]);
+    const double qnr = sqrtf(__ldg(qn2 + bh * nb + i0 + r));
     const bool wide = !(qnr < 1e18 && kmax < 1e18);
-    const double E = (D + 8) * 5.9604644775390625e-8 * 1.05 * qnr * kmax + D * 2.4e-38;
+    const double E = (3.1 * 3.814697265625e-6 + 3.09 * D * 1.1920928955078125e-7) * 1.05 * qnr * kmax +
+                     D * 1.0e-36 * (1.0 + qnr + kmax);
     auto count_ge = [&](float t) -> int {
       unsigned cnt = 0;
 #pragma unroll
@@ -410,7 +505,7 @@ __global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
     if (!wide && (c_hi = count_ge(mx)) < topk) {
       float lo = mn, hi = mx;
       int c_lo = nb;               // cnt(>= lo) >= topk > cnt(>= hi) = c_hi
-      for (int it = 0; it < 64 && static_cast<double>(hi) - lo > 0.5 * E && c_lo - c_hi > 32;
+      for (int it = 0; it < 64 && static_cast<double>(hi) - lo > 0.5 * E && c_lo - c_hi > 8;
            ++it) {
         const float mid = lo + 0.5f * (hi - lo);
         if (!(mid > lo && mid < hi)) break;   // adjacent floats
@@ -419,8 +514,8 @@ __global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
       }
       blo = lo;
       bhi = hi;
-      if (c_lo - c_hi <= 32) {
-        // At most 32 scores lie in [lo, hi): gather them, one per lane, and
+      if (c_lo - c_hi <= 8) {
+        // At most 8 scores lie in [lo, hi): gather them, one per lane, and
         // take T exactly: the largest x with cnt(>= x) >= topk - c_hi among
         // them (every score >= hi is counted in c_hi).
         float* gbuf = reinterpret_cast<float*>(hist);
@@ -447,10 +542,12 @@ __global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
     // The float64 k-th largest lies within [blo - E, bhi + E]: above
     // bhi + 2E a block is kept for certain, below blo - 2E dropped.
     const double lo = wide ? -INFINITY : blo - 2.0 * E, hi = wide ? INFINITY : bhi + 2.0 * E;
-    auto is_cand_v = [&](float v) {
-      const double dv = static_cast<double>(v);
-      return !(dv > hi) && (wide || dv >= lo);
-    };
+    // The same tests in float32 against the band's ends rounded outward
+    // (hi up, lo down): a score above hi_f is above hi, and every score in
+    // the band is a candidate (a few just outside it may be too).
+    const float hi_f = wide ? INFINITY : __double2float_ru(hi);
+    const float lo_f = wide ? -INFINITY : __double2float_rd(lo);
+    auto is_cand_v = [&](float v) { return !(v > hi_f) && v >= lo_f; };
     // Certain members (word u of the kept bitmap is the ballot over u) and
     // the candidates.
     int n_in = 0, n_cand = 0;
@@ -458,7 +555,7 @@ __global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
 #pragma unroll
     for (int u = 0; u < VPL; ++u) {
       const bool valid = lane + 32 * u < nb;
-      const bool in = valid && static_cast<double>(vals[u]) > hi;
+      const bool in = valid && vals[u] > hi_f;
       const bool cand = valid && is_cand_v(vals[u]);
       const unsigned bin = __ballot_sync(0xffffffffu, in);
       cand_w[u] = __ballot_sync(0xffffffffu, cand);
@@ -478,7 +575,7 @@ __global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
     } else if (need > 0) {
       const double* qrow = qbar64 + (bh * nb + i0 + r) * D;
       const double* kb64 = kbar64 + bh * nb * D;
-      if (n_cand <= C::kCandMax) {
+      if (n_cand <= kCandMax) {
         // Buffer the candidates (ascending j) with their float64 scores and
         // keep the `need` best by (score desc, j asc).
         int nc = 0;
@@ -533,12 +630,26 @@ __global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
     // The kept list, ascending.
     if (idx != nullptr) {
       int32_t* out = idx + (bh * nb + i0 + r) * static_cast<long long>(topk);
+      // Lane w writes the blocks of word w after those of the words before it.
       int written = 0;
-      for (int w = 0; w < nw; ++w) {
-        const unsigned word = kept[w];
-        const int pos = written + __popc(word & ((1u << lane) - 1u));
-        if (((word >> lane) & 1u) && pos < topk) out[pos] = 32 * w + lane;
-        written += __popc(word);
+      for (int w0 = 0; w0 < nw; w0 += 32) {
+        const int w = w0 + lane;
+        unsigned word = w < nw ? kept[w] : 0u;
+        const int cnt = __popc(word);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        int pos = written + incl - cnt;
+        while (word) {
+          const int bit = __ffs(word) - 1;
+          word &= word - 1;
+          if (pos < topk) out[pos] = 32 * w + bit;
+          ++pos;
+        }
+        written += __shfl_sync(0xffffffffu, incl, 31);
       }
     }
   }
@@ -547,7 +658,7 @@ __global__ void __launch_bounds__(256, VPL <= 16 ? 3 : 1) select_fused_kernel(
 
   // ---- phase 3: union of the kept sets of each pair (2p, 2p+1) of the chunk
   const int npairs_all = (nb + 1) / 2;
-  for (int pr = warp; pr < (rows + 1) / 2; pr += C::kWarps) {
+  for (int pr = warp; pr < (rows + 1) / 2; pr += kWarps) {
     const int p = i0 / 2 + pr;
     const unsigned* A = bits + (2 * pr) * nw;
     const bool has_b = 2 * pr + 1 < rows;
@@ -638,89 +749,127 @@ __global__ void pair_union_kernel(const int32_t* __restrict__ idx, int BH, int n
   if (lane == 0) counts[item] = min(base, 2 * topk);
 }
 
+
+size_t sel_smem_bytes(int RB, int nb) {
+  const size_t nw = (static_cast<size_t>(nb) + 31) / 32;
+  return static_cast<size_t>(kWarps) * (256 + kCandMax * 3) * 4 + RB * nw * 4 + kSelThreads * 4;
+}
+
 struct SelectLayout {
-  size_t qbar, kbar, qbar32, kbar32t, kn2, total;
-  int nbs;   // row length of the channel-major float32 K means
+  size_t qbar, kbar, qhi, qlo, khi, klo, qn2, kn2, S, total;
+  int nbs;   // row length of the score matrix (whole 128-column chunks)
 };
 SelectLayout select_layout(int B, int H, int N, int d, int block) {
   const size_t nb = (static_cast<size_t>(N) + block - 1) / block;
   const size_t BH = static_cast<size_t>(B) * H;
   SelectLayout L;
-  // Whole 512-column tiles, so a chunk's copies never leave their row.
-  L.nbs = static_cast<int>((nb + 511) / 512 * 512);
-  L.qbar = 0;
-  L.kbar = L.qbar + align256(BH * nb * d * sizeof(double));
-  L.qbar32 = L.kbar + align256(BH * nb * d * sizeof(double));
-  L.kbar32t = L.qbar32 + align256(BH * nb * d * sizeof(float));
-  L.kn2 = L.kbar32t + align256(BH * d * L.nbs * sizeof(float));
-  L.total = L.kn2 + align256(BH * nb * sizeof(float));
+  L.nbs = static_cast<int>((nb + 127) / 128 * 128);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  L.qbar = take(BH * nb * d * sizeof(double));
+  L.kbar = take(BH * nb * d * sizeof(double));
+  L.qhi = take(BH * nb * d * 2);
+  L.qlo = take(BH * nb * d * 2);
+  L.khi = take(BH * nb * d * 2);
+  L.klo = take(BH * nb * d * 2);
+  L.qn2 = take(BH * nb * sizeof(float));
+  L.kn2 = take(BH * nb * sizeof(float));
+  L.S = take(BH * nb * L.nbs * sizeof(float));
+  L.total = off;
   return L;
 }
 
-template <int D, int RB, int VPL, int RPT = 4>
-cudaError_t launch_select_fused(const Ctx& c, const float* q32, const float* k32t,
-                                const float* kn2, const double* q64, const double* k64, int BH,
-                                int nb, int nbs, int topk, int32_t* idx, int32_t* lists,
-                                int32_t* counts) {
-  const size_t smem = sel_smem_bytes<D, RB, RPT>(nb);
-  cudaError_t e = cudaFuncSetAttribute(select_fused_kernel<D, RB, VPL, RPT>,
+template <int D, int RB, int VPL>
+cudaError_t launch_select_rows(const Ctx& c, const float* S, int nbs, const float* qn2,
+                               const float* kn2, const double* q64, const double* k64, int BH,
+                               int nb, int topk, int32_t* idx, int32_t* lists, int32_t* counts) {
+  const size_t smem = sel_smem_bytes(RB, nb);
+  cudaError_t e = cudaFuncSetAttribute(select_rows_kernel<D, RB, VPL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid((nb + RB - 1) / RB, BH);
-  select_fused_kernel<D, RB, VPL, RPT><<<grid, SelCfg<D, RB, RPT>::kThreads, smem, c.stream>>>(
-      q32, k32t, kn2, q64, k64, nb, nbs, topk, idx, lists, counts);
+  select_rows_kernel<D, RB, VPL><<<grid, kSelThreads, smem, c.stream>>>(
+      S, nbs, qn2, kn2, q64, k64, nb, topk, idx, lists, counts);
   return cudaGetLastError();
 }
 
-// The chunk size (16 query blocks per CTA while their scores fit next to the
-// staging ring, else 8; every nb up to 4096 fits) and the row's scores per
-// lane kept in registers (nb <= 32 VPL).
+// The row's scores per lane kept in registers (nb <= 32 VPL); 16 query blocks
+// (two per warp) per CTA.
 template <int D>
-cudaError_t dispatch_select(const Ctx& c, const float* q32, const float* k32t, const float* kn2,
-                            const double* q64, const double* k64, int BH, int nb, int nbs,
-                            int topk, int32_t* idx, int32_t* lists, int32_t* counts) {
-  const bool rb16 = sel_smem_bytes<D, 16, 4>(nb) <= 200 * 1024;
+cudaError_t dispatch_select(const Ctx& c, const float* S, int nbs, const float* qn2,
+                            const float* kn2, const double* q64, const double* k64, int BH,
+                            int nb, int topk, int32_t* idx, int32_t* lists, int32_t* counts) {
   if (nb <= 512)
-    return launch_select_fused<D, 16, 16, 8>(c, q32, k32t, kn2, q64, k64, BH, nb, nbs, topk, idx,
-                                          lists, counts);
+    return launch_select_rows<D, 16, 16>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
+                                         counts);
   if (nb <= 2048)
-    return rb16 ? launch_select_fused<D, 16, 64>(c, q32, k32t, kn2, q64, k64, BH, nb, nbs, topk,
-                                                 idx, lists, counts)
-                : launch_select_fused<D, 8, 64>(c, q32, k32t, kn2, q64, k64, BH, nb, nbs, topk,
-                                                idx, lists, counts);
-  return launch_select_fused<D, 8, 128>(c, q32, k32t, kn2, q64, k64, BH, nb, nbs, topk, idx,
-                                        lists, counts);
+    return launch_select_rows<D, 16, 64>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
+                                         counts);
+  return launch_select_rows<D, 8, 128>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
+                                        counts);
 }
 
-// Pools Q (z = 0) and K (z = 1), then selects.
+template <int D>
+cudaError_t launch_score(const Ctx& c, const SelectLayout& L, char* base, int BH, int nb) {
+  CUtensorMap mqh, mql, mkh, mkl;
+  if (!make_tmap_bf16_3d_rows(&mqh, base + L.qhi, BH, nb, D, 128) ||
+      !make_tmap_bf16_3d_rows(&mql, base + L.qlo, BH, nb, D, 128) ||
+      !make_tmap_bf16_3d_rows(&mkh, base + L.khi, BH, nb, D, 128) ||
+      !make_tmap_bf16_3d_rows(&mkl, base + L.klo, BH, nb, D, 128))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SC<D>::kSmem);
+  if (e != cudaSuccess) return e;
+  // Split each row tile's key chunks over CTAs while the grid is under one
+  // CTA per SM.
+  const int tiles = (nb + 127) / 128, nchunks = tiles;
+  int splits = c.num_sms / (tiles * BH);
+  if (splits > nchunks) splits = nchunks;
+  if (splits < 1) splits = 1;
+  dim3 grid(tiles, splits, BH);
+  score_kernel<D><<<grid, 192, SC<D>::kSmem, c.stream>>>(
+      mqh, mql, mkh, mkl, nb, L.nbs, splits, reinterpret_cast<float*>(base + L.S), c.err,
+      c.wait_ns);
+  return cudaGetLastError();
+}
+
+// Pools Q (z = 0) and K (z = 1), scores, then selects.
 cudaError_t pool_and_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
                             int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts) {
   const SelectLayout L = select_layout(B, H, N, d, kBlock);
   char* base = static_cast<char*>(ws);
   double* qbar = reinterpret_cast<double*>(base + L.qbar);
   double* kbar = reinterpret_cast<double*>(base + L.kbar);
-  float* qbar32 = reinterpret_cast<float*>(base + L.qbar32);
-  float* kbar32t = reinterpret_cast<float*>(base + L.kbar32t);
+  auto bf = [&](size_t o) { return reinterpret_cast<__nv_bfloat16*>(base + o); };
+  float* qn2 = reinterpret_cast<float*>(base + L.qn2);
   float* kn2 = reinterpret_cast<float*>(base + L.kn2);
+  const float* S = reinterpret_cast<const float*>(base + L.S);
   const int nb = (N + kBlock - 1) / kBlock;
   const int BH = B * H;
   dim3 pg(nb, BH, 2);
   if (d == 128)
     pool_kernel<128><<<pg, 128, 0, c.stream>>>(static_cast<const uint4*>(q),
-                                                static_cast<const uint4*>(k), N, nb, L.nbs, qbar,
-                                                kbar, qbar32, kbar32t, kn2);
+                                                static_cast<const uint4*>(k), N, nb, qbar, kbar,
+                                                bf(L.qhi), bf(L.qlo), bf(L.khi), bf(L.klo), qn2,
+                                                kn2);
   else
     pool_kernel<64><<<pg, 128, 0, c.stream>>>(static_cast<const uint4*>(q),
-                                               static_cast<const uint4*>(k), N, nb, L.nbs, qbar,
-                                               kbar, qbar32, kbar32t, kn2);
+                                               static_cast<const uint4*>(k), N, nb, qbar, kbar,
+                                               bf(L.qhi), bf(L.qlo), bf(L.khi), bf(L.klo), qn2,
+                                               kn2);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  e = d == 128 ? launch_score<128>(c, L, base, BH, nb) : launch_score<64>(c, L, base, BH, nb);
+  if (e != cudaSuccess) return e;
   if (d == 128)
-    return dispatch_select<128>(c, qbar32, kbar32t, kn2, qbar, kbar, BH, nb, L.nbs, topk, idx,
-                                lists, counts);
-  return dispatch_select<64>(c, qbar32, kbar32t, kn2, qbar, kbar, BH, nb, L.nbs, topk, idx,
-                             lists, counts);
+    return dispatch_select<128>(c, S, L.nbs, qn2, kn2, qbar, kbar, BH, nb, topk, idx, lists,
+                                counts);
+  return dispatch_select<64>(c, S, L.nbs, qn2, kn2, qbar, kbar, BH, nb, topk, idx, lists, counts);
 }
 
 }  // namespace

@@ -65,4 +65,4 @@ def test_step_flops_match_the_stated_counts():
     assert f["dense"] == pytest.approx(5.98e12, rel=2e-3)
     f4 = bench.step_flops(WORKLOADS["topk720"])
     assert f4["sparse"] == pytest.approx(2.09e13, rel=5e-3)
-    assert bench.launches_per_step(WORKLOADS["topk480"]) == 7
+    assert bench.launches_per_step(WORKLOADS["topk480"]) == 8

@@ -108,7 +108,12 @@ salad_status salad_gate_noalloc(const void* x, const void* w, float bias, int B,
  * the `topk` largest per query block (ties: lower block index first).
  * q, k: bf16 [B, H, N, d] device.  idx: int32 [B, H, nb, topk] device (out),
  * nb = ceil(N/block), each row in ascending block order.  1 <= topk <= nb.
- * Workspace: salad_select_workspace_bytes(B, H, N, d, block).
+ * The float64 decision is reached by tensor-core scores of a two-term bf16
+ * split of the means with a certified error bound, and a float64 rescoring
+ * of the blocks the bound leaves undecided (the bound assumes float32
+ * accumulation in the tensor core no worse than float32 additions).
+ * Workspace: salad_select_workspace_bytes(B, H, N, d, block); it holds the
+ * float32 score matrix [B, H, nb, ceil(nb/128)*128] among others.
  */
 size_t salad_select_workspace_bytes(int B, int H, int N, int d, int block);
 salad_status salad_select_blocks(const void* q, const void* k, int B, int H, int N, int d,

@@ -112,8 +112,9 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
 
 // ----------------------------------------------------------------- score --
 // S[bh][i][j] = Qbar_i . Kbar_j for 128 query blocks (one CTA, M = 128) and
-// all key blocks, 128 at a time (N = 128, accumulators in four 128-column
-// TMEM buffers), as three bf16 products of the split means:
+// its share of the key blocks, 64 at a time (N = 64; four chunks of key
+// means in flight, accumulators in eight 64-column TMEM buffers), as three
+// bf16 products of the split means:
 //   S~ = qhi khi + qhi klo + qlo khi   (float32 accumulation).
 // The error bound (used by select_rows_kernel): with f = fl32(m), hi =
 // bf16(f), lo = bf16(f - hi), a mean is hi + lo + e with |e| <= 1.02 2^-18 |m|;
@@ -132,10 +133,14 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
 // lane quarter w % 4) and write the scores.
 template <int D>
 struct SC {
+  static constexpr int kN = 64;                     // key blocks per chunk (MMA N)
+  static constexpr int kStages = 4;                 // key-mean chunks in flight
+  static constexpr int kBufs = 512 / kN;            // TMEM accumulator buffers
   static constexpr int kSlabA = 128 * 128;          // 128 rows of one 64-channel slab
+  static constexpr int kSlabB = kN * 128;           // kN rows of one 64-channel slab
   static constexpr int kA = (D / 64) * kSlabA;      // one operand (hi or lo) of 128 rows
-  static constexpr int kB = kA;                     // 128 key rows
-  static constexpr int kSmemUsed = 1024 + 2 * kA + 2 * 2 * kB + 256;   // A hi/lo, B hi/lo x 2 stages
+  static constexpr int kB = (D / 64) * kSlabB;      // one operand of kN key rows
+  static constexpr int kSmemUsed = 1024 + 2 * kA + kStages * 2 * kB + 512;   // A hi/lo, B hi/lo stages
   // Over half of the SM's shared memory, so one CTA (and its 512 TMEM
   // columns) occupies each SM.
   static constexpr int kSmem = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
@@ -155,33 +160,36 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ C
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* a_hi = sm;
   unsigned char* a_lo = a_hi + C::kA;
-  unsigned char* b_st = a_lo + C::kA;                    // [2 stages][hi, lo]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(b_st + 2 * 2 * C::kB);
-  // bars: a_full, b_full[2], b_empty[2], acc_full[4], acc_empty[4], drain
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
+  unsigned char* b_st = a_lo + C::kA;                    // [kStages][hi, lo]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(b_st + C::kStages * 2 * C::kB);
+  // bars: a_full, b_full[kStages], b_empty[kStages], acc_full[kBufs],
+  // acc_empty[kBufs], drain
+  constexpr int NS = C::kStages, NB = C::kBufs;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 + 2 * NS + 2 * NB);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  static_assert((2 + 2 * NS + 2 * NB) * 8 + 8 <= 512, "barrier region");
   const uint32_t a_full = smem_u32(bars);
   auto b_full = [&](int s) { return smem_u32(bars + 1 + s); };
-  auto b_empty = [&](int s) { return smem_u32(bars + 3 + s); };
-  auto acc_full = [&](int b) { return smem_u32(bars + 5 + b); };
-  auto acc_empty = [&](int b) { return smem_u32(bars + 9 + b); };
-  const uint32_t drain = smem_u32(bars + 13);
+  auto b_empty = [&](int s) { return smem_u32(bars + 1 + NS + s); };
+  auto acc_full = [&](int b) { return smem_u32(bars + 1 + 2 * NS + b); };
+  auto acc_empty = [&](int b) { return smem_u32(bars + 1 + 2 * NS + NB + b); };
+  const uint32_t drain = smem_u32(bars + 1 + 2 * NS + 2 * NB);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int i0 = blockIdx.x * 128;
   const int bh = blockIdx.z;
-  // This CTA's key chunks: [cbeg, cbeg + nch) of the row's 128-column chunks
+  // This CTA's key chunks: [cbeg, cbeg + nch) of the row's kN-column chunks
   // (the chunks are split over gridDim.y = splits CTAs).
-  const int nchunks = (nb + 127) / 128;
+  const int nchunks = (nb + C::kN - 1) / C::kN;
   const int cbeg = static_cast<int>(static_cast<long long>(nchunks) * blockIdx.y / splits);
   const int nch = static_cast<int>(static_cast<long long>(nchunks) * (blockIdx.y + 1) / splits) - cbeg;
 
   if (threadIdx.x == 0) {
     mbar_init(a_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(b_full(s), 1);
       mbar_init(b_empty(s), 1);
     }
-    for (int b = 0; b < 4; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(acc_full(b), 1);
       mbar_init(acc_empty(b), 4);   // the four epilogue warps
     }
@@ -207,14 +215,15 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ C
       bool ok = true;
       int loaded = 0, consumed = 0;   // chunks whose K means were requested / have landed
       auto load_b = [&](int c) {
-        const int s = c & 1;
+        const int s = c % NS;
         unsigned char* bh_ = b_st + s * 2 * C::kB;
         mbar_arrive_expect_tx(b_full(s), 2 * C::kB);
 #pragma unroll
         for (int hh = 0; hh < D / 64; ++hh) {
-          tma_load_3d(smem_u32(bh_ + hh * C::kSlabA), &mkh, b_full(s), hh * 64, (cbeg + c) * 128, bh);
-          tma_load_3d(smem_u32(bh_ + C::kB + hh * C::kSlabA), &mkl, b_full(s), hh * 64,
-                      (cbeg + c) * 128, bh);
+          tma_load_3d(smem_u32(bh_ + hh * C::kSlabB), &mkh, b_full(s), hh * 64, (cbeg + c) * C::kN,
+                      bh);
+          tma_load_3d(smem_u32(bh_ + C::kB + hh * C::kSlabB), &mkl, b_full(s), hh * 64,
+                      (cbeg + c) * C::kN, bh);
         }
         loaded = c + 1;
       };
@@ -224,17 +233,16 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ C
         tma_load_3d(smem_u32(a_hi + hh * C::kSlabA), &mqh, a_full, hh * 64, i0, bh);
         tma_load_3d(smem_u32(a_lo + hh * C::kSlabA), &mql, a_full, hh * 64, i0, bh);
       }
-      load_b(0);
-      if (nch > 1) load_b(1);
-      constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+      for (int c = 0; c < NS && c < nch; ++c) load_b(c);
+      constexpr uint32_t idesc = idesc_bf16(128, C::kN, false, false);
       ok = mbar_wait(a_full, 0, wait_ns, abort_flag);
       const uint64_t dah = sdesc_sw128(smem_u32(a_hi), 16, 1024);
       const uint64_t dal = sdesc_sw128(smem_u32(a_lo), 16, 1024);
       for (int c = 0; c < nch && ok; ++c) {
-        const int s = c & 1, buf = c & 3;
-        if (!mbar_wait(b_full(s), (c / 2) & 1, wait_ns, abort_flag)) { ok = false; break; }
+        const int s = c % NS, buf = c % NB;
+        if (!mbar_wait(b_full(s), (c / NS) & 1, wait_ns, abort_flag)) { ok = false; break; }
         consumed = c + 1;
-        if (c >= 4 && !mbar_wait(acc_empty(buf), ((c - 4) / 4) & 1, wait_ns, abort_flag)) {
+        if (c >= NB && !mbar_wait(acc_empty(buf), ((c - NB) / NB) & 1, wait_ns, abort_flag)) {
           ok = false;
           break;
         }
@@ -242,30 +250,32 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ C
         const unsigned char* bs = b_st + s * 2 * C::kB;
         const uint64_t dbh = sdesc_sw128(smem_u32(bs), 16, 1024);
         const uint64_t dbl = sdesc_sw128(smem_u32(bs + C::kB), 16, 1024);
-        const uint32_t acc = tmem + 128 * buf;
+        const uint32_t acc = tmem + C::kN * buf;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t off = static_cast<uint64_t>(((ks / 4) * C::kSlabA + (ks % 4) * 32) >> 4);
-          mma_ss(acc, dah + off, dbh + off, idesc, ks > 0 ? 1u : 0u);
-          mma_ss(acc, dah + off, dbl + off, idesc, 1u);
-          mma_ss(acc, dal + off, dbh + off, idesc, 1u);
+          const uint64_t oa = static_cast<uint64_t>(((ks / 4) * C::kSlabA + (ks % 4) * 32) >> 4);
+          const uint64_t ob = static_cast<uint64_t>(((ks / 4) * C::kSlabB + (ks % 4) * 32) >> 4);
+          mma_ss(acc, dah + oa, dbh + ob, idesc, ks > 0 ? 1u : 0u);
+          mma_ss(acc, dah + oa, dbl + ob, idesc, 1u);
+          mma_ss(acc, dal + oa, dbh + ob, idesc, 1u);
         }
         mma_commit(b_empty(s));
         mma_commit(acc_full(buf));
         // The previous chunk's stage is free once its MMAs have read it
-        // (they run ahead of the ones just issued): refill it with chunk c + 1.
-        if (c >= 1 && c + 1 < nch) {
-          if (!mbar_wait(b_empty((c - 1) & 1), ((c - 1) / 2) & 1, wait_ns, abort_flag)) {
+        // (they run ahead of the ones just issued): refill it with chunk
+        // c - 1 + NS.
+        if (c >= 1 && c - 1 + NS < nch) {
+          if (!mbar_wait(b_empty((c - 1) % NS), ((c - 1) / NS) & 1, wait_ns, abort_flag)) {
             ok = false;
             break;
           }
-          load_b(c + 1);
+          load_b(c - 1 + NS);
         }
       }
       if (!ok) raise_timeout(err, abort_flag);
       // Leave nothing in flight: requested loads landed, issued MMAs done.
       for (int c = consumed; c < loaded; ++c)
-        if (!mbar_wait(b_full(c & 1), (c / 2) & 1, wait_ns, nullptr)) atomicOr(err, kErrTimeout);
+        if (!mbar_wait(b_full(c % NS), (c / NS) & 1, wait_ns, nullptr)) atomicOr(err, kErrTimeout);
       mma_commit(drain);
       if (!mbar_wait(drain, 0, wait_ns, nullptr)) atomicOr(err, kErrTimeout);
     }
@@ -277,18 +287,18 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ C
     float* srow = S + (static_cast<long long>(bh) * nb + (row_ok ? i0 + r : 0)) * nbs;
     bool ok = true;
     for (int c = 0; c < nch && ok; ++c) {
-      const int buf = c & 3;
-      if (!__all_sync(0xffffffffu, mbar_wait(acc_full(buf), (c / 4) & 1, wait_ns, abort_flag))) {
+      const int buf = c % NB;
+      if (!__all_sync(0xffffffffu, mbar_wait(acc_full(buf), (c / NB) & 1, wait_ns, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = 0; c0 < C::kN; c0 += 32) {
         uint32_t v[32];
-        tmem_ld32(lane_base + 128 * buf + c0, v);
+        tmem_ld32(lane_base + C::kN * buf + c0, v);
         if (row_ok) {
-          float4* dst = reinterpret_cast<float4*>(srow + (cbeg + c) * 128 + c0);
+          float4* dst = reinterpret_cast<float4*>(srow + (cbeg + c) * C::kN + c0);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
@@ -331,8 +341,10 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ C
 // kept bitmap and the ascending index list.  Per pair of query blocks (one
 // warp): the union of the two kept bitmaps as an ascending list of entries
 // j | mask << 16.
-constexpr int kSelThreads = 256;
-constexpr int kWarps = kSelThreads / 32;
+// Threads per CTA: 256, or 192 for many scores per lane (their registers
+// then allow two CTAs, 12 warps, per SM).
+template <int VPL> constexpr int sel_threads() { return VPL <= 16 ? 256 : (VPL <= 64 ? 192 : 256); }
+template <int VPL> constexpr int sel_min_blocks() { return VPL <= 16 ? 3 : (VPL <= 64 ? 2 : 1); }
 constexpr int kCandMax = 64;              // float64 candidates buffered per warp
 
 __device__ __forceinline__ unsigned long long dkey(double x) {
@@ -412,7 +424,7 @@ __device__ __forceinline__ void radix_select64(int n, int& want, unsigned long l
 
 // VPL: scores of a row each lane keeps in registers (column j = lane + 32 u).
 template <int D, int RB, int VPL>
-__global__ void __launch_bounds__(kSelThreads, VPL <= 16 ? 3 : 1) select_rows_kernel(
+__global__ void __launch_bounds__(sel_threads<VPL>(), sel_min_blocks<VPL>()) select_rows_kernel(
     const float* __restrict__ S, int nbs, const float* __restrict__ qn2,
     const float* __restrict__ kn2, const double* __restrict__ qbar64,
     const double* __restrict__ kbar64, int nb, int topk, int32_t* __restrict__ idx,
@@ -420,6 +432,7 @@ __global__ void __launch_bounds__(kSelThreads, VPL <= 16 ? 3 : 1) select_rows_ke
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int nw = (nb + 31) / 32;
   unsigned* scratch = reinterpret_cast<unsigned*>(smem_raw);              // [warps][256 + 3 kCandMax]
+  constexpr int kSelThreads = sel_threads<VPL>(), kWarps = kSelThreads / 32;
   unsigned* bits = scratch + kWarps * (256 + kCandMax * 3);               // [RB][nw]
   float* red = reinterpret_cast<float*>(bits + RB * nw);                  // [threads]
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -750,9 +763,9 @@ __global__ void pair_union_kernel(const int32_t* __restrict__ idx, int BH, int n
 }
 
 
-size_t sel_smem_bytes(int RB, int nb) {
+size_t sel_smem_bytes(int threads, int RB, int nb) {
   const size_t nw = (static_cast<size_t>(nb) + 31) / 32;
-  return static_cast<size_t>(kWarps) * (256 + kCandMax * 3) * 4 + RB * nw * 4 + kSelThreads * 4;
+  return static_cast<size_t>(threads / 32) * (256 + kCandMax * 3) * 4 + RB * nw * 4 + threads * 4;
 }
 
 struct SelectLayout {
@@ -787,13 +800,13 @@ template <int D, int RB, int VPL>
 cudaError_t launch_select_rows(const Ctx& c, const float* S, int nbs, const float* qn2,
                                const float* kn2, const double* q64, const double* k64, int BH,
                                int nb, int topk, int32_t* idx, int32_t* lists, int32_t* counts) {
-  const size_t smem = sel_smem_bytes(RB, nb);
+  const size_t smem = sel_smem_bytes(sel_threads<VPL>(), RB, nb);
   cudaError_t e = cudaFuncSetAttribute(select_rows_kernel<D, RB, VPL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid((nb + RB - 1) / RB, BH);
-  select_rows_kernel<D, RB, VPL><<<grid, kSelThreads, smem, c.stream>>>(
+  select_rows_kernel<D, RB, VPL><<<grid, sel_threads<VPL>(), smem, c.stream>>>(
       S, nbs, qn2, kn2, q64, k64, nb, topk, idx, lists, counts);
   return cudaGetLastError();
 }
@@ -808,7 +821,7 @@ cudaError_t dispatch_select(const Ctx& c, const float* S, int nbs, const float* 
     return launch_select_rows<D, 16, 16>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
                                          counts);
   if (nb <= 2048)
-    return launch_select_rows<D, 16, 64>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
+    return launch_select_rows<D, 12, 64>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
                                          counts);
   return launch_select_rows<D, 8, 128>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
                                         counts);
@@ -819,15 +832,15 @@ cudaError_t launch_score(const Ctx& c, const SelectLayout& L, char* base, int BH
   CUtensorMap mqh, mql, mkh, mkl;
   if (!make_tmap_bf16_3d_rows(&mqh, base + L.qhi, BH, nb, D, 128) ||
       !make_tmap_bf16_3d_rows(&mql, base + L.qlo, BH, nb, D, 128) ||
-      !make_tmap_bf16_3d_rows(&mkh, base + L.khi, BH, nb, D, 128) ||
-      !make_tmap_bf16_3d_rows(&mkl, base + L.klo, BH, nb, D, 128))
+      !make_tmap_bf16_3d_rows(&mkh, base + L.khi, BH, nb, D, SC<D>::kN) ||
+      !make_tmap_bf16_3d_rows(&mkl, base + L.klo, BH, nb, D, SC<D>::kN))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SC<D>::kSmem);
   if (e != cudaSuccess) return e;
   // Split each row tile's key chunks over CTAs while the grid is under one
   // CTA per SM.
-  const int tiles = (nb + 127) / 128, nchunks = tiles;
+  const int tiles = (nb + 127) / 128, nchunks = (nb + SC<D>::kN - 1) / SC<D>::kN;
   int splits = c.num_sms / (tiles * BH);
   if (splits > nchunks) splits = nchunks;
   if (splits < 1) splits = 1;

@@ -116,14 +116,16 @@ __global__ void __launch_bounds__(128) pool_kernel(const uint4* __restrict__ q,
 // means in flight, accumulators in eight 64-column TMEM buffers), as three
 // bf16 products of the split means:
 //   S~ = qhi khi + qhi klo + qlo khi   (float32 accumulation).
-// The error bound (used by select_rows_kernel): with f = fl32(m), hi =
-// bf16(f), lo = bf16(f - hi), a mean is hi + lo + e with |e| <= 1.02 2^-18 |m|;
-// the dropped qlo klo and the e terms give at most 3.1 2^-18 |q_c||k_c| per
-// channel; the 3d products are exact in float32 (8-bit by 8-bit
-// significands) and their float32 sum, in any order and rounding to nearest
-// or toward zero, is off by at most 3d 2^-23 times the sum of their moduli
-// (<= 1.03 sum_c |q_c||k_c|).  With Cauchy-Schwarz:
-//   |S~ - S| <= (3.1 2^-18 + 3.09 d 2^-23) |qbar_i| |kbar_j|
+// The error bound (used by select_rows_kernel), with u = 2^-8 the unit
+// roundoff of bf16 (8-bit significand): f = fl32(m) is within 2^-24 |m| of
+// m; hi = bf16(f) within u |f| of f; r = f - hi is exact and lo = bf16(r)
+// within u |r| <= u^2 |f| of r.  So a mean is hi + lo + e with |e| <=
+// 1.004 2^-16 |m|, and the dropped qlo klo and the e terms give at most
+// 3.1 2^-16 |q_c||k_c| per channel.  The 3d products are exact in float32
+// (8-bit by 8-bit significands) and their float32 sum, in any order and
+// rounding to nearest or toward zero, is off by at most 3d 2^-23 times the
+// sum of their moduli (<= 1.016 sum_c |q_c||k_c|).  With Cauchy-Schwarz:
+//   |S~ - S| <= (3.1 2^-16 + 3.09 d 2^-23) |qbar_i| |kbar_j|
 // plus an absolute term for values below float32's normal range.  (Reading:
 // the tensor core's float32 accumulation is taken to be no worse than
 // float32 additions; bf16 products are exact.)
@@ -494,7 +496,7 @@ __global__ void __launch_bounds__(sel_threads<VPL>(), sel_min_blocks<VPL>()) sel
     // narrower than the bound E allows.
     const double qnr = sqrtf(__ldg(qn2 + bh * nb + i0 + r));
     const bool wide = !(qnr < 1e18 && kmax < 1e18);
-    const double E = (3.1 * 3.814697265625e-6 + 3.09 * D * 1.1920928955078125e-7) * 1.05 * qnr * kmax +
+    const double E = (3.1 * 1.52587890625e-5 + 3.09 * D * 1.1920928955078125e-7) * 1.05 * qnr * kmax +
                      D * 1.0e-36 * (1.0 + qnr + kmax);
     auto count_ge = [&](float t) -> int {
       unsigned cnt = 0;

@@ -604,12 +604,25 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
     return cudaEventRecord(static_cast<cudaEvent_t>(a->phase_events[i]), st) == cudaSuccess;
   };
   if (!mark(0, c.stream)) return SALAD_ERR_CUDA;
-  if (dv != nullptr && (cudaEventRecord(dv->fork, c.stream) != cudaSuccess ||
-                        cudaStreamWaitEvent(cg.stream, dv->fork, 0) != cudaSuccess ||
-                        cudaStreamWaitEvent(cl.stream, dv->fork, 0) != cudaSuccess))
-    return SALAD_ERR_CUDA;
   bool ok = true;
   auto check = [&](cudaError_t e) { ok = ok && e == cudaSuccess; };
+  // Top-K: the selection chain is enqueued first and the side chains fork
+  // once its pooling pass has read Q and K.  The pool then has the memory
+  // bandwidth to itself, and the gate and the linear branch share it with
+  // the scores and the decision instead, which read little (measured: the
+  // attention can start 8 us earlier at 480p, 100 us at 720p).
+  const bool topk = a->mode == SALAD_MODE_TOPK;
+  int32_t* idx = a->idx_out != nullptr ? a->idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  int32_t* lists = reinterpret_cast<int32_t*>(ws + L.lists);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  if (topk)
+    check(launch_select(c, a->q, a->k, B, H, N, d, a->topk, idx, ws + L.sel, lists, counts,
+                        dv != nullptr ? dv->fork : nullptr));
+  else if (dv != nullptr && cudaEventRecord(dv->fork, c.stream) != cudaSuccess)
+    return SALAD_ERR_CUDA;
+  if (dv != nullptr && (cudaStreamWaitEvent(cg.stream, dv->fork, 0) != cudaSuccess ||
+                        cudaStreamWaitEvent(cl.stream, dv->fork, 0) != cudaSuccess))
+    return SALAD_ERR_CUDA;
 
   // 1. gate (paper.rainbus.top 方法步骤详情 step 5), side stream 0
   float* s = a->s_out != nullptr ? a->s_out : reinterpret_cast<float*>(ws + L.s);
@@ -663,11 +676,8 @@ salad_status salad_forward(const salad_forward_args* a, salad_stream stream) {
   if (dv != nullptr) check(cudaEventRecord(dv->join_lin, cl.stream));
 
   // 2. sparse-branch pattern (ijyty.com 1.1 / 1.2), the caller's stream
-  if (a->mode == SALAD_MODE_TOPK) {
-    int32_t* idx = a->idx_out != nullptr ? a->idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
-    int32_t* lists = reinterpret_cast<int32_t*>(ws + L.lists);
-    int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
-    if (ok) check(launch_select(c, a->q, a->k, B, H, N, d, a->topk, idx, ws + L.sel, lists, counts));
+  if (topk) {
+    // (enqueued above)
     at.mode = kModeTopk;
     at.lists = lists;
     at.counts = counts;

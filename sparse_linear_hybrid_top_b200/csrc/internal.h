@@ -29,9 +29,11 @@ cudaError_t launch_fill_f32(const Ctx& c, float* dst, float value, int n);
 size_t select_ws_bytes(int B, int H, int N, int d, int block);
 // Kept lists idx [B,H,nb,topk] (ascending; may be null) and, when lists is
 // not null, the pair unions of launch_pair_union in the same launch.
+// `pooled` (optional) is recorded on c.stream once the pooling pass, the
+// chain's only full read of Q and K, has been enqueued.
 cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
                           int topk, int32_t* idx, void* ws, int32_t* lists = nullptr,
-                          int32_t* counts = nullptr);
+                          int32_t* counts = nullptr, cudaEvent_t pooled = nullptr);
 // Merge the kept lists of query blocks (2p, 2p+1) into one ascending list of
 // entries (j | mask << 16), mask bit 0 = block 2p keeps j, bit 1 = block 2p+1.
 size_t pairs_ws_bytes(int B, int H, int N, int topk);

@@ -855,7 +855,8 @@ cudaError_t launch_score(const Ctx& c, const SelectLayout& L, char* base, int BH
 
 // Pools Q (z = 0) and K (z = 1), scores, then selects.
 cudaError_t pool_and_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
-                            int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts) {
+                            int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts,
+                            cudaEvent_t pooled) {
   const SelectLayout L = select_layout(B, H, N, d, kBlock);
   char* base = static_cast<char*>(ws);
   double* qbar = reinterpret_cast<double*>(base + L.qbar);
@@ -879,6 +880,7 @@ cudaError_t pool_and_select(const Ctx& c, const void* q, const void* k, int B, i
                                                kn2);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (pooled != nullptr && (e = cudaEventRecord(pooled, c.stream)) != cudaSuccess) return e;
   e = d == 128 ? launch_score<128>(c, L, base, BH, nb) : launch_score<64>(c, L, base, BH, nb);
   if (e != cudaSuccess) return e;
   if (d == 128)
@@ -894,8 +896,9 @@ size_t select_ws_bytes(int B, int H, int N, int d, int block) {
 }
 
 cudaError_t launch_select(const Ctx& c, const void* q, const void* k, int B, int H, int N, int d,
-                          int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts) {
-  return pool_and_select(c, q, k, B, H, N, d, topk, idx, ws, lists, counts);
+                          int topk, int32_t* idx, void* ws, int32_t* lists, int32_t* counts,
+                          cudaEvent_t pooled) {
+  return pool_and_select(c, q, k, B, H, N, d, topk, idx, ws, lists, counts, pooled);
 }
 
 size_t pairs_ws_bytes(int B, int H, int N, int topk) {

@@ -813,14 +813,15 @@ cudaError_t launch_select_rows(const Ctx& c, const float* S, int nbs, const floa
   return cudaGetLastError();
 }
 
-// The row's scores per lane kept in registers (nb <= 32 VPL); 16 query blocks
-// (two per warp) per CTA.
+// The row's scores per lane kept in registers (nb <= 32 VPL); query blocks
+// per CTA: 8 (one per warp) for nb <= 512, 12 (two per warp, 192 threads)
+// up to 2048, 8 beyond.
 template <int D>
 cudaError_t dispatch_select(const Ctx& c, const float* S, int nbs, const float* qn2,
                             const float* kn2, const double* q64, const double* k64, int BH,
                             int nb, int topk, int32_t* idx, int32_t* lists, int32_t* counts) {
   if (nb <= 512)
-    return launch_select_rows<D, 16, 16>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
+    return launch_select_rows<D, 8, 16>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
                                          counts);
   if (nb <= 2048)
     return launch_select_rows<D, 12, 64>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,

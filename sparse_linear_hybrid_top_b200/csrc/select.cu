@@ -463,33 +463,18 @@ __global__ void __launch_bounds__(sel_threads<VPL>(), sel_min_blocks<VPL>()) sel
   unsigned* hist = scratch + warp * (256 + kCandMax * 3);
   double* cs = reinterpret_cast<double*>(hist + 256);
   int* cj = reinterpret_cast<int*>(cs + kCandMax);
-  // The row's scores in registers: column j = lane + 32 u (-inf past nb).
-  // With few per lane, the warp's next row is read while this one is
-  // processed.
-  constexpr bool kAhead = VPL <= 16;
-  auto load_row = [&](int r, float (&v)[VPL]) {
-    const float* srow = S + (bh * nb + i0 + r) * static_cast<long long>(nbs);
-#pragma unroll
-    for (int u = 0; u < VPL; ++u) {
-      const int j = lane + 32 * u;
-      v[u] = (r < rows && j < nb) ? __ldg(srow + j) : -INFINITY;
-    }
-  };
-  float ahead[kAhead ? VPL : 1];
-  if constexpr (kAhead) load_row(warp, ahead);
   for (int r = warp; r < RB; r += kWarps) {
     unsigned* kept = bits + r * nw;
     for (int w = lane; w < nw; w += 32) kept[w] = 0u;
     __syncwarp();
     if (r >= rows) continue;
+    // The row's scores in registers: column j = lane + 32 u (-inf past nb).
     const float* srow = S + (bh * nb + i0 + r) * static_cast<long long>(nbs);
     float vals[VPL];
-    if constexpr (kAhead) {
 #pragma unroll
-      for (int u = 0; u < VPL; ++u) vals[u] = ahead[u];
-      if (r + kWarps < rows) load_row(r + kWarps, ahead);
-    } else {
-      load_row(r, vals);
+    for (int u = 0; u < VPL; ++u) {
+      const int j = lane + 32 * u;
+      vals[u] = j < nb ? __ldg(srow + j) : -INFINITY;
     }
     // Bracket the k-th largest float32 score T: cnt(>= lo) >= topk > cnt(>= hi),
     // so lo <= T < hi, by bisection on the value until the bracket is
@@ -520,8 +505,10 @@ __global__ void __launch_bounds__(sel_threads<VPL>(), sel_min_blocks<VPL>()) sel
     if (!wide && (c_hi = count_ge(mx)) < topk) {
       float lo = mn, hi = mx;
       int c_lo = nb;               // cnt(>= lo) >= topk > cnt(>= hi) = c_hi
-      for (int it = 0; it < 64 && static_cast<double>(hi) - lo > 0.5 * E && c_lo - c_hi > 8;
-           ++it) {
+      // The stopping width in float32 (any bracket is sound: it only sets how
+      // many candidates the band holds).
+      const float half_e = static_cast<float>(0.5 * E);
+      for (int it = 0; it < 64 && hi - lo > half_e && c_lo - c_hi > 8; ++it) {
         const float mid = lo + 0.5f * (hi - lo);
         if (!(mid > lo && mid < hi)) break;   // adjacent floats
         const int cm = count_ge(mid);
@@ -813,9 +800,9 @@ cudaError_t launch_select_rows(const Ctx& c, const float* S, int nbs, const floa
   return cudaGetLastError();
 }
 
-// The row's scores per lane kept in registers (nb <= 32 VPL); query blocks
-// per CTA: 8 (one per warp) for nb <= 512, 12 (two per warp, 192 threads)
-// up to 2048, 8 beyond.
+// The row's scores per lane kept in registers (nb <= 32 VPL); one query
+// block per warp: 8 per CTA (256 threads), or 6 (192 threads, two CTAs per
+// SM) for 512 < nb <= 2048.
 template <int D>
 cudaError_t dispatch_select(const Ctx& c, const float* S, int nbs, const float* qn2,
                             const float* kn2, const double* q64, const double* k64, int BH,
@@ -824,7 +811,7 @@ cudaError_t dispatch_select(const Ctx& c, const float* S, int nbs, const float* 
     return launch_select_rows<D, 8, 16>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
                                          counts);
   if (nb <= 2048)
-    return launch_select_rows<D, 12, 64>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
+    return launch_select_rows<D, 6, 64>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
                                          counts);
   return launch_select_rows<D, 8, 128>(c, S, nbs, qn2, kn2, q64, k64, BH, nb, topk, idx, lists,
                                         counts);

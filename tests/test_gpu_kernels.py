@@ -78,6 +78,24 @@ def test_select_blocks(salad, w):
     salad.check_error()
 
 
+# Rows longer than 2048 key blocks (128 scores per lane, 8 query blocks per
+# CTA): 2091 full blocks and a ragged one of 51 rows, one head of d = 64,
+# 10% kept.
+LONG_ROWS = Workload(name="long_rows", B=1, H=1, d=64, F=5, Hh=105, Wh=255, D=64, mode="topk",
+                     topk=210, lowrank_scale=0.5, seeds=(14,))      # N = 133875, nb = 2092
+
+
+def test_select_blocks_long_rows(salad):
+    w = LONG_ROWS
+    assert w.nb > 2048
+    inp = generate(w)
+    dev = device_inputs(inp)
+    idx = salad.select_blocks(dev["q"], dev["k"], w.topk)
+    torch.cuda.synchronize()
+    _check_selection(idx, to64(inp["q"]), to64(inp["k"]), w.block, w.topk)
+    salad.check_error()
+
+
 def test_select_all_blocks_and_ties(salad):
     # topk = nb keeps everything; equal scores (all-zero Q) keep the lowest
     # indices -- including the -0.0 / +0.0 mix a zero query produces.

@@ -402,7 +402,10 @@ class ForwardPlan:
     """Arguments and workspace of repeated salad_forward calls on fixed buffers.
 
     The plan owns its workspace (a torch uint8 tensor) and the packed argument
-    struct; ``run()`` enqueues the whole layer on the given stream.
+    struct; ``run()`` enqueues the whole layer on the given stream.  The
+    keyword arguments mirror ``salad_forward_args`` (include/salad.h), e.g.
+    ``regroup_in_load=True`` regroups the ST-SWA heads inside the attention's
+    loads instead of copying them (no copy workspace; slower on a B200).
     """
 
     def __init__(self, q, k, v, x, w_gate, w_lin, *, mode: str = "topk", topk: int = 0,
